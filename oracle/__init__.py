@@ -1,0 +1,25 @@
+"""CPU oracle for paged attention over a block-paged KV pool.
+
+TEST INFRASTRUCTURE ONLY.  This package is the plain, slow, obviously correct
+definition of what the CUDA library computes, in NumPy float64.  Only the tests,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference`` legs
+of ``bench.py`` may import it.  It shares no code with the CUDA path and imports
+nothing from it; the only thing both sides share is the seeded input generator
+in ``workloads``.
+
+Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
+invariants the pages state, a brute-force scalar implementation and the pages'
+own worked numbers; see each docstring for the passage it follows.
+"""
+from .paged_attention import (  # noqa: F401
+    bf16_bits_to_f64,
+    f64_to_bf16_bits,
+    slot_of,
+    gather_kv,
+    attend,
+    decode,
+    chunked_prefill,
+    reshape_and_cache,
+    copy_blocks,
+    CopyBlocksError,
+)
