@@ -1,0 +1,90 @@
+"""ctypes view of ``libpa.so`` (declared in ``include/pa.h``).
+
+Only argument marshalling lives here; every step of the computation runs in the
+library's CUDA kernels.  Loading fails loudly when the library has not been
+built: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpa.so")
+
+PA_OK = 0
+PA_ERR_ARG = 1
+PA_ERR_SHAPE = 2
+PA_ERR_UNSUPPORTED = 3
+PA_ERR_WORKSPACE = 4
+PA_ERR_CUDA = 5
+
+PA_DEV_ERR_BLOCK_ID = 0x1
+PA_DEV_ERR_SLOT = 0x2
+PA_DEV_ERR_CONTEXT = 0x4
+PA_DEV_ERR_TIMEOUT = 0x8
+
+PA_KERNEL_AUTO = 0
+PA_KERNEL_SIMT = 1
+PA_KERNEL_TCGEN05 = 2
+
+# Every entry point of include/pa.h, with its ctypes signature.
+c_int, c_i32, c_i64, c_f32 = ctypes.c_int, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+c_vp, c_size = ctypes.c_void_p, ctypes.c_size_t
+
+
+class PoolDesc(ctypes.Structure):
+    _fields_ = [("num_blocks", c_i32), ("num_kv_heads", c_i32), ("block_size", c_i32),
+                ("head_dim", c_i32)]
+
+
+SIGNATURES = {
+    "pa_reshape_and_cache": (c_int, [c_vp, c_vp, c_i64, c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp]),
+    "pa_copy_blocks": (c_int, [c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp]),
+    "pa_decode_workspace_size": (c_size, [c_i32, c_i32, PoolDesc, c_i32]),
+    "pa_decode": (c_int, [c_vp, c_i64, c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp, c_i32, c_i32,
+                          c_f32, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "pa_decode_workspace_size_ex": (c_size, [c_i32, c_i32, PoolDesc, c_i32, c_i32]),
+    "pa_decode_ex": (c_int, [c_vp, c_i64, c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp, c_i32, c_i32,
+                             c_f32, c_vp, c_vp, c_vp, c_size, c_i32, c_i32, c_vp]),
+    "pa_chunked_prefill": (c_int, [c_vp, c_i64, c_vp, c_i32, c_i32, c_vp, c_vp, PoolDesc, c_vp,
+                                   c_i32, c_vp, c_i32, c_i32, c_f32, c_vp, c_vp, c_vp]),
+    "pa_gather_kv": (c_int, [c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp, c_vp, c_i32, c_i32, c_vp,
+                             c_vp, c_vp]),
+    "pa_get_device_error": (c_int, [ctypes.POINTER(ctypes.c_uint32), c_vp]),
+    "pa_status_string": (ctypes.c_char_p, [c_int]),
+    "pa_abi_version": (c_int, []),
+}
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libpa.so and attach the signatures.  Raises if it is missing."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m paged_kv_cache_454_b200.build` "
+            "(there is no non-CUDA fallback)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+class PaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = load().pa_status_string(status)
+        super().__init__(f"{fn} failed: {msg.decode() if msg else status}")
+
+
+def check(fn: str, status: int) -> None:
+    if status != PA_OK:
+        raise PaError(fn, status)

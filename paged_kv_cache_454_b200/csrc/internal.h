@@ -1,0 +1,117 @@
+// Host-side declarations shared by the translation units of libpa.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/pa.h"
+
+namespace pa {
+
+// Device address of the sticky error word of the current device (looked up
+// once per device with cudaGetSymbolAddress).  NULL if the lookup failed.
+unsigned int* device_error_word();
+
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms();
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-kernel, per-device launch facts: sets the dynamic shared-memory limit
+// once per device and caches the occupancy (resident CTAs per SM).
+struct KernelLaunchCache {
+  int per_sm[64] = {0};
+  int blocks_per_sm(const void* func, int threads, int smem_bytes);
+};
+
+// Host checks of a pool descriptor shared by every entry point.
+int check_pool(const pa_pool_desc& pool);
+
+// Launch status -> PA status.
+inline int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Decode: the work plan shared by the decode kernels and the merge kernel.
+// ---------------------------------------------------------------------------
+// The workspace holds, in order:
+//   header       int32[4]: total items, total partitions
+//   part_base    int32[num_seqs + 1]: exclusive prefix of partitions per sequence
+//   work list    int2[num_seqs * max_parts * Hkv]: (seq, kv_head << 16 | partition)
+//   partial out  float[num_seqs * max_parts * Hq * D]
+//   partial lse  float[num_seqs * max_parts * Hq]   (base-2 log-sum-exp)
+struct DecodeWorkspace {
+  int* header;
+  int* part_base;
+  int2* items;
+  float* part_o;
+  float* part_lse;
+};
+
+size_t decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                              int max_parts);
+DecodeWorkspace carve_decode_workspace(void* ws, int num_seqs, int num_q_heads,
+                                       int num_kv_heads, int head_dim, int max_parts);
+
+struct DecodeArgs {
+  const uint16_t* q;
+  int64_t q_stride;
+  const uint16_t* k_pool;
+  const uint16_t* v_pool;
+  pa_pool_desc pool;
+  const int32_t* block_tables;
+  int max_blocks;
+  const int32_t* context_lens;
+  int num_seqs;
+  int num_q_heads;
+  float scale;
+  uint16_t* out;
+  float* lse;
+  int partition_tokens;
+  int max_parts;
+  DecodeWorkspace ws;
+  unsigned int* err;
+  cudaStream_t stream;
+};
+
+// Kernel launchers (return PA_OK / PA_ERR_*).
+int launch_decode_plan(const DecodeArgs& a);
+int launch_decode_simt(const DecodeArgs& a);
+int launch_decode_tcgen05(const DecodeArgs& a);
+int launch_decode_merge(const DecodeArgs& a);
+
+// Default partition lengths (tokens) of the two decode kernels.
+constexpr int kSimtPartition = 512;
+constexpr int kTcPartition = 1024;
+
+struct PrefillArgs {
+  const uint16_t* q;
+  int64_t q_stride;
+  const int32_t* cu_q;
+  int total_q;
+  int max_q_len;
+  const uint16_t* k_pool;
+  const uint16_t* v_pool;
+  pa_pool_desc pool;
+  const int32_t* block_tables;
+  int max_blocks;
+  const int32_t* context_lens;
+  int num_seqs;
+  int num_q_heads;
+  float scale;
+  uint16_t* out;
+  float* lse;
+  unsigned int* err;
+  cudaStream_t stream;
+};
+
+int launch_prefill_simt(const PrefillArgs& a);
+int launch_prefill_tcgen05(const PrefillArgs& a);
+bool prefill_tcgen05_supported(const PrefillArgs& a);
+bool decode_tcgen05_supported(int head_dim, int group);
+
+}  // namespace pa

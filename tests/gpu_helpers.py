@@ -1,0 +1,164 @@
+"""Helpers for the GPU parity tests: move the seeded inputs to the device, run
+one batch step through the library, run the same step through the oracle, and
+compare.  The oracle always works on host copies of the inputs taken before any
+library call touched them."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from workloads import synth
+
+ATOL = 2e-3
+RTOL = 1e-2
+LSE_ATOL = 1e-3
+
+
+def torch():
+    import torch as t
+    return t
+
+
+def dev_bf16(bits):
+    t = torch()
+    return t.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(t.bfloat16)
+
+
+def dev_i32(a):
+    t = torch()
+    return t.from_numpy(np.ascontiguousarray(np.asarray(a, np.int32))).cuda()
+
+
+def dev_i64(a):
+    t = torch()
+    return t.from_numpy(np.ascontiguousarray(np.asarray(a, np.int64))).cuda()
+
+
+def host_bits(x) -> np.ndarray:
+    t = torch()
+    return x.contiguous().view(t.int16).cpu().numpy().view(np.uint16)
+
+
+def host_f64(x) -> np.ndarray:
+    return x.float().cpu().numpy().astype(np.float64)
+
+
+def assert_close(got, want, atol=ATOL, rtol=RTOL, what=""):
+    """Element passes if |got - want| <= atol or <= rtol * |want|."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    diff = np.abs(got - want)
+    ok = (diff <= atol) | (diff <= rtol * np.abs(want))
+    if not ok.all():
+        bad = np.argwhere(~ok)
+        i = tuple(bad[0])
+        big = np.abs(want) > atol
+        rel = (diff[big] / np.abs(want[big])).max() if big.any() else 0.0
+        raise AssertionError(
+            f"{what}: {len(bad)} of {ok.size} elements out of tolerance; first at {i}: "
+            f"got {got[i]!r} want {want[i]!r}; max abs {diff.max():.3e}, max rel {rel:.3e}")
+    return float(diff.max())
+
+
+def assert_lse_close(got, want, what=""):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    inf = np.isinf(want)
+    assert np.array_equal(np.isinf(got), inf), f"{what}: -inf pattern differs"
+    if (~inf).any():
+        d = np.abs(got[~inf] - want[~inf]).max()
+        assert d <= LSE_ATOL, f"{what}: lse max abs diff {d:.3e}"
+
+
+# ----------------------------------------------------------------------------
+# One batch step
+# ----------------------------------------------------------------------------
+class Step:
+    """Device copies of a step's inputs plus the host copies the oracle uses."""
+
+    def __init__(self, layout: synth.Layout, host: dict):
+        t = torch()
+        self.layout = layout
+        self.host = host  # bf16 bit patterns (NumPy) as generated
+        self.k_pool = dev_bf16(host["k_pool"])
+        self.v_pool = dev_bf16(host["v_pool"])
+        self.q = dev_bf16(host["q"])
+        self.key = dev_bf16(host["key"])
+        self.value = dev_bf16(host["value"])
+        self.slot_mapping = dev_i64(layout.slot_mapping())
+        self.tables = dev_i32(layout.block_tables)
+        self.lens = dev_i32(layout.context_lens)
+        self.device = t.device("cuda")
+
+    @classmethod
+    def from_host(cls, layout, seed=None, poison=True):
+        return cls(layout, synth.fill_host(layout, seed=seed, poison=poison))
+
+    def rows_tensor(self, rows):
+        return torch().as_tensor(np.asarray(rows, np.int64), device="cuda")
+
+    def run_gpu(self, kernel=0, partition=0, want_lse=True):
+        """copy_blocks -> reshape_and_cache -> decode (decode rows) and chunked
+        prefill (prefill rows).  Returns dict of outputs keyed 'decode'/'prefill'."""
+        import paged_kv_cache_454_b200 as pa
+        lay = self.layout
+        res = {}
+        if lay.copy_pairs.size:
+            pa.pa_copy_blocks(self.k_pool, self.v_pool, lay.copy_pairs)
+        pa.pa_reshape_and_cache(self.key, self.value, self.k_pool, self.v_pool, self.slot_mapping)
+        dec = lay.decode_rows()
+        if len(dec):
+            r = self.rows_tensor(dec)
+            qi = self.rows_tensor(synth.token_rows(lay, dec))
+            out, lse = pa.pa_decode(self.q.index_select(0, qi), self.k_pool, self.v_pool,
+                                    self.tables.index_select(0, r).contiguous(),
+                                    self.lens.index_select(0, r).contiguous(), lay.scale,
+                                    kernel=kernel, partition_tokens=partition, want_lse=want_lse)
+            res["decode"] = (out, lse)
+        pf = lay.prefill_rows()
+        if len(pf):
+            r = self.rows_tensor(pf)
+            qi = self.rows_tensor(synth.token_rows(lay, pf))
+            cu = dev_i32(lay.cu_q_lens(pf))
+            out, lse = pa.pa_chunked_prefill(self.q.index_select(0, qi), cu,
+                                             int(lay.q_lens[pf].max()), self.k_pool, self.v_pool,
+                                             self.tables.index_select(0, r).contiguous(),
+                                             self.lens.index_select(0, r).contiguous(), lay.scale,
+                                             want_lse=want_lse)
+            res["prefill"] = (out, lse)
+        torch().cuda.synchronize()
+        return res
+
+    def run_oracle(self):
+        lay = self.layout
+        h = self.host
+        kp, vp = h["k_pool"], h["v_pool"]
+        if lay.copy_pairs.size:
+            kp, vp = oracle.copy_blocks(kp, vp, lay.copy_pairs)
+        kp, vp = oracle.reshape_and_cache(kp, vp, h["key"], h["value"], lay.slot_mapping())
+        res = {"pools": (kp, vp)}
+        dec = lay.decode_rows()
+        if len(dec):
+            qi = synth.token_rows(lay, dec)
+            res["decode"] = oracle.decode(h["q"][qi], kp, vp, lay.block_tables[dec],
+                                          lay.context_lens[dec], lay.scale)
+        pf = lay.prefill_rows()
+        if len(pf):
+            qi = synth.token_rows(lay, pf)
+            res["prefill"] = oracle.chunked_prefill(h["q"][qi], lay.cu_q_lens(pf), kp, vp,
+                                                    lay.block_tables[pf], lay.context_lens[pf],
+                                                    lay.scale)
+        return res
+
+
+def compare_step(gpu: dict, ref: dict, what=""):
+    worst = 0.0
+    for key in ("decode", "prefill"):
+        if key in ref:
+            out, lse = gpu[key]
+            worst = max(worst, assert_close(host_f64(out), ref[key][0], what=f"{what} {key} out"))
+            if lse is not None:
+                assert_lse_close(lse.cpu().numpy(), ref[key][1], what=f"{what} {key} lse")
+    return worst

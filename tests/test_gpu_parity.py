@@ -1,0 +1,276 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on seeded
+inputs at sizes the oracle finishes in seconds: several 128-token tiles, several
+split-context partitions, ragged tails, every poison of the batch builder.
+
+Bit-exact: cache writes, block copies, gathers.  Attention outputs: each element
+within 2e-3 absolute or 1e-2 relative of the fp64 oracle (bf16 inputs, fp32
+accumulation, bf16 output); log-sum-exp within 1e-3.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from workloads import synth
+
+import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+def pa():
+    import paged_kv_cache_454_b200 as m
+    return m
+
+
+# ----------------------------------------------------------------------------
+# Layouts (small enough for the oracle; big enough for tiles, splits, tails)
+# ----------------------------------------------------------------------------
+def lay_mha128():
+    return synth.build_layout("mha128", 101, [1, 15, 16, 17, 700, 2049], num_q_heads=4,
+                              num_kv_heads=4, head_dim=128)
+
+
+def lay_gqa8():
+    return synth.build_layout("gqa8", 102, [1, 130, 1025, 3000, 4100], num_q_heads=16,
+                              num_kv_heads=2, head_dim=128)
+
+
+def lay_gqa5():
+    return synth.build_layout("gqa5", 103, [33, 600, 1500, 2222], num_q_heads=10, num_kv_heads=2,
+                              head_dim=128)
+
+
+def lay_gqa4_d64():
+    return synth.build_layout("gqa4d64", 104, [5, 300, 999], num_q_heads=8, num_kv_heads=2,
+                              head_dim=64)
+
+
+def lay_g16():
+    return synth.build_layout("g16", 105, [64, 777], num_q_heads=32, num_kv_heads=2,
+                              head_dim=128)
+
+
+def lay_shared():
+    lay = synth.llama13b_sampling(seed=106, groups=3, samples=4, prefix=512, max_suffix=300)
+    lay.num_q_heads = lay.num_kv_heads = 4
+    return lay
+
+
+def lay_mixed(hq=10, hkv=2, d=128):
+    # prefill chunks: fresh prompt, short cache, long cache with a ragged chunk;
+    # plus two decode sequences
+    cached = [0, 100, 1000]
+    chunk = [37, 128, 300]
+    lens = [c + n for c, n in zip(cached, chunk)] + [513, 70]
+    return synth.build_layout("mixed", 107, lens, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
+                              q_lens=chunk + [1, 1], is_prefill=[True] * 3 + [False] * 2)
+
+
+DECODE_LAYOUTS = {
+    "tiny": synth.tiny,
+    "mha128": lay_mha128,
+    "gqa8": lay_gqa8,
+    "gqa5": lay_gqa5,
+    "gqa4_d64": lay_gqa4_d64,
+    "g16": lay_g16,
+    "shared_prefix": lay_shared,
+}
+
+
+# ----------------------------------------------------------------------------
+# Bit-exact data movement
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("make", [synth.tiny, lay_mha128, lay_shared, lambda: lay_mixed()],
+                         ids=["tiny", "mha128", "shared", "mixed"])
+def test_reshape_and_cache_and_copy_blocks_bit_exact(make):
+    lay = make()
+    st = H.Step.from_host(lay)
+    if lay.copy_pairs.size:
+        pa().pa_copy_blocks(st.k_pool, st.v_pool, lay.copy_pairs)
+    pa().pa_reshape_and_cache(st.key, st.value, st.k_pool, st.v_pool, st.slot_mapping)
+    ref = st.run_oracle()["pools"]
+    assert np.array_equal(H.host_bits(st.k_pool), ref[0])
+    assert np.array_equal(H.host_bits(st.v_pool), ref[1])
+    assert pa().pa_get_device_error() == 0
+
+
+def test_copy_blocks_many_pairs_bit_exact():
+    # more pairs than one launch carries (480), on D = 64 pools
+    rng = np.random.default_rng(7)
+    nb = 1200
+    kp = synth.normal_bf16(rng, (nb, 2, 16, 64))
+    vp = synth.normal_bf16(rng, (nb, 2, 16, 64))
+    perm = rng.permutation(nb)
+    pairs = np.stack([perm[:500], perm[500:1000]], axis=1)
+    k, v = H.dev_bf16(kp), H.dev_bf16(vp)
+    pa().pa_copy_blocks(k, v, pairs)
+    rk, rv = oracle.copy_blocks(kp, vp, pairs)
+    assert np.array_equal(H.host_bits(k), rk) and np.array_equal(H.host_bits(v), rv)
+
+
+def test_reshape_and_cache_strided_and_padding():
+    lay = lay_mha128()
+    h = synth.fill_host(lay)
+    T, hkv, d = h["key"].shape
+    # key/value as views into a wider [T, 3*Hkv, D] buffer (a fused projection)
+    wide = np.zeros((T, 3 * hkv, d), np.uint16)
+    wide[:, :hkv] = h["key"]
+    wide[:, hkv:2 * hkv] = h["value"]
+    wd = H.dev_bf16(wide)
+    sm = lay.slot_mapping().copy()
+    sm[2] = -1  # padding token
+    kp, vp = H.dev_bf16(h["k_pool"]), H.dev_bf16(h["v_pool"])
+    pa().pa_reshape_and_cache(wd[:, :hkv], wd[:, hkv:2 * hkv], kp, vp, H.dev_i64(sm))
+    rk, rv = oracle.reshape_and_cache(h["k_pool"], h["v_pool"], h["key"], h["value"], sm)
+    assert np.array_equal(H.host_bits(kp), rk) and np.array_equal(H.host_bits(vp), rv)
+
+
+@pytest.mark.parametrize("make", [synth.tiny, lay_gqa8, lay_shared], ids=["tiny", "gqa8", "shared"])
+def test_gather_kv_bit_exact(make):
+    lay = make()
+    st = H.Step.from_host(lay)
+    ref_pools = st.run_oracle()["pools"]
+    if lay.copy_pairs.size:
+        pa().pa_copy_blocks(st.k_pool, st.v_pool, lay.copy_pairs)
+    pa().pa_reshape_and_cache(st.key, st.value, st.k_pool, st.v_pool, st.slot_mapping)
+    cu = np.concatenate([[0], np.cumsum(lay.context_lens)]).astype(np.int32)
+    k, v = pa().pa_gather_kv(st.k_pool, st.v_pool, st.tables, st.lens, H.dev_i32(cu),
+                             int(lay.context_lens.max()), int(cu[-1]))
+    kb, vb = H.host_bits(k), H.host_bits(v)
+    for s in range(lay.num_seqs):
+        K, V = oracle.gather_kv(ref_pools[0], ref_pools[1], lay.block_tables[s],
+                                int(lay.context_lens[s]))
+        assert np.array_equal(kb[cu[s]:cu[s + 1]], K.transpose(1, 0, 2))
+        assert np.array_equal(vb[cu[s]:cu[s + 1]], V.transpose(1, 0, 2))
+
+
+# ----------------------------------------------------------------------------
+# Decode
+# ----------------------------------------------------------------------------
+_oracle_cache = {}
+
+
+def _step_and_ref(name):
+    if name not in _oracle_cache:
+        lay = DECODE_LAYOUTS[name]()
+        st = H.Step.from_host(lay)
+        _oracle_cache[name] = (lay, st.host, st.run_oracle())
+    lay, host, ref = _oracle_cache[name]
+    return H.Step(lay, host), ref
+
+
+@pytest.mark.parametrize("name", list(DECODE_LAYOUTS))
+@pytest.mark.parametrize("partition", [0, 128, 512, 1 << 20])
+def test_decode_simt(name, partition):
+    st, ref = _step_and_ref(name)
+    got = st.run_gpu(kernel=pa().PA_KERNEL_SIMT, partition=partition)
+    H.compare_step(got, ref, what=f"{name} simt p={partition}")
+    assert pa().pa_get_device_error() == 0
+
+
+@pytest.mark.parametrize("name", ["gqa8", "gqa5", "g16", "shared_prefix", "mha128"])
+@pytest.mark.parametrize("partition", [0, 128, 1024, 1 << 20])
+def test_decode_tcgen05(name, partition):
+    st, ref = _step_and_ref(name)
+    lay = st.layout
+    from paged_kv_cache_454_b200 import _abi
+    try:
+        got = st.run_gpu(kernel=pa().PA_KERNEL_TCGEN05, partition=partition)
+    except pa().PaError as e:
+        if e.status == _abi.PA_ERR_UNSUPPORTED:
+            pytest.skip(f"tcgen05 decode not built for D={lay.head_dim}, G={lay.group_size}")
+        raise
+    H.compare_step(got, ref, what=f"{name} tcgen05 p={partition}")
+    assert pa().pa_get_device_error() == 0
+
+
+def test_decode_default_kernel_choice():
+    st, ref = _step_and_ref("gqa8")
+    H.compare_step(st.run_gpu(), ref, what="gqa8 auto")
+
+
+# ----------------------------------------------------------------------------
+# Chunked prefill
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("hq,hkv,d", [(10, 2, 128), (16, 2, 128), (4, 4, 128), (8, 2, 64)],
+                         ids=["g5", "g8", "mha", "g4_d64"])
+def test_chunked_prefill(hq, hkv, d):
+    lay = lay_mixed(hq, hkv, d)
+    st = H.Step.from_host(lay)
+    ref = st.run_oracle()
+    got = st.run_gpu()
+    H.compare_step(got, ref, what=f"mixed {hq}/{hkv}/{d}")
+    assert pa().pa_get_device_error() == 0
+
+
+def test_prefill_of_twelve_tokens_in_chunks_of_four_equals_one_chunk():
+    # the pages' example (budget 6, 12-token prompt, 4 tokens a round), run as
+    # three chunked-prefill calls against one 12-token call
+    lay = synth.build_layout("p12", 108, [12], num_q_heads=8, num_kv_heads=2, head_dim=128,
+                             q_lens=[12], is_prefill=[True])
+    st = H.Step.from_host(lay)
+    ref = st.run_oracle()
+    pa().pa_reshape_and_cache(st.key, st.value, st.k_pool, st.v_pool, st.slot_mapping)
+    whole, _ = pa().pa_chunked_prefill(st.q, H.dev_i32([0, 12]), 12, st.k_pool, st.v_pool,
+                                       st.tables, st.lens, lay.scale)
+    parts = []
+    for s, e, _ in synth.chunk_schedule(12, 4, 6):
+        o, _ = pa().pa_chunked_prefill(st.q[s:e].contiguous(), H.dev_i32([0, e - s]), e - s,
+                                       st.k_pool, st.v_pool, st.tables, H.dev_i32([e]), lay.scale)
+        parts.append(H.host_f64(o))
+    H.assert_close(np.concatenate(parts), ref["prefill"][0], what="chunks of 4")
+    H.assert_close(H.host_f64(whole), ref["prefill"][0], what="one chunk")
+
+
+# ----------------------------------------------------------------------------
+# Edge cases and device-side checks
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_empty_and_single_token_contexts(kernel):
+    lay = synth.build_layout("edge", 109, [0, 1, 2], num_q_heads=8, num_kv_heads=1, head_dim=128,
+                             num_blocks=4)
+    lay.q_lens = np.array([0, 1, 1], np.int32)
+    st = H.Step.from_host(lay)
+    pa().pa_reshape_and_cache(st.key, st.value, st.k_pool, st.v_pool, st.slot_mapping)
+    try:
+        out, lse = pa().pa_decode(st.q[[0, 0, 1]].contiguous(), st.k_pool, st.v_pool, st.tables,
+                                  st.lens, lay.scale, kernel=kernel, want_lse=True)
+    except pa().PaError:
+        pytest.skip("kernel not built for this shape")
+    o = H.host_f64(out)
+    assert np.all(o[0] == 0) and np.all(np.isneginf(lse[0].cpu().numpy()))
+    # one token: the output is that token's value, exactly
+    v0 = oracle.bf16_bits_to_f64(st.host["value"][0])
+    assert np.array_equal(o[1], np.broadcast_to(v0, o[1].shape))
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_bad_block_id_is_flagged_not_read(kernel):
+    lay = lay_gqa8()
+    st = H.Step.from_host(lay)
+    pa().pa_reshape_and_cache(st.key, st.value, st.k_pool, st.v_pool, st.slot_mapping)
+    assert pa().pa_get_device_error() == 0
+    tab = lay.block_tables.copy()
+    tab[3, 5] = lay.num_blocks + 7  # needed by sequence 3 (3000 tokens)
+    try:
+        out, _ = pa().pa_decode(st.q, st.k_pool, st.v_pool, H.dev_i32(tab), st.lens, lay.scale,
+                                kernel=kernel)
+    except pa().PaError:
+        pytest.skip("kernel not built for this shape")
+    flags = pa().pa_get_device_error()
+    assert flags & pa().PA_DEV_ERR_BLOCK_ID
+    assert np.all(np.isfinite(H.host_f64(out)))
+    assert pa().pa_get_device_error() == 0  # cleared by the read
+
+
+def test_bad_slot_and_context_are_flagged():
+    lay = synth.tiny()
+    st = H.Step.from_host(lay)
+    sm = lay.slot_mapping().copy()
+    sm[0] = lay.num_blocks * 16 + 3
+    pa().pa_reshape_and_cache(st.key, st.value, st.k_pool, st.v_pool, H.dev_i64(sm))
+    assert pa().pa_get_device_error() & pa().PA_DEV_ERR_SLOT
+    lens = lay.context_lens.copy()
+    lens[1] = lay.max_blocks * 16 + 1
+    pa().pa_decode(st.q, st.k_pool, st.v_pool, st.tables, H.dev_i32(lens), lay.scale)
+    assert pa().pa_get_device_error() & pa().PA_DEV_ERR_CONTEXT

@@ -44,7 +44,7 @@ __all__ = [
     "normal_bf16", "build_layout", "tiny", "llama7b_decode", "llama13b_sampling",
     "gqa70b_long", "mixed_qwen32b", "CONFIGS", "fill_host", "fill_device",
     "chunk_schedule", "decode_kv_bytes", "kv_cache_bytes_per_layer",
-    "prefill_flops", "unique_kv_bytes",
+    "prefill_flops", "unique_kv_bytes", "subset", "token_rows",
 ]
 
 
@@ -471,3 +471,49 @@ def prefill_flops(layout: Layout, rows=None) -> int:
         keys = n * c + n * (n + 1) // 2
         total += 4 * D * Hq * keys
     return int(total)
+
+
+# ----------------------------------------------------------------------------
+# Restriction of a batch to some sequences (for checking sampled outputs)
+# ----------------------------------------------------------------------------
+def subset(layout: Layout, rows) -> tuple[Layout, np.ndarray]:
+    """The batch restricted to ``rows``, over a compact pool holding only the
+    blocks those rows read or write (plus the sources of the copy-on-write
+    pairs whose destinations they use).
+
+    Returns ``(sub_layout, blocks)`` where ``blocks[i]`` is the original
+    physical id of the sub-layout's block ``i``; the caller gathers
+    ``pool[blocks]`` to build the compact pools.  Token order of the new tokens
+    follows ``rows``.
+    """
+    rows = [int(r) for r in rows]
+    need = []
+    for s in rows:
+        need.extend(int(b) for b in layout.block_tables[s, : layout.blocks_used(s)])
+    used = set(need)
+    pairs = [(int(a), int(b)) for a, b in layout.copy_pairs if int(b) in used]
+    need.extend(a for a, _ in pairs)
+    blocks = np.asarray(sorted(set(need)), dtype=np.int64)
+    remap = {int(b): i for i, b in enumerate(blocks)}
+    mb = max([1] + [layout.blocks_used(s) for s in rows])
+    tables = np.full((len(rows), mb), INT32_MAX, dtype=np.int32)
+    for i, s in enumerate(rows):
+        for j in range(layout.blocks_used(s)):
+            tables[i, j] = remap[int(layout.block_tables[s, j])]
+    ref = np.zeros(len(blocks), np.int32)
+    for i in range(len(rows)):
+        for j in range(-(-int(layout.context_lens[rows[i]]) // layout.block_size)):
+            ref[tables[i, j]] += 1
+    cp = np.asarray([(remap[a], remap[b]) for a, b in pairs], np.int64).reshape(-1, 2)
+    sub = Layout(layout.name + "-subset", layout.seed, layout.num_q_heads, layout.num_kv_heads,
+                 layout.head_dim, layout.block_size, len(blocks),
+                 layout.context_lens[rows].copy(), tables, layout.q_lens[rows].copy(),
+                 layout.is_prefill[rows].copy(), copy_pairs=cp, ref_counts=ref)
+    return sub, blocks
+
+
+def token_rows(layout: Layout, rows) -> np.ndarray:
+    """Indices, into the step's packed new-token arrays (q, key, value), of the
+    new tokens of ``rows`` in ``rows`` order."""
+    starts = np.concatenate([[0], np.cumsum(layout.q_lens)]).astype(np.int64)
+    return np.concatenate([np.arange(starts[s], starts[s + 1]) for s in rows]).astype(np.int64)
