@@ -175,6 +175,36 @@ PA_API int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, con
                  int32_t partition_tokens, int32_t kernel, void* stream);
 
 /*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call: it only changes where the
+ * split-context scratch comes from.  A caller that gives all free HBM to its KV
+ * pool at start-up, or that runs inside a host framework whose op interface
+ * passes no workspace, cannot provide the workspace pa_decode needs.  This call
+ * takes the same arguments minus the workspace and uses a scratch array of
+ * PA_NOALLOC_SCRATCH_BYTES compiled into the library instead; it allocates
+ * nothing.
+ *
+ *   - Every GPU that loads the library holds the array until the process exits.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture on the device.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents; nothing in it needs to start at zero.  Calls whose kernels
+ *     overlap on the GPU (e.g. on two streams) race on it: do not issue them.
+ *   - A batch whose workspace (pa_decode_workspace_size for the same sizes)
+ *     exceeds PA_NOALLOC_SCRATCH_BYTES returns PA_ERR_WORKSPACE and launches
+ *     nothing.  Other errors as for pa_decode.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+PA_API int pa_decode_noalloc(const void* q, int64_t q_stride, const void* k_pool,
+                             const void* v_pool, pa_pool_desc pool, const int32_t* block_tables,
+                             int32_t max_blocks_per_seq, const int32_t* context_lens,
+                             int32_t num_seqs, int32_t num_q_heads, float scale, void* out,
+                             float* lse, void* stream);
+
+/*
  * pa_chunked_prefill -- each sequence's new chunk of tokens attends causally to
  * its cached context plus the chunk itself.
  *

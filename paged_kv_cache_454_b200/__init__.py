@@ -18,6 +18,7 @@ from ._abi import (PA_DEV_ERR_BLOCK_ID, PA_DEV_ERR_CONTEXT, PA_DEV_ERR_SLOT,  # 
 
 __all__ = [
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
+    "pa_decode_noalloc",
     "pa_chunked_prefill", "pa_gather_kv", "pa_get_device_error", "pool_desc", "lib",
     "PaError", "PA_KERNEL_AUTO", "PA_KERNEL_SIMT", "PA_KERNEL_TCGEN05",
 ]
@@ -134,6 +135,34 @@ def pa_decode(q, k_pool, v_pool, block_tables, context_lens, scale, out=None, ls
         _ptr(q), qs, _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(block_tables), mb,
         _ptr(context_lens), S, hq, float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel(), int(partition_tokens), int(kernel), _stream(stream)))
+    return out, lse
+
+
+def pa_decode_noalloc(q, k_pool, v_pool, block_tables, context_lens, scale, out=None, lse=None,
+                      stream=None, want_lse=False):
+    """``pa_decode`` for callers that cannot allocate device memory: the split
+    scratch comes from a fixed array inside the library (``_abi.PA_NOALLOC_SCRATCH_BYTES``
+    per device, shared by all calls on the device, so calls must not overlap on
+    the GPU).  This wrapper itself allocates ``out``/``lse`` only when they are
+    not given."""
+    torch = _torch()
+    _check_pools(k_pool, v_pool)
+    _need_cuda("q", q, torch.bfloat16, contiguous=False)
+    _need_cuda("block_tables", block_tables, torch.int32)
+    _need_cuda("context_lens", context_lens, torch.int32)
+    S, hq, d = q.shape
+    qs = _row_stride("q", q)
+    if out is None:
+        out = torch.empty((S, hq, d), dtype=torch.bfloat16, device=q.device)
+    _need_cuda("out", out, torch.bfloat16)
+    if lse is None and want_lse:
+        lse = torch.empty((S, hq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need_cuda("lse", lse, torch.float32)
+    _abi.check("pa_decode_noalloc", lib().pa_decode_noalloc(
+        _ptr(q), qs, _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), S, hq, float(scale), _ptr(out), _ptr(lse),
+        _stream(stream)))
     return out, lse
 
 

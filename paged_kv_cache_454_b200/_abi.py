@@ -28,6 +28,8 @@ PA_KERNEL_AUTO = 0
 PA_KERNEL_SIMT = 1
 PA_KERNEL_TCGEN05 = 2
 
+PA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
 # Every entry point of include/pa.h, with its ctypes signature.
 c_int, c_i32, c_i64, c_f32 = ctypes.c_int, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
 c_vp, c_size = ctypes.c_void_p, ctypes.c_size_t
@@ -47,6 +49,8 @@ SIGNATURES = {
     "pa_decode_workspace_size_ex": (c_size, [c_i32, c_i32, PoolDesc, c_i32, c_i32]),
     "pa_decode_ex": (c_int, [c_vp, c_i64, c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp, c_i32, c_i32,
                              c_f32, c_vp, c_vp, c_vp, c_size, c_i32, c_i32, c_vp]),
+    "pa_decode_noalloc": (c_int, [c_vp, c_i64, c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp, c_i32,
+                                  c_i32, c_f32, c_vp, c_vp, c_vp]),
     "pa_chunked_prefill": (c_int, [c_vp, c_i64, c_vp, c_i32, c_i32, c_vp, c_vp, PoolDesc, c_vp,
                                    c_i32, c_vp, c_i32, c_i32, c_f32, c_vp, c_vp, c_vp]),
     "pa_gather_kv": (c_int, [c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp, c_vp, c_i32, c_i32, c_vp,
