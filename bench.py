@@ -103,11 +103,14 @@ class ClockSampler:
 # the batch step
 # ----------------------------------------------------------------------------
 class Workload:
-    def __init__(self, name, seed, device, kernel=0, partition=0):
+    def __init__(self, name, seed, device, kernel=0, partition=0, num_seqs=None):
         import torch
         self.torch = torch
         self.name = name
-        self.layout = synth.CONFIGS[name](seed=seed) if seed is not None else synth.CONFIGS[name]()
+        kw = {} if seed is None else {"seed": seed}
+        if num_seqs:
+            kw["batch"] = num_seqs  # a smaller batch of the same shape (profiling)
+        self.layout = synth.CONFIGS[name](**kw)
         lay = self.layout
         self.dev = device
         t = synth.fill_device(lay, device)
@@ -320,6 +323,8 @@ def main():
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="smaller batch of the same workload shape (profiling captures)")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
 
@@ -340,7 +345,8 @@ def main():
     peaks, peak_src = load_peaks()
 
     w = Workload(a.workload, None if rank == 0 else synth.CONFIGS[a.workload]().seed + 100 * rank,
-                 dev, kernel={"auto": 0, "simt": 1, "tcgen05": 2}[a.kernel], partition=a.partition)
+                 dev, kernel={"auto": 0, "simt": 1, "tcgen05": 2}[a.kernel], partition=a.partition,
+                 num_seqs=a.num_seqs or None)
     # host copies for the CPU baseline are taken before any kernel touches the pools
     cpu = None
     if rank == 0 and world == 1 and not a.skip_cpu_baseline:
@@ -412,7 +418,8 @@ def main():
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 K/V/q; shuffled block pool; no dataset)",
-        "config": {"workload": a.workload, "num_seqs": lay.num_seqs,
+        "config": {"workload": a.workload if not a.num_seqs else f"{a.workload} (batch {a.num_seqs})",
+                   "num_seqs": lay.num_seqs,
                    "decode_seqs": int(len(w.dec)), "prefill_tokens": int(lay.q_lens[w.pf].sum()) if len(w.pf) else 0,
                    "num_q_heads": lay.num_q_heads, "num_kv_heads": lay.num_kv_heads,
                    "head_dim": lay.head_dim, "block_size": lay.block_size,

@@ -80,6 +80,7 @@ size_t decode_workspace_bytes(int S, int Hq, int Hkv, int D, int max_parts) {
   const size_t slots = size_t(S) * size_t(max_parts);
   size_t b = align256(4 * sizeof(int));
   b += align256(sizeof(int) * (size_t(S) + 1));
+  b += align256(sizeof(int) * size_t(S) * size_t(Hkv));
   b += align256(sizeof(int2) * slots * size_t(Hkv));
   b += align256(sizeof(float) * slots * size_t(Hq) * size_t(D));
   b += align256(sizeof(float) * slots * size_t(Hq));
@@ -94,6 +95,8 @@ DecodeWorkspace carve_decode_workspace(void* ws, int S, int Hq, int Hkv, int D, 
   p += align256(4 * sizeof(int));
   w.part_base = reinterpret_cast<int*>(p);
   p += align256(sizeof(int) * (size_t(S) + 1));
+  w.merge_cnt = reinterpret_cast<int*>(p);
+  p += align256(sizeof(int) * size_t(S) * size_t(Hkv));
   w.items = reinterpret_cast<int2*>(p);
   p += align256(sizeof(int2) * slots * size_t(Hkv));
   w.part_o = reinterpret_cast<float*>(p);
@@ -160,6 +163,7 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
   if (group > 16) return PA_ERR_UNSUPPORTED;
   if (kernel < PA_KERNEL_AUTO || kernel > PA_KERNEL_TCGEN05) return PA_ERR_ARG;
   if (partition_tokens < 0 || (partition_tokens > 0 && partition_tokens % 128)) return PA_ERR_ARG;
+  if (partition_tokens > 0 && partition_tokens < 128) return PA_ERR_ARG;
   if (num_seqs == 0) return PA_OK;
   if (!q || !k_pool || !v_pool || !block_tables || !context_lens || !out) return PA_ERR_ARG;
   if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
@@ -169,7 +173,13 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
   const int kind = choose_kernel(kernel, pool.head_dim, group);
   if (kind == PA_KERNEL_TCGEN05 && !decode_tcgen05_supported(pool.head_dim, group))
     return PA_ERR_UNSUPPORTED;
-  const int part = partition_or_default(partition_tokens, kind);
+  int part = partition_or_default(partition_tokens, kind);
+  {
+    // a partition longer than any context the table can describe is one partition
+    const long long max_ctx = static_cast<long long>(max_blocks_per_seq) * pool.block_size;
+    const long long cap = ((max_ctx + 127) / 128) * 128;
+    if (part > cap) part = static_cast<int>(cap < 128 ? 128 : cap);
+  }
   const int max_parts = max_parts_for(max_blocks_per_seq, pool.block_size, part);
   const size_t need = decode_workspace_bytes(num_seqs, num_q_heads, pool.num_kv_heads,
                                              pool.head_dim, max_parts);
@@ -189,7 +199,13 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
   a.scale = scale;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
-  a.partition_tokens = part;
+  if (partition_tokens > 0) {
+    a.min_part = a.max_part = part;  // the caller fixed the length
+  } else {
+    a.min_part = part;
+    a.max_part = kind == PA_KERNEL_TCGEN05 ? kTcMaxPartition : part;
+  }
+  a.target_items = kTcItemsPerSm * num_sms();
   a.max_parts = max_parts;
   a.ws = carve_decode_workspace(workspace, num_seqs, num_q_heads, pool.num_kv_heads,
                                 pool.head_dim, max_parts);
@@ -199,7 +215,8 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
 
   st = launch_decode_plan(a);
   if (st != PA_OK) return st;
-  st = (kind == PA_KERNEL_TCGEN05) ? launch_decode_tcgen05(a) : launch_decode_simt(a);
+  if (kind == PA_KERNEL_TCGEN05) return launch_decode_tcgen05(a);
+  st = launch_decode_simt(a);
   if (st != PA_OK) return st;
   return launch_decode_merge(a);
 }

@@ -1,0 +1,163 @@
+// The decode work plan: one CTA turns context lengths into the list of
+// (sequence, KV head, partition) work items both decode kernels consume.
+//
+//  * Partition length: `min_part` tokens, or -- when the caller leaves the
+//    choice to the library -- the largest power-of-two multiple of it (up to
+//    `max_part`) that still leaves at least `target_items` items, so long
+//    contexts are split only as far as load balance needs.
+//  * Order: longest items first (all full partitions, then the tails by
+//    decreasing length, then empty contexts), so a kernel that hands items out
+//    dynamically schedules them longest-processing-time first.
+//  * It also clears the dynamic item counter and the per-(sequence, KV head)
+//    counters the tensor-core kernel uses to find the last partition to finish.
+#include "common.cuh"
+#include "internal.h"
+
+namespace pa {
+namespace {
+
+__device__ __forceinline__ int clamp_len(int L, int max_blocks, unsigned int* err) {
+  const int cap = max_blocks * 16;
+  if (L < 0 || L > cap) {
+    raise_error(err, PA_DEV_ERR_CONTEXT);
+    return L < 0 ? 0 : cap;
+  }
+  return L;
+}
+
+// Items are bucketed by their tile count n (128 tokens per tile): bucket 0
+// holds n >= 64, bucket 64 - n holds 1 <= n < 64, bucket 64 the empty items.
+constexpr int kMaxBuckets = 65;
+__device__ __forceinline__ int bucket_of(int ntiles) {
+  return ntiles == 0 ? 64 : (ntiles >= 64 ? 0 : 64 - ntiles);
+}
+
+__global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ context_lens,
+                                                           int S, int max_blocks, int hkv,
+                                                           int min_part, int max_part,
+                                                           int target_items, int* header,
+                                                           int* part_base, int2* items,
+                                                           int* merge_cnt, unsigned int* err) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  __shared__ int cand[4];
+  __shared__ int bucket[kMaxBuckets];
+  __shared__ int cursor[kMaxBuckets];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // ---- partition length ----
+  int ncand = 1;
+  while (ncand < 4 && (min_part << ncand) <= max_part) ++ncand;
+  if (tid < 4) cand[tid] = 0;
+  __syncthreads();
+  if (ncand > 1) {
+    int cnt[4] = {0, 0, 0, 0};
+    for (int s = tid; s < S; s += 1024) {
+      const int L = clamp_len(context_lens[s], max_blocks, nullptr);
+      for (int k = 0; k < ncand; ++k) {
+        const int pk = min_part << k;
+        const int n = (L + pk - 1) / pk;
+        cnt[k] += n < 1 ? 1 : n;
+      }
+    }
+    for (int k = 0; k < ncand; ++k) {
+      int v = cnt[k];
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) atomicAdd(&cand[k], v);
+    }
+  }
+  __syncthreads();
+  int part = min_part;
+  for (int k = ncand - 1; k > 0; --k)
+    if (static_cast<long long>(cand[k]) * hkv >= target_items) {
+      part = min_part << k;
+      break;
+    }
+  const int full_bucket = bucket_of(part / 128);
+
+  // ---- partitions per sequence and their exclusive prefix ----
+  if (tid == 0) carry = 0;
+  if (tid < kMaxBuckets) bucket[tid] = 0;
+  __syncthreads();
+  for (int base = 0; base < S; base += 1024) {
+    const int s = base + tid;
+    int np = 0;
+    if (s < S) {
+      const int L = clamp_len(context_lens[s], max_blocks, err);
+      np = (L + part - 1) / part;
+      if (np < 1) np = 1;
+      // bucket counts: full partitions, the tail, or an empty context
+      const int full = L / part, rem = L - full * part;
+      if (full) atomicAdd(&bucket[full_bucket], full * hkv);
+      if (rem) atomicAdd(&bucket[bucket_of((rem + 127) / 128)], hkv);
+      if (L == 0) atomicAdd(&bucket[bucket_of(0)], hkv);
+    }
+    int x = np;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_tot[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int incl = x + (warp > 0 ? warp_tot[warp - 1] : 0);
+    if (s < S) part_base[s] = carry + incl - np;
+    __syncthreads();
+    if (tid == 1023) carry += incl;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    part_base[S] = carry;
+    int acc = 0;
+    for (int b = 0; b < kMaxBuckets; ++b) {
+      cursor[b] = acc;
+      acc += bucket[b];
+    }
+    header[0] = carry * hkv;  // items
+    header[1] = carry;        // partitions
+    header[2] = 0;            // dynamic item counter
+    header[3] = part;         // partition length
+  }
+  __syncthreads();
+
+  // ---- the work list, longest items first ----
+  for (int s = tid; s < S; s += 1024) {
+    const int L = clamp_len(context_lens[s], max_blocks, nullptr);
+    const int full = L / part, rem = L - full * part;
+    if (full) {
+      int at = atomicAdd(&cursor[full_bucket], full * hkv);
+      for (int g = 0; g < hkv; ++g)
+        for (int q = 0; q < full; ++q) items[at++] = make_int2(s, (g << 16) | q);
+    }
+    if (rem) {
+      const int at = atomicAdd(&cursor[bucket_of((rem + 127) / 128)], hkv);
+      for (int g = 0; g < hkv; ++g) items[at + g] = make_int2(s, (g << 16) | full);
+    }
+    if (L == 0) {
+      const int at = atomicAdd(&cursor[bucket_of(0)], hkv);
+      for (int g = 0; g < hkv; ++g) items[at + g] = make_int2(s, g << 16);
+    }
+  }
+  for (int i = tid; i < S * hkv; i += 1024) merge_cnt[i] = 0;
+}
+
+}  // namespace
+
+int launch_decode_plan(const DecodeArgs& a) {
+  decode_plan_kernel<<<1, 1024, 0, a.stream>>>(
+      a.context_lens, a.num_seqs, a.max_blocks, a.pool.num_kv_heads, a.min_part, a.max_part,
+      a.target_items, a.ws.header, a.ws.part_base, a.ws.items, a.ws.merge_cnt, a.err);
+  return launch_status();
+}
+
+}  // namespace pa

@@ -25,7 +25,7 @@
 namespace pa {
 
 // ---------------------------------------------------------------------------
-// Plan: partitions per sequence, their prefix, and the flat work list.
+// Context lengths are clamped to the table width (the plan kernel flags it).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int clamp_context(int L, int max_blocks, unsigned int* err) {
   const int cap = max_blocks * 16;
@@ -34,62 +34,6 @@ __device__ __forceinline__ int clamp_context(int L, int max_blocks, unsigned int
     return L < 0 ? 0 : cap;
   }
   return L;
-}
-
-__device__ __forceinline__ int parts_of(int L, int part_tokens) {
-  const int n = (L + part_tokens - 1) / part_tokens;
-  return n < 1 ? 1 : n;
-}
-
-__global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ context_lens,
-                                                           int S, int max_blocks, int part_tokens,
-                                                           int hkv, int* header, int* part_base,
-                                                           int2* items, unsigned int* err) {
-  __shared__ int warp_tot[32];
-  __shared__ int carry;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) carry = 0;
-  __syncthreads();
-  for (int base = 0; base < S; base += 1024) {
-    const int s = base + tid;
-    int np = 0;
-    if (s < S) np = parts_of(clamp_context(context_lens[s], max_blocks, err), part_tokens);
-    int x = np;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_tot[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int w = warp_tot[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
-      }
-      warp_tot[lane] = w;  // inclusive over warps
-    }
-    __syncthreads();
-    const int incl = x + (warp > 0 ? warp_tot[warp - 1] : 0);
-    if (s < S) part_base[s] = carry + incl - np;
-    __syncthreads();
-    if (tid == 1023) carry += incl;
-    __syncthreads();
-  }
-  if (tid == 0) {
-    part_base[S] = carry;
-    header[0] = carry * hkv;  // items
-    header[1] = carry;        // partitions
-  }
-  __syncthreads();
-  for (int s = tid; s < S; s += 1024) {
-    const int np = part_base[s + 1] - part_base[s];
-    const int b = part_base[s] * hkv;
-    for (int g = 0; g < hkv; ++g)
-      for (int p = 0; p < np; ++p) items[b + g * np + p] = make_int2(s, (g << 16) | p);
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -135,7 +79,7 @@ struct Item {
   int pbase;  // part_base[seq]
 };
 
-__device__ __forceinline__ Item load_item(const SimtParams& p, int item) {
+__device__ __forceinline__ Item load_item(const SimtParams& p, int item, int part_tokens) {
   Item it;
   if (!p.prefill) {
     const int2 d = p.items[item];
@@ -144,8 +88,8 @@ __device__ __forceinline__ Item load_item(const SimtParams& p, int item) {
     it.g = d.y >> 16;
     it.part = d.y & 0xffff;
     const int L = clamp_context(p.context_lens[it.seq], p.max_blocks, nullptr);
-    it.tok0 = it.part * p.part_tokens;
-    it.tok1 = min(L, it.tok0 + p.part_tokens);
+    it.tok0 = it.part * part_tokens;
+    it.tok1 = min(L, it.tok0 + part_tokens);
     it.pbase = p.part_base[it.seq];
     it.npart = p.part_base[it.seq + 1] - it.pbase;
   } else {
@@ -209,6 +153,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const SimtParams p
   __syncthreads();
 
   const int total_items = p.prefill ? p.total_q * p.hkv : p.header[0];
+  const int part_tokens = p.prefill ? (1 << 30) : p.header[3];
   const int64_t head_stride = 16LL * D;  // elements per (block, head) page
 
   // ---- producer cursor (all lanes track it; lane 0 issues) ----
@@ -217,7 +162,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const SimtParams p
   Item l_it;
   int l_npages = 0;
   auto enter_item = [&](int item) {
-    l_it = load_item(p, item);
+    l_it = load_item(p, item, part_tokens);
     l_npages = (l_it.tok1 - l_it.tok0 + 15) >> 4;
     if (l_it.tok1 <= l_it.tok0) l_npages = 0;
   };
@@ -267,7 +212,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const SimtParams p
   const uint32_t ring_base = smem_u32(ring);
 
   for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
-    const Item it = load_item(p, item);
+    const Item it = load_item(p, item, part_tokens);
     const int npages = it.tok1 > it.tok0 ? (it.tok1 - it.tok0 + 15) >> 4 : 0;
 
     // q fragments of this lane, pre-scaled into the log2 domain
@@ -527,13 +472,6 @@ int launch_simt(const SimtParams& prm, int head_dim, int group, int64_t item_bou
 
 }  // namespace
 
-int launch_decode_plan(const DecodeArgs& a) {
-  decode_plan_kernel<<<1, 1024, 0, a.stream>>>(a.context_lens, a.num_seqs, a.max_blocks,
-                                               a.partition_tokens, a.pool.num_kv_heads,
-                                               a.ws.header, a.ws.part_base, a.ws.items, a.err);
-  return launch_status();
-}
-
 int launch_decode_merge(const DecodeArgs& a) {
   const int64_t n = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
   if (n > 0x7fffffff) return PA_ERR_UNSUPPORTED;
@@ -567,7 +505,7 @@ int launch_decode_simt(const DecodeArgs& a) {
   p.items = a.ws.items;
   p.part_o = a.ws.part_o;
   p.part_lse = a.ws.part_lse;
-  p.part_tokens = a.partition_tokens;
+  p.part_tokens = 0;  // read from the plan's header
   p.prefill = 0;
   p.err = a.err;
   const int64_t bound = static_cast<int64_t>(a.num_seqs) * a.max_parts * a.pool.num_kv_heads;

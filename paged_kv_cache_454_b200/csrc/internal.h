@@ -36,17 +36,23 @@ inline int launch_status() {
 }
 
 // ---------------------------------------------------------------------------
-// Decode: the work plan shared by the decode kernels and the merge kernel.
+// Decode: the work plan shared by the decode kernels and the merge.
 // ---------------------------------------------------------------------------
 // The workspace holds, in order:
-//   header       int32[4]: total items, total partitions
+//   header       int32[4]: total items, total partitions, dynamic item counter,
+//                partition length chosen by the plan
 //   part_base    int32[num_seqs + 1]: exclusive prefix of partitions per sequence
-//   work list    int2[num_seqs * max_parts * Hkv]: (seq, kv_head << 16 | partition)
+//   merge_cnt    int32[num_seqs * Hkv]: partitions finished per (sequence, KV head)
+//   work list    int2[num_seqs * max_parts * Hkv]: (seq, kv_head << 16 | partition),
+//                longest items first
 //   partial out  float[num_seqs * max_parts * Hq * D]
 //   partial lse  float[num_seqs * max_parts * Hq]   (base-2 log-sum-exp)
+// max_parts is the partition count of the longest possible context at the
+// shortest partition length the call may use.
 struct DecodeWorkspace {
   int* header;
   int* part_base;
+  int* merge_cnt;
   int2* items;
   float* part_o;
   float* part_lse;
@@ -71,8 +77,10 @@ struct DecodeArgs {
   float scale;
   uint16_t* out;
   float* lse;
-  int partition_tokens;
-  int max_parts;
+  int min_part;      // partition length bounds for the plan (tokens, multiples of 128)
+  int max_part;
+  int target_items;  // the plan lengthens partitions while at least this many items remain
+  int max_parts;     // workspace bound (partitions of the longest context at min_part)
   DecodeWorkspace ws;
   unsigned int* err;
   cudaStream_t stream;
@@ -81,12 +89,17 @@ struct DecodeArgs {
 // Kernel launchers (return PA_OK / PA_ERR_*).
 int launch_decode_plan(const DecodeArgs& a);
 int launch_decode_simt(const DecodeArgs& a);
-int launch_decode_tcgen05(const DecodeArgs& a);
+int launch_decode_tcgen05(const DecodeArgs& a);  // merges split partitions itself
 int launch_decode_merge(const DecodeArgs& a);
 
-// Default partition lengths (tokens) of the two decode kernels.
+// Partition lengths (tokens) of the two decode kernels: the CUDA-core kernel
+// uses a fixed length; the tensor-core kernel starts from kTcPartition and
+// lengthens partitions up to kTcMaxPartition while each SM keeps at least
+// kTcItemsPerSm items.
 constexpr int kSimtPartition = 512;
 constexpr int kTcPartition = 1024;
+constexpr int kTcMaxPartition = 8192;
+constexpr int kTcItemsPerSm = 16;
 
 struct PrefillArgs {
   const uint16_t* q;
