@@ -19,14 +19,16 @@
 //   warp 1      allocates 64 TMEM columns; one lane issues the MMAs and commits
 //               them to mbarriers (S of tile t before O of tile t-1, so the
 //               tensor core computes scores while the softmax warps work).
-//   warps 2-5   softmax and epilogue: thread r owns token r of S^T and output
-//               dimension r of O^T.  Online softmax in the log2 domain with one
-//               max exchange per tile; p goes to shared memory as bf16 in the
-//               operand layout of the second product; the tile's O^T is folded
-//               into registers (acc = acc * alpha + O).  At the end of an item
-//               they write the output, or the partition's partial result; the
-//               last partition of a (sequence, KV head) to finish merges all of
-//               them by log-sum-exp.
+//   warps 2-5   softmax: thread r owns token r of S^T and output dimension r of
+//               O^T.  Online softmax in the log2 domain with one max exchange
+//               per tile; p goes to shared memory as bf16 in the operand layout
+//               of the second product; the tile's O^T is folded into registers
+//               (acc = acc * alpha + O).  At the end of an item they hand the
+//               normalised result and its log-sum-exp to the epilogue through a
+//               shared-memory buffer and move on.
+//   warps 7-10  epilogue: write the output, or the partition's partial result;
+//               the last partition of a (sequence, KV head) to finish merges all
+//               of them by log-sum-exp (one pass over the partitions).
 // Tokens past the context (and pages with a bad block id) get p = 0 and their
 // V rows are zeroed before the second product, so NaN padding is never read
 // into a result.  Every wait is bounded and the softmax warps exchange data
@@ -58,17 +60,21 @@ constexpr int kStageBytes = 2 * kKBytes + 2 * kQRegion;  // K, V, Q: 69632
 constexpr int kPBytes = 2 * kN * 128;             // P: 2 token halves x 16 rows x 128 B
 constexpr int kOffP = kStages * kStageBytes;
 constexpr int kOffDesc = kOffP + 2 * kPBytes;
-constexpr int kOffBar = kOffDesc + kDescSlots * 64;
+constexpr int kOffRes = kOffDesc + kDescSlots * 64;  // item result handed to the epilogue
+constexpr int kResBytes = kN * 128 * 4 + kN * 4 + 32;  // res[16][128], lse2[16], meta
+constexpr int kOffBar = kOffRes + kResBytes;
 // full, empty (x stages); s_full, s_free, p_full, o_full, o_free (x2);
-// desc_full, desc_empty (x slots); drain; exchange
-constexpr int kNumBars = 2 * kStages + 10 + 2 * kDescSlots + 2;
+// desc_full, desc_empty (x slots); drain; softmax exchange; res_full, res_empty;
+// epilogue exchange
+constexpr int kNumBars = 2 * kStages + 10 + 2 * kDescSlots + 2 + 3;
 constexpr int kOffRed = kOffBar + kNumBars * 8;
 constexpr int kRedFloats = 2 * 4 * kN + 2 * 4 * kN;  // tile max (x2), l sums (x2)
 constexpr int kOffMisc = kOffRed + kRedFloats * 4;
 constexpr int kSmemUsed = kOffMisc + 64;
 constexpr int kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 constexpr int kTmemCols = 64;                 // S x2, O x2
-constexpr int kThreads = 224;
+constexpr int kThreads = 352;                 // 11 warps
 constexpr uint32_t kQBytes = 2 * kQRegion;
 constexpr uint32_t kPageBytes = 4 * 16 * 128;  // K and V halves of one page: 8 KiB
 
@@ -131,7 +137,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   uint64_t* desc_full = o_free + 2;
   uint64_t* desc_empty = desc_full + kDescSlots;
   uint64_t* drain = desc_empty + kDescSlots;
-  uint64_t* xbar = drain + 1;  // softmax warps' exchange barrier
+  uint64_t* xbar = drain + 1;       // softmax warps' exchange barrier
+  uint64_t* res_full = xbar + 1;    // softmax -> epilogue: an item result is ready
+  uint64_t* res_empty = res_full + 1;
+  uint64_t* ebar = res_empty + 1;   // epilogue warps' exchange barrier
+  float* resbuf = reinterpret_cast<float*>(sptr + kOffRes);          // [kN][128]
+  float* reslse = resbuf + kN * 128;                                  // [kN]
+  int* resmeta = reinterpret_cast<int*>(reslse + kN);                 // s, g, part, npart, pbase
   TileDesc* descs = reinterpret_cast<TileDesc*>(sptr + kOffDesc);
   float* red = reinterpret_cast<float*>(sptr + kOffRed);
   float* red_max = red;               // [2][4][kN]
@@ -139,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sptr + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + kOffMisc + 4);
   volatile int* merge_flag = reinterpret_cast<volatile int*>(sptr + kOffMisc + 8);  // [2]
+  (void)merge_flag;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -161,6 +174,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     }
     mbar_init(drain, 1);
     mbar_init(xbar, 4);
+    mbar_init(res_full, 4);
+    mbar_init(res_empty, 4);
+    mbar_init(ebar, 4);
     *abort_flag = 0;
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
@@ -365,8 +381,106 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_wait(drain, 0, nullptr, p.err);
     }
     __syncwarp();
+  } else if (warp >= 7) {
+    // =========================== epilogue ============================
+    const int e = tid - 224;  // output dimension
+    uint32_t k = 0, ek = 0;
+    auto eexchange = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ebar);
+      mbar_wait(ebar, ek & 1, abort_flag, p.err);
+      ++ek;
+    };
+    while (!*abort_flag) {
+      mbar_wait(res_full, k & 1, abort_flag, p.err);
+      const int npart = resmeta[3];
+      if (npart < 0 || *abort_flag) break;
+      const int s = resmeta[0], g = resmeta[1], part = resmeta[2], pbase = resmeta[4];
+      float res[NH], l2[NH];
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        res[h] = h < p.group ? resbuf[h * 128 + e] : 0.f;
+        l2[h] = reslse[h];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(res_empty);
+      ++k;
+      if (npart == 1) {
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          if (h < p.group) {
+            const int64_t o = static_cast<int64_t>(s) * p.hq + g * p.group + h;
+            p.out[o * kD + e] = f32_to_bf16_bits(res[h]);
+            if (e == 0 && p.lse) p.lse[o] = l2[h] * kLn2;
+          }
+        }
+        continue;
+      }
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        if (h < p.group) {
+          const int64_t rec = static_cast<int64_t>(pbase + part) * p.hq + g * p.group + h;
+          __stcg(p.part_o + rec * kD + e, res[h]);
+          if (e == 0) __stcg(p.part_lse + rec, l2[h]);
+        }
+      }
+      // the last partition of (s, g) to finish merges all of them
+      eexchange();
+      if (e == 0) {
+        __threadfence();
+        const int old = atomicAdd(p.merge_cnt + s * p.hkv + g, 1);
+        merge_flag[k & 1] = (old == npart - 1);
+      }
+      eexchange();
+      if (!merge_flag[k & 1]) continue;
+      __threadfence();
+      float M[NH], W[NH], A[NH];
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        M[h] = -CUDART_INF_F;
+        W[h] = 0.f;
+        A[h] = 0.f;
+      }
+      const int64_t rec0 = static_cast<int64_t>(pbase) * p.hq + g * p.group;
+      for (int q = 0; q < npart; ++q) {
+        float li[NH], oi[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          if (h < p.group) {
+            const int64_t rec = rec0 + static_cast<int64_t>(q) * p.hq + h;
+            li[h] = __ldcg(p.part_lse + rec);
+            oi[h] = __ldcg(p.part_o + rec * kD + e);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          if (h < p.group && li[h] != -CUDART_INF_F) {
+            // one-pass log-sum-exp merge: rescale when a larger partition max appears
+            if (li[h] > M[h]) {
+              const float sc = exp2f(M[h] - li[h]);
+              W[h] = W[h] * sc + 1.f;
+              A[h] = A[h] * sc + oi[h];
+              M[h] = li[h];
+            } else {
+              const float f = exp2f(li[h] - M[h]);
+              W[h] += f;
+              A[h] += f * oi[h];
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        if (h < p.group) {
+          const bool live = W[h] > 0.f;
+          const int64_t o = static_cast<int64_t>(s) * p.hq + g * p.group + h;
+          p.out[o * kD + e] = f32_to_bf16_bits(live ? A[h] / W[h] : 0.f);
+          if (e == 0 && p.lse) p.lse[o] = live ? (M[h] + log2f(W[h])) * kLn2 : -CUDART_INF_F;
+        }
+      }
+    }
   } else {
-    // ======================= softmax / epilogue =======================
+    // ============================ softmax =============================
     const int q4 = warp & 3;          // TMEM lane quadrant of this warp
     const int r = q4 * 32 + lane;     // token row of S^T, output dim of O^T
     const int wi = warp - 2;          // index among the softmax warps
@@ -403,7 +517,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_wait(&desc_full[slot], (d / kDescSlots) & 1, abort_flag, p.err);
       const TileDesc* td = descs + slot;
       const int flags = td->flags;
-      if (flags & kEnd) break;
+      if ((flags & kEnd) || *abort_flag) {
+        // no more items: tell the epilogue warps
+        mbar_wait(res_empty, (nfin & 1) ^ 1, abort_flag, p.err);
+        if (r == 0) resmeta[3] = -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(res_full);
+        break;
+      }
       const int s = td->s, g = td->g, part = td->part, npart = td->npart, pbase = td->pbase;
       const int tok0 = td->tok0, tok1 = td->tok1;
       const int mypb = td->pb[r >> 4];
@@ -496,60 +617,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         res[h] = live ? acc[h] / l : 0.f;
         lse2[h] = live ? m_run[h] + log2f(l) : -CUDART_INF_F;
       }
-      if (npart == 1) {
+      // hand the item's result to the epilogue warps
+      mbar_wait(res_empty, (nfin & 1) ^ 1, abort_flag, p.err);
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          if (h < p.group) {
-            const int64_t o = static_cast<int64_t>(s) * p.hq + g * p.group + h;
-            p.out[o * kD + r] = f32_to_bf16_bits(res[h]);
-            if (r == 0 && p.lse) p.lse[o] = lse2[h] * kLn2;
-          }
-        }
-      } else {
+      for (int h = 0; h < NH; ++h)
+        if (h < p.group) resbuf[h * 128 + r] = res[h];
+      if (r == 0) {
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          if (h < p.group) {
-            const int64_t rec = static_cast<int64_t>(pbase + part) * p.hq + g * p.group + h;
-            p.part_o[rec * kD + r] = res[h];
-            if (r == 0) p.part_lse[rec] = lse2[h];
-          }
-        }
-        // the last partition of (s, g) to finish merges all of them
-        __threadfence();
-        exchange();
-        if (wi == 0 && lane == 0) {
-          const int old = atomicAdd(p.merge_cnt + s * p.hkv + g, 1);
-          merge_flag[nfin & 1] = (old == npart - 1);
-        }
-        exchange();
-        if (merge_flag[nfin & 1]) {
-          __threadfence();
-#pragma unroll
-          for (int h = 0; h < NH; ++h) {
-            if (h < p.group) {
-              const int hq = g * p.group + h;
-              float M = -CUDART_INF_F;
-              for (int q = 0; q < npart; ++q)
-                M = fmaxf(M, __ldcg(p.part_lse + static_cast<int64_t>(pbase + q) * p.hq + hq));
-              float wsum = 0.f, a = 0.f;
-              if (M != -CUDART_INF_F) {
-                for (int q = 0; q < npart; ++q) {
-                  const int64_t rec = static_cast<int64_t>(pbase + q) * p.hq + hq;
-                  const float li = __ldcg(p.part_lse + rec);
-                  if (li == -CUDART_INF_F) continue;
-                  const float f = exp2f(li - M);
-                  wsum += f;
-                  a += f * __ldcg(p.part_o + rec * kD + r);
-                }
-              }
-              const bool live = wsum > 0.f;
-              const int64_t o = static_cast<int64_t>(s) * p.hq + hq;
-              p.out[o * kD + r] = f32_to_bf16_bits(live ? a / wsum : 0.f);
-              if (r == 0 && p.lse) p.lse[o] = live ? (M + log2f(wsum)) * kLn2 : -CUDART_INF_F;
-            }
-          }
-        }
+        for (int h = 0; h < NH; ++h) reslse[h] = lse2[h];
+        resmeta[0] = s;
+        resmeta[1] = g;
+        resmeta[2] = part;
+        resmeta[3] = npart;
+        resmeta[4] = pbase;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(res_full);
       ++nfin;
     }
   }
