@@ -154,7 +154,7 @@ PA_API int pa_decode(const void* q, int64_t q_stride, const void* k_pool, const 
               void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Kernel choices for pa_decode_ex (testing and measurement). */
-#define PA_KERNEL_AUTO 0   /* tensor-core kernel for group size >= 4, else CUDA cores */
+#define PA_KERNEL_AUTO 0   /* tensor-core kernel for head_dim 128, else CUDA cores */
 #define PA_KERNEL_SIMT 1   /* CUDA-core kernel (any supported group size) */
 #define PA_KERNEL_TCGEN05 2 /* tcgen05 tensor-core kernel (head_dim 128, group size <= 16) */
 

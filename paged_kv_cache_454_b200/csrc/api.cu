@@ -124,8 +124,7 @@ int max_parts_for(int max_blocks, int block_size, int partition_tokens) {
 
 int choose_kernel(int kernel, int head_dim, int group) {
   if (kernel == PA_KERNEL_AUTO)
-    return (group >= 4 && decode_tcgen05_supported(head_dim, group)) ? PA_KERNEL_TCGEN05
-                                                                     : PA_KERNEL_SIMT;
+    return decode_tcgen05_supported(head_dim, group) ? PA_KERNEL_TCGEN05 : PA_KERNEL_SIMT;
   return kernel;
 }
 

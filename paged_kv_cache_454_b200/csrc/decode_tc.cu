@@ -4,6 +4,8 @@
 // tile of 128 context tokens the work is two small dense products:
 //     S^T [128 tokens x 16] = K_tile [128 x D] . Q^T [D x 16]       (q heads padded to 16)
 //     O^T [D x 16]          = V_tile^T [D x 128] . P [128 x 16]
+// (for group sizes up to 8, columns 8-15 of P carry the bf16 remainder of p, so
+// the weights reach the product with about 16 significant bits)
 // each issued as 8 tcgen05.mma (M = 128, N = 16, K = 16) with fp32 accumulators
 // in tensor memory.  Every K/V byte is read from HBM once for all G heads.
 //
@@ -510,7 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(&o_free[b]);
 #pragma unroll
-      for (int h = 0; h < NH; ++h) acc[h] = acc[h] * alpha_prev[h] + ov[h];
+      for (int h = 0; h < NH; ++h)
+        acc[h] = acc[h] * alpha_prev[h] + ov[h] + (NH <= 8 ? ov[(h + 8) & 15] : 0.f);
     };
     while (true) {
       const int slot = d % kDescSlots;
@@ -574,12 +577,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           l_part[h] = l_part[h] * alpha[h] + pr[h];
           m_run[h] = mn;
         }
-        // p as bf16 into P[b]: row h (head), column r (token), K-major 128B swizzle
+        // p into P[b]: row h (head), column r (token), K-major 128B swizzle.  For
+        // group sizes up to 8, p is split into a bf16 high part (row h) and the
+        // bf16 rounding of its remainder (row 8 + h), so the product carries p to
+        // about 16 significant bits; larger groups use the high part only.
         const uint32_t pbuf = sbase + kOffP + b * kPBytes + (r >> 6) * (kN * 128);
         const int c = r & 63;
 #pragma unroll
-        for (int h = 0; h < NH; ++h)
-          if (h < p.group) sts16(pbuf + swz(h, c >> 3) + (c & 7) * 2, f32_to_bf16_bits(pr[h]));
+        for (int h = 0; h < NH; ++h) {
+          if (h < p.group) {
+            const uint16_t hi = f32_to_bf16_bits(pr[h]);
+            sts16(pbuf + swz(h, c >> 3) + (c & 7) * 2, hi);
+            if (NH <= 8) {
+              const float rem = pr[h] - __uint_as_float(static_cast<uint32_t>(hi) << 16);
+              sts16(pbuf + swz(h + 8, c >> 3) + (c & 7) * 2, f32_to_bf16_bits(rem));
+            }
+          }
+        }
         if (!valid) {
           // zero this token's V row (both 64-dim halves) so padding never reaches O
           const uint32_t vrow = sbase + st * kStageBytes + kKBytes + r * 128;

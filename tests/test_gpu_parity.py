@@ -66,6 +66,17 @@ def lay_mixed(hq=10, hkv=2, d=128):
                               q_lens=chunk + [1, 1], is_prefill=[True] * 3 + [False] * 2)
 
 
+def lay_short_gqa():
+    # contexts of a few keys, where rounding of the softmax weights matters most
+    return synth.build_layout("short_gqa", 109, [2, 3, 4, 5, 6, 7, 8, 9, 12, 16, 2, 3] * 3,
+                              num_q_heads=16, num_kv_heads=2, head_dim=128)
+
+
+def lay_short_mha():
+    return synth.build_layout("short_mha", 110, [2, 3, 5, 8, 13, 16, 17, 2] * 4, num_q_heads=8,
+                              num_kv_heads=8, head_dim=128)
+
+
 DECODE_LAYOUTS = {
     "tiny": synth.tiny,
     "mha128": lay_mha128,
@@ -74,6 +85,8 @@ DECODE_LAYOUTS = {
     "gqa4_d64": lay_gqa4_d64,
     "g16": lay_g16,
     "shared_prefix": lay_shared,
+    "short_gqa": lay_short_gqa,
+    "short_mha": lay_short_mha,
 }
 
 
@@ -168,7 +181,8 @@ def test_decode_simt(name, partition):
     assert pa().pa_get_device_error() == 0
 
 
-@pytest.mark.parametrize("name", ["gqa8", "gqa5", "g16", "shared_prefix", "mha128"])
+@pytest.mark.parametrize("name", ["gqa8", "gqa5", "g16", "shared_prefix", "mha128", "short_gqa",
+                                  "short_mha"])
 @pytest.mark.parametrize("partition", [0, 128, 1024, 1 << 20])
 def test_decode_tcgen05(name, partition):
     st, ref = _step_and_ref(name)
@@ -201,6 +215,18 @@ def test_chunked_prefill(hq, hkv, d):
     got = st.run_gpu()
     H.compare_step(got, ref, what=f"mixed {hq}/{hkv}/{d}")
     assert pa().pa_get_device_error() == 0
+
+
+@pytest.mark.parametrize("hq,hkv", [(16, 2), (10, 2), (4, 4)], ids=["g8", "g5", "mha"])
+def test_chunked_prefill_short_prompts(hq, hkv):
+    # fresh prompts of a few tokens (c = 0) and short chunks on short caches
+    chunks = [2, 3, 5, 8, 16, 1, 4, 7]
+    cached = [0, 0, 0, 0, 0, 3, 2, 9]
+    lens = [c + n for c, n in zip(cached, chunks)]
+    lay = synth.build_layout("pf_short", 111, lens, num_q_heads=hq, num_kv_heads=hkv,
+                             head_dim=128, q_lens=chunks, is_prefill=[True] * len(chunks))
+    st = H.Step.from_host(lay)
+    H.compare_step(st.run_gpu(), st.run_oracle(), what=f"short prefill {hq}/{hkv}")
 
 
 def test_prefill_of_twelve_tokens_in_chunks_of_four_equals_one_chunk():
