@@ -162,3 +162,95 @@ def compare_step(gpu: dict, ref: dict, what=""):
             if lse is not None:
                 assert_lse_close(lse.cpu().numpy(), ref[key][1], what=f"{what} {key} lse")
     return worst
+
+
+# ----------------------------------------------------------------------------
+# Full-size steps (pools drawn on the device), checked on sampled sequences
+# ----------------------------------------------------------------------------
+class FullStep:
+    """A full-size batch step on the device.  Before any library call, host
+    copies of the sampled sequences' blocks and tokens are taken for the oracle
+    (through ``synth.subset``)."""
+
+    def __init__(self, layout: synth.Layout, sample_rows, seed=None):
+        t = torch()
+        self.layout = layout
+        self.dev = t.device("cuda")
+        self.t = synth.fill_device(layout, self.dev, seed=seed)
+        self.sample_rows = [int(r) for r in sample_rows]
+        self.sub, blocks = synth.subset(layout, self.sample_rows)
+        idx = t.as_tensor(blocks, device=self.dev)
+        tok = t.as_tensor(synth.token_rows(layout, self.sample_rows), device=self.dev)
+        self.host = {
+            "k_pool": host_bits(self.t["k_pool"].index_select(0, idx)),
+            "v_pool": host_bits(self.t["v_pool"].index_select(0, idx)),
+            "q": host_bits(self.t["q"].index_select(0, tok)),
+            "key": host_bits(self.t["key"].index_select(0, tok)),
+            "value": host_bits(self.t["value"].index_select(0, tok)),
+        }
+
+    def run_gpu(self):
+        """The step as bench.py runs it: block copies, cache write, chunked
+        prefill of the prefill rows, decode of the decode rows (default kernel
+        choice and partitioning)."""
+        import paged_kv_cache_454_b200 as pa
+        t = torch()
+        lay, d = self.layout, self.t
+        tens = lambda a, dt: t.as_tensor(np.ascontiguousarray(a), dtype=dt, device=self.dev)
+        if lay.copy_pairs.size:
+            pa.pa_copy_blocks(d["k_pool"], d["v_pool"], lay.copy_pairs)
+        pa.pa_reshape_and_cache(d["key"], d["value"], d["k_pool"], d["v_pool"],
+                                tens(lay.slot_mapping(), t.int64))
+        res = {}
+        pf = lay.prefill_rows()
+        if len(pf):
+            q = d["q"][tens(synth.token_rows(lay, pf), t.int64)].contiguous()
+            res["prefill"] = pa.pa_chunked_prefill(
+                q, tens(lay.cu_q_lens(pf), t.int32), int(lay.q_lens[pf].max()), d["k_pool"],
+                d["v_pool"], tens(lay.block_tables[pf], t.int32),
+                tens(lay.context_lens[pf], t.int32), lay.scale, want_lse=True)
+            res["prefill_rows"] = pf
+        dec = lay.decode_rows()
+        if len(dec):
+            q = d["q"][tens(synth.token_rows(lay, dec), t.int64)].contiguous()
+            res["decode"] = pa.pa_decode(q, d["k_pool"], d["v_pool"],
+                                         tens(lay.block_tables[dec], t.int32),
+                                         tens(lay.context_lens[dec], t.int32), lay.scale,
+                                         want_lse=True)
+            res["decode_rows"] = dec
+        t.cuda.synchronize()
+        return res
+
+    def check(self, res, what=""):
+        """Sampled sequences against the oracle, plus whole-batch properties."""
+        lay, sub, h = self.layout, self.sub, self.host
+        kp, vp = h["k_pool"], h["v_pool"]
+        if sub.copy_pairs.size:
+            kp, vp = oracle.copy_blocks(kp, vp, sub.copy_pairs)
+        kp, vp = oracle.reshape_and_cache(kp, vp, h["key"], h["value"], sub.slot_mapping())
+        starts = np.concatenate([[0], np.cumsum(sub.q_lens)])
+        for kind in ("decode", "prefill"):
+            if kind not in res:
+                continue
+            out, lse = res[kind]
+            outf = out.float()
+            assert bool(torch().isfinite(outf).all()), f"{what} {kind}: non-finite output"
+            rows = list(res[kind + "_rows"])
+            # packed token offsets of each row of this call
+            ql = lay.q_lens[rows]
+            offs = dict(zip(rows, np.concatenate([[0], np.cumsum(ql)])[:-1]))
+            for i, s in enumerate(self.sample_rows):
+                if s not in offs:
+                    continue
+                n = int(lay.q_lens[s])
+                qs = h["q"][starts[i]:starts[i] + n]
+                if kind == "decode":
+                    ref_o, ref_l = oracle.decode(qs, kp, vp, sub.block_tables[i:i + 1],
+                                                 sub.context_lens[i:i + 1], lay.scale)
+                else:
+                    ref_o, ref_l = oracle.chunked_prefill(qs, np.array([0, n]), kp, vp,
+                                                          sub.block_tables[i:i + 1],
+                                                          sub.context_lens[i:i + 1], lay.scale)
+                o0 = int(offs[s])
+                assert_close(host_f64(out[o0:o0 + n]), ref_o, what=f"{what} {kind} seq {s}")
+                assert_lse_close(lse[o0:o0 + n].cpu().numpy(), ref_l, what=f"{what} {kind} seq {s}")

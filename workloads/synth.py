@@ -212,12 +212,15 @@ def llama7b_decode(seed: int = 1, batch: int = 64) -> Layout:
 
 
 def llama13b_sampling(seed: int = 2, groups: int = 64, samples: int = 4,
-                      prefix: int = 512, max_suffix: int = 512) -> Layout:
+                      prefix: int = 512, max_suffix: int = 512, batch: int | None = None) -> Layout:
     """Llama-2-13B-shaped parallel sampling: ``groups`` prompts x ``samples``
     samples, MHA 40/40, head_dim 128.  Every sample of a group points at the
     same physical prompt blocks (ref count = samples).  Samples 1.. take a
     copy-on-write copy of the last prompt block (``copy_pairs``); every sample
-    then owns a private suffix of uniform [1, max_suffix] tokens."""
+    then owns a private suffix of uniform [1, max_suffix] tokens.  ``batch``,
+    when given, is the number of sequences (groups = batch // samples)."""
+    if batch is not None:
+        groups = max(1, batch // samples)
     rng = np.random.default_rng(seed)
     bs = BLOCK_SIZE
     pre_blocks = -(-prefix // bs)
@@ -268,11 +271,14 @@ def gqa70b_long(seed: int = 3, batch: int = 128) -> Layout:
 
 
 def mixed_qwen32b(seed: int = 4, n_prefill: int = 8, chunk: int = 512,
-                  n_decode: int = 192) -> Layout:
+                  n_decode: int = 192, batch: int | None = None) -> Layout:
     """Continuous-batching mixed step, Qwen-32B-like: 40 q heads / 8 KV heads,
     head_dim 128.  ``n_prefill`` sequences each add a ``chunk``-token causal
     chunk onto an existing context uniform in [0, 4096]; ``n_decode`` decode
-    sequences have contexts uniform in [256, 8192]."""
+    sequences have contexts uniform in [256, 8192].  ``batch``, when given,
+    replaces ``n_decode`` (a smaller step of the same shape)."""
+    if batch is not None:
+        n_decode = batch
     rng = np.random.default_rng(seed)
     cached = rng.integers(0, 4096 + 1, size=n_prefill)
     dec = rng.integers(256, 8192 + 1, size=n_decode)
