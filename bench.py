@@ -50,6 +50,23 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def rank_seed(workload: str, rank: int):
+    """Seed of rank's batch: rank 0 runs the named workload itself, every other
+    rank an independent batch of the same shape (weak scaling)."""
+    return None if rank == 0 else synth.CONFIGS[workload]().seed + 100 * rank
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise max of per-rank timings (the job is as slow as its slowest
+    rank).  Without a process group, the values themselves."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -344,8 +361,7 @@ def main():
         pg = dist
     peaks, peak_src = load_peaks()
 
-    w = Workload(a.workload, None if rank == 0 else synth.CONFIGS[a.workload]().seed + 100 * rank,
-                 dev, kernel={"auto": 0, "simt": 1, "tcgen05": 2}[a.kernel], partition=a.partition,
+    w = Workload(a.workload, rank_seed(a.workload, rank), dev, kernel={"auto": 0, "simt": 1, "tcgen05": 2}[a.kernel], partition=a.partition,
                  num_seqs=a.num_seqs or None)
     # host copies for the CPU baseline are taken before any kernel touches the pools
     cpu = None
@@ -383,9 +399,7 @@ def main():
         e2e_ms, h2d, d2h = e2e_run(w, stream, max(10, a.steps // 4), a.warmup)
     clk = clocks.stop()
     if pg:
-        tt = torch.tensor([ms, e2e_ms if not a.skip_e2e else 0.0], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        ms, e2e_ms = float(tt[0]), float(tt[1])
+        ms, e2e_ms = max_over_ranks([ms, e2e_ms if not a.skip_e2e else 0.0], pg, dev)
     if not a.skip_e2e:
         e2e = {"value": world * w.tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}

@@ -1,0 +1,69 @@
+"""The N-GPU bench path on CPU: two gloo ranks run the bench's rank seeding and
+its max-over-ranks timing reduction; the reference arm does no work on ranks
+other than 0."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch.distributed as dist
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        # rank r reports (r + 1) ms for the step and (10 - r) ms end to end
+        got = bench.max_over_ranks([rank + 1.0, 10.0 - rank], dist, "cpu")
+        seed = bench.rank_seed("gqa70b_long", rank)
+        dist.barrier()
+        q.put((rank, got, seed))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_reduce_timings_by_max():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert res[0][1] == res[1][1] == [2.0, 10.0]
+    # rank 0 runs the named workload, rank 1 an independent batch of its shape
+    assert res[0][2] is None and res[1][2] is not None
+
+
+def test_reference_arm_skips_nonzero_ranks():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class A:
+        workload = "tiny"
+        steps = 1
+        warmup = 1
+
+    assert bench.reference_arm(A(), rank=1, world=2) is None
+
+
+def test_max_over_ranks_without_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks([1, 2.5]) == [1.0, 2.5]
