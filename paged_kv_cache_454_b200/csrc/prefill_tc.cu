@@ -6,25 +6,33 @@
 // ordered token-major, so one 128-row tile holds floor(128/G) tokens x G heads
 // and shares every K/V tile among them.  Per 128-key tile of the paged context:
 //     S [128 rows x 128 keys] = Q_tile [128 x D] . K_tile^T         (8 MMAs, K = 16)
-//     O [128 rows x D]        = P [128 x 128 keys] . V_tile         (16 MMAs, K = 16)
-// where P = P_hi + P_lo: the bf16 rounding of p and the bf16 rounding of what it
-// left out, so the weights reach the product with about 16 significant bits
-// (bf16 p alone misses the output tolerance on contexts of a few keys)
-// with fp32 accumulators in tensor memory (S and O double-buffered: all 512
-// columns) and operands in 128-byte-swizzled shared memory.
+//     O [128 rows x D]       += P [128 x 128 keys] . V_tile         (16 MMAs, K = 16)
+// with fp32 accumulators in tensor memory.  P = P_hi + P_lo, the bf16 rounding
+// of p and the bf16 rounding of what it left out, so the weights reach the
+// product with about 16 significant bits (bf16 p alone misses the output
+// tolerance on contexts of a few keys).  P is written back into the tensor
+// memory its scores came from (for each 16-key group: 8 columns of P_hi, then 8
+// of P_lo) and the second product reads it from there.
+//
+// Softmax with a lazily raised maximum: each row keeps the maximum m it last
+// used; a tile whose maximum exceeds m by more than 8 (log2 units) raises m,
+// and only then is the row of O in tensor memory (and the row sum) rescaled.
+// Otherwise exp2(s - m) <= 256 is used as is; the final division by the row
+// sum accumulated with the same m makes the result exact either way.
+//
+// Tensor memory (512 columns): S/P of three tiles (128 each) and O (128).
+// Shared memory: q of one row tile, two K slots, three V slots (128B swizzle).
 //
 // Roles (one CTA per SM, persistent over (sequence, KV head, row tile) items,
 // longest causal ranges first):
-//   warp 0     producer: the row tile of q with one 3-D tensor copy (tokens x
-//              heads x 64 dims, twice; one q slot), then each key tile's 8 pages, K and V
-//              in separate two-slot rings so a K slot frees as soon as its
-//              scores are computed.
-//   warp 1     allocates tensor memory; one lane issues S of tile t, then O of
-//              tile t-1.
-//   warps 2-5  softmax: thread r owns row r.  Two passes over its S row
-//              (maximum, then exponentials written as bf16 into the P operand),
-//              online rescaling, and the tile's O folded into registers; the
-//              row is normalised and written at the end of the item.
+//   warp 0      producer of q and K: the row tile of q with one 3-D tensor copy
+//               (tokens x heads x 64 dims, twice), then each key tile's 8 pages.
+//   warp 10     producer of V: each key tile's 8 pages.
+//   warp 1      allocates tensor memory; one lane issues S of tile t, then the
+//               P.V of tile t-1.
+//   warps 2-9   softmax, two warpgroups: thread (r, half) owns row r and key
+//               columns (and output dims) 64*half .. +63; row maxima and sums
+//               are exchanged with the partner warp through shared memory.
 // Keys past a row's causal limit get p = 0; key rows past the context or in
 // pages with a bad block id are zeroed in V before the second product.  Every
 // wait is bounded; no unbounded barrier is used inside the role loops.
@@ -41,22 +49,24 @@ using namespace tc;
 constexpr int kD = 128;
 constexpr int kRegion = 128 * 128;            // 128 rows x 128 bytes
 constexpr int kTileBytes = 2 * kRegion;       // one 128 x 128 bf16 operand tile
-constexpr int kOffQ = 0;                      // Q
-constexpr int kOffK = kOffQ + kTileBytes;     // K[2]
-constexpr int kOffV = kOffK + 2 * kTileBytes; // V[2]
-constexpr int kOffP = kOffV + 2 * kTileBytes; // P high parts
-constexpr int kOffPlo = kOffP + kTileBytes;   // P remainders
-constexpr int kOffBar = kOffPlo + kTileBytes;
-// q_full, q_empty, k_full, k_empty, v_full, v_empty, s_full, s_free (x2 each);
-// p_full; o_full, o_free (x2); drain
-constexpr int kNumBars = 8 * 2 + 1 + 4 + 1;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemUsed = kOffMisc + 64;
+constexpr int kQSlots = 1, kKSlots = 2, kVSlots = 3, kSP = 3;
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kQSlots * kTileBytes;
+constexpr int kOffV = kOffK + kKSlots * kTileBytes;
+constexpr int kOffBar = kOffV + kVSlots * kTileBytes;
+// q_full/empty, k_full/empty, v_full/empty (per slot); s_full, p_full, pv_done
+// (per S/P buffer); o_free; drain; row-quadrant exchange (x4)
+constexpr int kNumBars = 2 * (kQSlots + kKSlots + kVSlots) + 3 * kSP + 1 + 1 + 4;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem slot, abort flag, kmask[8]
+constexpr int kOffX = kOffMisc + 64;                // exchange buffer [2][2][128] floats
+constexpr int kSmemUsed = kOffX + 2 * 2 * 128 * 4;
 constexpr int kSmemBytes = kSmemUsed + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-constexpr int kThreads = 192;
-constexpr int kTmemCols = 512;  // S x2 (128 each), O x2 (128 each)
+constexpr int kThreads = 352;   // q/K producer, MMA, 8 softmax warps, V producer
+constexpr int kTmemCols = 512;  // S/P x3 (128 each), O (128)
+constexpr int kOcol = kSP * 128;
 constexpr uint32_t kPageHalf = 16 * 128;  // one 64-dim half of one page: 2 KiB
+constexpr float kRescaleLog2 = 8.f;       // raise the row maximum only past 2^8
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);
@@ -119,13 +129,24 @@ __device__ __forceinline__ PfItem pf_item(const PfParams& p, int v, bool flag_er
   return it;
 }
 
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return static_cast<uint32_t>(f32_to_bf16_bits(lo)) |
          (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
+}
+
+// Block-table entries of one key tile (lanes 0-7), range-checked.
+__device__ __forceinline__ int tile_page(const PfParams& p, const PfItem& I, int j, int lane,
+                                         bool flag_errors) {
+  const int ptok = j * 128 + lane * 16;
+  int pb = -1;
+  if (lane < 8 && ptok < I.kv_end) {
+    pb = p.block_tables[static_cast<int64_t>(I.s) * p.max_blocks + (ptok >> 4)];
+    if (pb < 0 || pb >= p.num_blocks) {
+      if (flag_errors) raise_error(p.err, PA_DEV_ERR_BLOCK_ID);
+      pb = -1;
+    }
+  }
+  return pb;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ PfParams p) {
@@ -135,37 +156,46 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   unsigned char* sptr = smem_raw + (sbase - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sptr + kOffBar);
   uint64_t* q_full = bars;
-  uint64_t* q_empty = bars + 2;
-  uint64_t* k_full = bars + 4;
-  uint64_t* k_empty = bars + 6;
-  uint64_t* v_full = bars + 8;
-  uint64_t* v_empty = bars + 10;
-  uint64_t* s_full = bars + 12;
-  uint64_t* s_free = bars + 14;
-  uint64_t* p_full = bars + 16;
-  uint64_t* o_full = bars + 17;
-  uint64_t* o_free = bars + 19;
-  uint64_t* drain = bars + 21;
+  uint64_t* q_empty = q_full + kQSlots;
+  uint64_t* k_full = q_empty + kQSlots;
+  uint64_t* k_empty = k_full + kKSlots;
+  uint64_t* v_full = k_empty + kKSlots;
+  uint64_t* v_empty = v_full + kVSlots;
+  uint64_t* s_full = v_empty + kVSlots;   // S of tile t in buffer t % 3
+  uint64_t* p_full = s_full + kSP;        // P of tile t written back
+  uint64_t* pv_done = p_full + kSP;       // P.V of tile t complete
+  uint64_t* o_free = pv_done + kSP;       // O of an item read out
+  uint64_t* drain = o_free + 1;
+  uint64_t* xq = drain + 1;               // [4]: the two softmax warps sharing a row quadrant
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sptr + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + kOffMisc + 4);
-  uint32_t* kmask = reinterpret_cast<uint32_t*>(sptr + kOffMisc + 16);  // [4] valid pages per key tile
+  // loaded pages of key tile t, in slot t % 8 (written by the K producer; the
+  // slot is rewritten only after the scores of tile t + 6 are done)
+  uint32_t* kmask = reinterpret_cast<uint32_t*>(sptr + kOffMisc + 16);
+  float* xbuf = reinterpret_cast<float*>(sptr + kOffX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kQSlots; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < kKSlots; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kVSlots; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&o_full[i], 1);
-      mbar_init(&o_free[i], 128);
     }
-    mbar_init(p_full, 128);
+    for (int i = 0; i < kSP; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 256);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(o_free, 256);
     mbar_init(drain, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&xq[i], 2);
     *abort_flag = 0;
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
@@ -180,123 +210,128 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   const int rows_box = p.tpt * p.group;
 
   if (warp == 0) {
-    // =========================== producer ===========================
+    // ========================= q and K producer =========================
     uint32_t t = 0, it = 0;
     for (int v = blockIdx.x; v < p.total; v += gridDim.x) {
       const PfItem I = pf_item(p, v, lane == 0);
       if (!I.valid) continue;
-      const int qb = 0;
-      mbar_wait(&q_empty[qb], (it & 1) ^ 1, abort_flag, p.err);
+      const int qs = it % kQSlots;
+      mbar_wait(&q_empty[qs], ((it / kQSlots) & 1) ^ 1, abort_flag, p.err);
       if (!*abort_flag && lane == 0) {
-        const uint32_t qd = sbase + kOffQ;
-        mbar_arrive_expect_tx(&q_full[qb], 2 * rows_box * 128);
-        tma_load_3d(qd, &p.tm_q, 0, I.g * p.group, I.q0 + I.i0, &q_full[qb]);
-        tma_load_3d(qd + kRegion, &p.tm_q, 64, I.g * p.group, I.q0 + I.i0, &q_full[qb]);
+        const uint32_t qd = sbase + kOffQ + qs * kTileBytes;
+        mbar_arrive_expect_tx(&q_full[qs], 2 * rows_box * 128);
+        tma_load_3d(qd, &p.tm_q, 0, I.g * p.group, I.q0 + I.i0, &q_full[qs]);
+        tma_load_3d(qd + kRegion, &p.tm_q, 64, I.g * p.group, I.q0 + I.i0, &q_full[qs]);
       }
       ++it;
       for (int j = 0; j < I.ntiles; ++j, ++t) {
-        const int ptok = j * 128 + lane * 16;
-        int pb = -1;
-        if (lane < 8 && ptok < I.kv_end) {
-          pb = p.block_tables[static_cast<int64_t>(I.s) * p.max_blocks + (ptok >> 4)];
-          if (pb < 0 || pb >= p.num_blocks) {
-            raise_error(p.err, PA_DEV_ERR_BLOCK_ID);
-            pb = -1;
-          }
-        }
+        const int pb = tile_page(p, I, j, lane, true);
         const unsigned vm = __ballot_sync(0xffffffffu, pb >= 0) & 0xffu;
-        const int st = t & 1;
-        const uint32_t ph = (t >> 1) & 1;
-        const int row = (pb * p.hkv + I.g) * 16;
-        mbar_wait(&k_empty[st], ph ^ 1, abort_flag, p.err);
-        if (!*abort_flag) {
-          if (lane == 0) {
-            kmask[t & 3] = vm;
-            mbar_arrive_expect_tx(&k_full[st], __popc(vm) * 2 * kPageHalf);
-          }
-          __syncwarp();
-          if (pb >= 0) {
-            const uint32_t kd = sbase + kOffK + st * kTileBytes + lane * kPageHalf;
-            tma_load_2d(kd, &p.tm_k, 0, row, &k_full[st]);
-            tma_load_2d(kd + kRegion, &p.tm_k, 64, row, &k_full[st]);
-          }
+        const int ks = t % kKSlots;
+        mbar_wait(&k_empty[ks], ((t / kKSlots) & 1) ^ 1, abort_flag, p.err);
+        if (*abort_flag) continue;
+        if (lane == 0) {
+          kmask[t & 7] = vm;
+          mbar_arrive_expect_tx(&k_full[ks], __popc(vm) * 2 * kPageHalf);
         }
-        mbar_wait(&v_empty[st], ph ^ 1, abort_flag, p.err);
-        if (!*abort_flag) {
-          if (lane == 0) mbar_arrive_expect_tx(&v_full[st], __popc(vm) * 2 * kPageHalf);
-          __syncwarp();
-          if (pb >= 0) {
-            const uint32_t vd = sbase + kOffV + st * kTileBytes + lane * kPageHalf;
-            tma_load_2d(vd, &p.tm_v, 0, row, &v_full[st]);
-            tma_load_2d(vd + kRegion, &p.tm_v, 64, row, &v_full[st]);
-          }
+        __syncwarp();
+        if (pb >= 0) {
+          const int row = (pb * p.hkv + I.g) * 16;
+          const uint32_t kd = sbase + kOffK + ks * kTileBytes + lane * kPageHalf;
+          tma_load_2d(kd, &p.tm_k, 0, row, &k_full[ks]);
+          tma_load_2d(kd + kRegion, &p.tm_k, 64, row, &k_full[ks]);
         }
       }
     }
     if (*abort_flag && lane == 0) {
-      // wait (bounded) for copies still in flight
-      for (uint32_t u = t > 2 ? t - 2 : 0; u < t; ++u) {
-        mbar_wait(&k_full[u & 1], (u >> 1) & 1, nullptr, p.err);
-        mbar_wait(&v_full[u & 1], (u >> 1) & 1, nullptr, p.err);
-      }
-      if (it > 0) mbar_wait(&q_full[0], (it - 1) & 1, nullptr, p.err);
+      for (uint32_t u = t > kKSlots ? t - kKSlots : 0; u < t; ++u)
+        mbar_wait(&k_full[u % kKSlots], (u / kKSlots) & 1, nullptr, p.err);
+      for (uint32_t u = it > kQSlots ? it - kQSlots : 0; u < it; ++u)
+        mbar_wait(&q_full[u % kQSlots], (u / kQSlots) & 1, nullptr, p.err);
     }
+  } else if (warp == 10) {
+    // =========================== V producer ===========================
+    uint32_t t = 0;
+    for (int v = blockIdx.x; v < p.total; v += gridDim.x) {
+      const PfItem I = pf_item(p, v, false);
+      if (!I.valid) continue;
+      for (int j = 0; j < I.ntiles; ++j, ++t) {
+        const int pb = tile_page(p, I, j, lane, false);
+        const unsigned vm = __ballot_sync(0xffffffffu, pb >= 0) & 0xffu;
+        const int vs = t % kVSlots;
+        mbar_wait(&v_empty[vs], ((t / kVSlots) & 1) ^ 1, abort_flag, p.err);
+        if (*abort_flag) continue;
+        if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], __popc(vm) * 2 * kPageHalf);
+        __syncwarp();
+        if (pb >= 0) {
+          const int row = (pb * p.hkv + I.g) * 16;
+          const uint32_t vd = sbase + kOffV + vs * kTileBytes + lane * kPageHalf;
+          tma_load_2d(vd, &p.tm_v, 0, row, &v_full[vs]);
+          tma_load_2d(vd + kRegion, &p.tm_v, 64, row, &v_full[vs]);
+        }
+      }
+    }
+    if (*abort_flag && lane == 0)
+      for (uint32_t u = t > kVSlots ? t - kVSlots : 0; u < t; ++u)
+        mbar_wait(&v_full[u % kVSlots], (u / kVSlots) & 1, nullptr, p.err);
   } else if (warp == 1) {
     // ============================= MMA ==============================
     if (lane == 0) {
-      uint32_t t = 0, it = 0, prev = 0;
-      bool have_prev = false;
-      auto issue_pv = [&](uint32_t u) {
-        const int st = u & 1;
-        mbar_wait(&v_full[st], (u >> 1) & 1, abort_flag, p.err);
-        mbar_wait(p_full, u & 1, abort_flag, p.err);
-        mbar_wait(&o_free[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err);
+      uint32_t t = 0, it = 0, prev = 0, items_pv = 0;
+      bool have_prev = false, prev_first = false;
+      auto issue_pv = [&](uint32_t u, bool first) {
+        const int sb = u % kSP, vs = u % kVSlots;
+        mbar_wait(&v_full[vs], (u / kVSlots) & 1, abort_flag, p.err);
+        mbar_wait(&p_full[sb], (u / kSP) & 1, abort_flag, p.err);
+        if (first) {  // O of the previous item has been read out
+          mbar_wait(o_free, (items_pv & 1) ^ 1, abort_flag, p.err);
+          ++items_pv;
+        }
         if (*abort_flag) return;
         tc_fence_after();
-        const uint32_t vb = sbase + kOffV + st * kTileBytes;
+        const uint32_t vb = sbase + kOffV + vs * kTileBytes;
+        const uint32_t sp = tmem + sb * 128;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t pb = sbase + (part ? kOffPlo : kOffP);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint64_t a = smem_desc_sw128(pb + (k >> 2) * kRegion + (k & 3) * 32, 16, 1024);
-            const uint64_t b = smem_desc_sw128(vb + k * 2048, kRegion, 1024);
-            umma_ss(tmem + 256 + st * 128, a, b, kIdescO, (part | k) ? 1u : 0u);
-          }
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t bd = smem_desc_sw128(vb + k * 2048, kRegion, 1024);
+          umma_ts(tmem + kOcol, sp + 16 * k, bd, kIdescO, (first && k == 0) ? 0u : 1u);
+          umma_ts(tmem + kOcol, sp + 16 * k + 8, bd, kIdescO, 1u);
         }
-        umma_commit(&o_full[st]);
-        umma_commit(&v_empty[st]);
+        umma_commit(&pv_done[sb]);
+        umma_commit(&v_empty[vs]);
       };
       for (int v = blockIdx.x; v < p.total; v += gridDim.x) {
         const PfItem I = pf_item(p, v, false);
         if (!I.valid) continue;
-        const int qb = 0;
-        mbar_wait(&q_full[qb], it & 1, abort_flag, p.err);
-        const uint32_t qa = sbase + kOffQ;
+        const int qs = it % kQSlots;
+        mbar_wait(&q_full[qs], (it / kQSlots) & 1, abort_flag, p.err);
+        const uint32_t qa = sbase + kOffQ + qs * kTileBytes;
         for (int j = 0; j < I.ntiles; ++j, ++t) {
-          const int st = t & 1;
-          mbar_wait(&k_full[st], (t >> 1) & 1, abort_flag, p.err);
-          mbar_wait(&s_free[st], ((t >> 1) & 1) ^ 1, abort_flag, p.err);
+          const int sb = t % kSP, ks = t % kKSlots;
+          mbar_wait(&k_full[ks], (t / kKSlots) & 1, abort_flag, p.err);
+          // S/P buffer sb is free once the P.V of tile t-3 is done
+          mbar_wait(&pv_done[sb], ((t / kSP) & 1) ^ 1, abort_flag, p.err);
           if (!*abort_flag) {
             tc_fence_after();
-            const uint32_t kb = sbase + kOffK + st * kTileBytes;
+            const uint32_t kb = sbase + kOffK + ks * kTileBytes;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
-              umma_ss(tmem + st * 128, smem_desc_sw128(qa + off, 16, 1024),
+              umma_ss(tmem + sb * 128, smem_desc_sw128(qa + off, 16, 1024),
                       smem_desc_sw128(kb + off, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
             }
-            umma_commit(&s_full[st]);
-            umma_commit(&k_empty[st]);
-            if (j == I.ntiles - 1) umma_commit(&q_empty[qb]);
+            umma_commit(&s_full[sb]);
+            umma_commit(&k_empty[ks]);
+            if (j == I.ntiles - 1) umma_commit(&q_empty[qs]);
           }
-          if (have_prev) issue_pv(prev);
+          if (have_prev) issue_pv(prev, prev_first);
           prev = t;
+          prev_first = j == 0;
           have_prev = true;
         }
         ++it;
       }
-      if (have_prev) issue_pv(prev);
+      if (have_prev) issue_pv(prev, prev_first);
       umma_commit(drain);
       mbar_wait(drain, 0, nullptr, p.err);
     }
@@ -304,125 +339,152 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   } else {
     // ============================ softmax ============================
     const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;  // row of the tile, TMEM lane
+    const int r = q4 * 32 + lane;        // row of the tile, TMEM lane
+    const int half = (warp - 2) >> 2;    // key columns / output dims 64*half .. +63
+    const int cofs = half * 64;
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-    uint32_t t = 0;
-    float acc[kD];
+    const uint32_t ocol = tmem + lane_addr + kOcol + cofs;
+    uint32_t t = 0, xk = 0;
+    // the two warps that share this row quadrant have both passed this point
+    auto exchange = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xq[q4]);
+      mbar_wait(&xq[q4], xk & 1, abort_flag, p.err);
+      ++xk;
+    };
     for (int v = blockIdx.x; v < p.total; v += gridDim.x) {
       const PfItem I = pf_item(p, v, false);
       if (!I.valid) continue;
       const int ti = r / p.group;  // token of this row within the tile
       const bool row_ok = r < rows_box && ti < I.ntok;
       const int limit = row_ok ? I.c + I.i0 + ti + 1 : 0;  // keys 0 .. limit-1
-      float m = -CUDART_INF_F, l = 0.f, alpha_prev = 1.f;
-#pragma unroll
-      for (int d = 0; d < kD; ++d) acc[d] = 0.f;
-      auto fold = [&](uint32_t u) {
-        const int b = u & 1;
-        mbar_wait(&o_full[b], (u >> 1) & 1, abort_flag, p.err);
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float ov[16];
-          tmem_ld16(tmem + lane_addr + 256 + b * 128 + c * 16, ov);
-#pragma unroll
-          for (int k = 0; k < 16; ++k) acc[c * 16 + k] = acc[c * 16 + k] * alpha_prev + ov[k];
-        }
-        tc_fence_before();
-        mbar_arrive(&o_free[b]);
-      };
+      float m = -CUDART_INF_F, l = 0.f;
       for (int j = 0; j < I.ntiles; ++j, ++t) {
-        const int b = t & 1;
+        const int sb = t % kSP;
         const int kv0 = j * 128;
-        mbar_wait(&s_full[b], (t >> 1) & 1, abort_flag, p.err);
+        mbar_wait(&s_full[sb], (t / kSP) & 1, abort_flag, p.err);
         tc_fence_after();
-        const uint32_t vm = kmask[t & 3];
-        const uint32_t sa = tmem + lane_addr + b * 128;
-        // keys kv0 + k are visible to this row when below its limit and in a loaded page
-        auto visible = [&](int k) {
-          return kv0 + k < limit && ((vm >> (k >> 4)) & 1u);
-        };
-        // pass 1: row maximum
-        float mx = -CUDART_INF_F;
+        const uint32_t vm = kmask[t & 7];
+        float sv[64];
+        tmem_ld64(tmem + lane_addr + sb * 128 + cofs, sv);
+        // visibility of this half row's 64 keys as two 32-bit masks: keys below
+        // the row's causal limit, in pages that were loaded
+        uint32_t vis[2];
+        {
+          const int nvis = min(max(limit - kv0 - cofs, 0), 64);  // leading visible keys
+          const uint32_t pages = (vm >> (cofs >> 4)) & 0xfu;     // this half's 4 pages
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const int nw = min(max(nvis - 32 * w, 0), 32);
+            const uint32_t lead = nw >= 32 ? 0xffffffffu : ((1u << nw) - 1u);
+            const uint32_t pg = (((pages >> (2 * w)) & 1u) ? 0x0000ffffu : 0u) |
+                                (((pages >> (2 * w + 1)) & 1u) ? 0xffff0000u : 0u);
+            vis[w] = lead & pg;
+          }
+        }
+        float mx4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          sv[k] *= p.scale_log2;
+          const bool on = (vis[k >> 5] >> (k & 31)) & 1u;
+          mx4[k & 3] = fmaxf(mx4[k & 3], on ? sv[k] : -CUDART_INF_F);
+        }
+        float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        float* px = xbuf + (xk & 1) * 256;
+        px[half * 128 + r] = mx;
+        exchange();
+        mx = fmaxf(mx, px[(half ^ 1) * 128 + r]);
+        // raise the row maximum only when it grows past 2^8; then rescale O and l
+        const bool raise = mx > m + kRescaleLog2;
+        if (j > 0 && __any_sync(0xffffffffu, raise)) {
+          const float f = raise ? exp2f(m - mx) : 1.f;
+          mbar_wait(&pv_done[(t - 1) % kSP], ((t - 1) / kSP) & 1, abort_flag, p.err);
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float ov[16];
+            tmem_ld16(ocol + c * 16, ov);
+            uint32_t ow[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) ow[k] = __float_as_uint(ov[k] * f);
+            tmem_st16_nowait(ocol + c * 16, ow);
+          }
+          tmem_wait_st();
+          l *= f;
+        }
+        if (raise) m = mx;
+        // exponentials written back over the scores as P_hi / P_lo
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float sv[32];
-          tmem_ld32(sa + c * 32, sv);
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (visible(c * 32 + k)) mx = fmaxf(mx, sv[k] * p.scale_log2);
-        }
-        const float mn = fmaxf(m, mx);
-        const float alpha = (mn == -CUDART_INF_F) ? 1.f : exp2f(m - mn);
-        // O of the previous tile is done: P is free again, fold it in
-        if (j > 0) fold(t - 1);
-        // pass 2: exponentials into P (bf16, K-major 128B swizzle), row sum
-        float rs = 0.f;
-        const uint32_t prow = sbase + kOffP + r * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float sv[16];
-          tmem_ld16(sa + c * 16, sv);
-          uint32_t pk[8], pl[8];
+          uint32_t pw[16];
 #pragma unroll
           for (int k = 0; k < 16; k += 2) {
-            const float p0 = visible(c * 16 + k) ? exp2f(sv[k] * p.scale_log2 - mn) : 0.f;
-            const float p1 = visible(c * 16 + k + 1) ? exp2f(sv[k + 1] * p.scale_log2 - mn) : 0.f;
-            rs += p0 + p1;
-            const uint32_t hi = pack_bf16x2(p0, p1);
-            pk[k >> 1] = hi;
-            pl[k >> 1] = pack_bf16x2(p0 - __uint_as_float(hi << 16),
-                                     p1 - __uint_as_float(hi & 0xffff0000u));
+            const int kk = c * 16 + k;
+            const float e0 = exp2f(sv[kk] - m);
+            const float e1 = exp2f(sv[kk + 1] - m);
+            const float p0 = ((vis[kk >> 5] >> (kk & 31)) & 1u) ? e0 : 0.f;
+            const float p1 = ((vis[kk >> 5] >> ((kk + 1) & 31)) & 1u) ? e1 : 0.f;
+            rs4[(k >> 1) & 3] += p0 + p1;
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+            const float2 hf = __bfloat1622float2(hb);
+            const __nv_bfloat162 lb = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+            pw[k >> 1] = *reinterpret_cast<const uint32_t*>(&hb);
+            pw[8 + (k >> 1)] = *reinterpret_cast<const uint32_t*>(&lb);
           }
-          // keys c*16 .. c*16+15: region (c*16)/64, 16-byte chunks 2*(c%4) and 2*(c%4)+1
-          const uint32_t region = prow + (c >> 2) * kRegion;
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int chunk = (c & 3) * 2 + q;
-            const uint32_t off = region + ((chunk ^ (r & 7)) << 4);
-            sts128(off, make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]));
-            sts128(off + (kOffPlo - kOffP),
-                   make_uint4(pl[4 * q], pl[4 * q + 1], pl[4 * q + 2], pl[4 * q + 3]));
-          }
+          tmem_st16_nowait(tmem + lane_addr + sb * 128 + cofs + c * 16, pw);
         }
-        tc_fence_before();
-        mbar_arrive(&s_free[b]);
-        // key rows past the context or in an unloaded page: zero them in V
+        const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        tmem_wait_st();
+        l += rs;
+        // key rows past the context or in an unloaded page: zero this half of them in V
         if (kv0 + 128 > I.ctx || vm != 0xffu) {
           const int key = kv0 + r;
           if (key >= I.ctx || !((vm >> (r >> 4)) & 1u)) {
-            mbar_wait(&v_full[b], (t >> 1) & 1, abort_flag, p.err);
-            const uint32_t vrow = sbase + kOffV + b * kTileBytes + r * 128;
+            const int vs = t % kVSlots;
+            mbar_wait(&v_full[vs], (t / kVSlots) & 1, abort_flag, p.err);
+            const uint32_t vrow = sbase + kOffV + vs * kTileBytes + half * kRegion + r * 128;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              sts128_zero(vrow + k * 16);
-              sts128_zero(vrow + kRegion + k * 16);
-            }
+            for (int k = 0; k < 8; ++k) sts128_zero(vrow + k * 16);
+            fence_proxy_async_smem();
           }
         }
-        l = l * alpha + rs;
-        m = mn;
-        alpha_prev = alpha;
-        fence_proxy_async_smem();
-        mbar_arrive(p_full);
+        tc_fence_before();
+        mbar_arrive(&p_full[sb]);
       }
-      if (I.ntiles > 0) fold(t - 1);
+      // end of the item: O is final once the last P.V is done
+      float ov[64];
+      if (I.ntiles > 0) {
+        mbar_wait(&pv_done[(t - 1) % kSP], ((t - 1) / kSP) & 1, abort_flag, p.err);
+        tc_fence_after();
+        tmem_ld64(ocol, ov);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 64; ++k) ov[k] = 0.f;
+      }
+      tc_fence_before();
+      mbar_arrive(o_free);
+      // row sum over both halves
+      float* px = xbuf + (xk & 1) * 256;
+      px[half * 128 + r] = l;
+      exchange();
+      l += px[(half ^ 1) * 128 + r];
       if (row_ok) {
         const int h = r - ti * p.group;
         const int64_t orow = static_cast<int64_t>(I.q0 + I.i0 + ti) * p.hq + I.g * p.group + h;
         const bool live = l > 0.f;
         const float inv = live ? 1.f / l : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kD);
+        uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kD + cofs);
 #pragma unroll
-        for (int q = 0; q < kD / 8; ++q) {
+        for (int q = 0; q < 8; ++q) {
           uint4 w;
-          w.x = pack_bf16x2(acc[8 * q] * inv, acc[8 * q + 1] * inv);
-          w.y = pack_bf16x2(acc[8 * q + 2] * inv, acc[8 * q + 3] * inv);
-          w.z = pack_bf16x2(acc[8 * q + 4] * inv, acc[8 * q + 5] * inv);
-          w.w = pack_bf16x2(acc[8 * q + 6] * inv, acc[8 * q + 7] * inv);
+          w.x = pack_bf16x2(ov[8 * q] * inv, ov[8 * q + 1] * inv);
+          w.y = pack_bf16x2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv);
+          w.z = pack_bf16x2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv);
+          w.w = pack_bf16x2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv);
           dst[q] = w;
         }
-        if (p.lse) p.lse[orow] = live ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+        if (half == 0 && p.lse) p.lse[orow] = live ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
       }
     }
   }
