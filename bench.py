@@ -457,9 +457,15 @@ def main():
         pg.destroy_process_group()
 
 
-# Per-launch DRAM traffic of the decode call from an ncu capture, keyed by
-# workload and the kernel sources it was taken with (null once they change).
-TRAFFIC = {}
+# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# decode kernel from an ncu capture, keyed by workload and the kernel sources
+# it was taken with (reported as null once those sources change).  The
+# gqa70b_long figure is the 48-sequence capture (1,764,291,328 bytes for
+# 1,755,018,024 algorithmic bytes) scaled by algorithmic bytes to the full
+# 128-sequence batch; see profiles/decode_tc_gqa70b_long.md.
+TRAFFIC = {
+    "gqa70b_long": {"bytes": 4785697610, "sources": "b4a9199e941a"},
+}
 
 
 def kernel_source_digest():
