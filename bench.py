@@ -190,11 +190,17 @@ class Workload:
         mark("decode")
 
     def launches_per_step(self):
+        """Library kernel launches in one step: block copies (480 pairs per
+        launch), the cache write, the decode plan and decode kernel (plus the
+        merge kernel on the CUDA-core path), the prefill kernel."""
+        lay = self.layout
         n = 1  # cache write
-        if self.layout.copy_pairs.size:
-            n += -(-len(self.layout.copy_pairs) // 480)
+        if lay.copy_pairs.size:
+            n += -(-len(lay.copy_pairs) // 480)
         if len(self.dec):
-            n += 3  # plan, decode, merge
+            tensor_core = self.kernel == 2 or (
+                self.kernel == 0 and lay.head_dim == 128 and lay.group_size <= 16)
+            n += 2 if tensor_core else 3
         if len(self.pf):
             n += 1
         return n
