@@ -8,6 +8,12 @@
 //  * Order: longest items first (all full partitions, then the tails by
 //    decreasing length, then empty contexts), so a kernel that hands items out
 //    dynamically schedules them longest-processing-time first.
+//  * Shared prefixes: when sequences share their first physical block (parallel
+//    samples of one prompt, "vLLM 基本原理" / 内存共享) and every item is small
+//    next to one SM's share of the work, the list is instead ordered by that
+//    block, then KV head, then sequence: the samples of a group read the shared
+//    pages of one KV head at the same time, so DRAM serves them once and L2
+//    the rest.  (Up to kSortMax sequences.)
 //  * It also clears the dynamic item counter and the per-(sequence, KV head)
 //    counters the tensor-core kernel uses to find the last partition to finish.
 #include "common.cuh"
@@ -32,17 +38,50 @@ __device__ __forceinline__ int bucket_of(int ntiles) {
   return ntiles == 0 ? 64 : (ntiles >= 64 ? 0 : 64 - ntiles);
 }
 
+constexpr int kSortMax = 1024;  // sequences the locality order sorts (one per thread)
+
+// Inclusive block-wide scan (sum or max) of one value per thread, 1024 threads.
+template <bool kMax>
+__device__ __forceinline__ int block_scan(int x, int* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x = kMax ? max(x, y) : x + y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w = kMax ? max(w, y) : w + y;
+    }
+    warp_tot[lane] = w;
+  }
+  __syncthreads();
+  const int r = warp > 0 ? (kMax ? max(x, warp_tot[warp - 1]) : x + warp_tot[warp - 1]) : x;
+  __syncthreads();
+  return r;
+}
+
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ context_lens,
+                                                           const int32_t* __restrict__ block_tables,
                                                            int S, int max_blocks, int hkv,
                                                            int min_part, int max_part,
-                                                           int target_items, int* header,
-                                                           int* part_base, int2* items,
-                                                           int* merge_cnt, unsigned int* err) {
+                                                           int target_items, int num_sms,
+                                                           int* header, int* part_base,
+                                                           int2* items, int* merge_cnt,
+                                                           unsigned int* err) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
   __shared__ int cand[4];
   __shared__ int bucket[kMaxBuckets];
   __shared__ int cursor[kMaxBuckets];
+  __shared__ unsigned long long skey[kSortMax];  // (first block << 32 | sequence), sorted
+  __shared__ int run_tab[2 * kSortMax];           // per run start: partition prefix, run total
+  __shared__ int sflag[4];                        // [0] any sharing, [1] max item tiles, [2] total tiles x KV heads
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   // ---- partition length ----
@@ -130,8 +169,88 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   }
   __syncthreads();
 
+  // ---- shared prefixes: sort sequences by their first physical block ----
+  bool locality = false;
+  if (S > 1 && S <= kSortMax) {
+    int n2 = 1;
+    while (n2 < S) n2 <<= 1;
+    if (tid < 4) sflag[tid] = 0;
+    for (int i = tid; i < n2; i += 1024) {
+      unsigned long long k = ~0ull;
+      if (i < S) {
+        const int L = clamp_len(context_lens[i], max_blocks, nullptr);
+        const unsigned first =
+            L > 0 ? static_cast<unsigned>(block_tables[static_cast<int64_t>(i) * max_blocks])
+                  : 0xffffffffu;
+        k = (static_cast<unsigned long long>(first) << 32) | static_cast<unsigned>(i);
+      }
+      skey[i] = k;
+    }
+    __syncthreads();
+    for (int k = 2; k <= n2; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < n2; i += 1024) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const unsigned long long a = skey[i], b = skey[ixj];
+            if ((a > b) == ((i & k) == 0)) {
+              skey[i] = b;
+              skey[ixj] = a;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    if (tid < S) {
+      const unsigned first = static_cast<unsigned>(skey[tid] >> 32);
+      const bool shared = tid > 0 && first != 0xffffffffu &&
+                          first == static_cast<unsigned>(skey[tid - 1] >> 32);
+      const int L = clamp_len(context_lens[tid], max_blocks, nullptr);
+      if (shared) atomicOr(&sflag[0], 1);
+      atomicMax(&sflag[1], (min(L, part) + 127) / 128);
+      atomicAdd(&sflag[2], ((L + 127) / 128) * hkv);
+    }
+    __syncthreads();
+    // order for locality only when no single item is large next to one SM's work
+    locality = sflag[0] &&
+               static_cast<long long>(sflag[1]) * 16 * num_sms <= static_cast<long long>(sflag[2]);
+  }
+  if (locality) {
+    // thread i handles sorted position i (S <= 1024).  A run of equal first
+    // blocks is laid out KV head by KV head, the run's sequences in each head.
+    const int i = tid;
+    int s = 0, np = 0, start = 0;
+    bool last = false;
+    if (i < S) {
+      s = static_cast<int>(skey[i] & 0xffffffffull);
+      const int L = clamp_len(context_lens[s], max_blocks, nullptr);
+      np = max(1, (L + part - 1) / part);
+      const unsigned long long f = skey[i] >> 32;
+      const bool st = i == 0 || f == 0xffffffffull || f != (skey[i - 1] >> 32);
+      start = st ? i : 0;
+      last = i == S - 1 || (skey[i + 1] >> 32) == 0xffffffffull || (skey[i + 1] >> 32) != f;
+    }
+    const int pincl = block_scan<false>(np, warp_tot);
+    const int gs = block_scan<true>(start, warp_tot);  // first sorted position of this run
+    int* runP = run_tab;              // indexed by a run's first sorted position
+    int* runT = run_tab + kSortMax;
+    if (i < S && start == i) runP[i] = pincl - np;
+    __syncthreads();
+    if (i < S && last) runT[gs] = pincl - runP[gs];
+    __syncthreads();
+    if (i < S) {
+      const int p0 = runP[gs], tot = runT[gs];
+      const int within = (pincl - np) - p0;
+      for (int g = 0; g < hkv; ++g)
+        for (int q = 0; q < np; ++q)
+          items[static_cast<int64_t>(p0) * hkv + static_cast<int64_t>(g) * tot + within + q] =
+              make_int2(s, (g << 16) | q);
+    }
+  }
+
   // ---- the work list, longest items first ----
-  for (int s = tid; s < S; s += 1024) {
+  for (int s = tid; s < S && !locality; s += 1024) {
     const int L = clamp_len(context_lens[s], max_blocks, nullptr);
     const int full = L / part, rem = L - full * part;
     if (full) {
@@ -155,8 +274,9 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
 
 int launch_decode_plan(const DecodeArgs& a) {
   decode_plan_kernel<<<1, 1024, 0, a.stream>>>(
-      a.context_lens, a.num_seqs, a.max_blocks, a.pool.num_kv_heads, a.min_part, a.max_part,
-      a.target_items, a.ws.header, a.ws.part_base, a.ws.items, a.ws.merge_cnt, a.err);
+      a.context_lens, a.block_tables, a.num_seqs, a.max_blocks, a.pool.num_kv_heads, a.min_part,
+      a.max_part, a.target_items, num_sms(), a.ws.header, a.ws.part_base, a.ws.items,
+      a.ws.merge_cnt, a.err);
   return launch_status();
 }
 

@@ -56,6 +56,14 @@ def lay_shared():
     return lay
 
 
+def lay_shared_many():
+    # enough small items (160 sequences x 32 KV heads, one tile each) that the
+    # work plan orders them by shared first block instead of by length
+    lay = synth.llama13b_sampling(seed=112, groups=40, samples=4, prefix=64, max_suffix=60)
+    lay.num_q_heads = lay.num_kv_heads = 32
+    return lay
+
+
 def lay_mixed(hq=10, hkv=2, d=128):
     # prefill chunks: fresh prompt, short cache, long cache with a ragged chunk;
     # plus two decode sequences
@@ -85,6 +93,7 @@ DECODE_LAYOUTS = {
     "gqa4_d64": lay_gqa4_d64,
     "g16": lay_g16,
     "shared_prefix": lay_shared,
+    "shared_many": lay_shared_many,
     "short_gqa": lay_short_gqa,
     "short_mha": lay_short_mha,
 }
@@ -181,8 +190,8 @@ def test_decode_simt(name, partition):
     assert pa().pa_get_device_error() == 0
 
 
-@pytest.mark.parametrize("name", ["gqa8", "gqa5", "g16", "shared_prefix", "mha128", "short_gqa",
-                                  "short_mha"])
+@pytest.mark.parametrize("name", ["gqa8", "gqa5", "g16", "shared_prefix", "shared_many", "mha128",
+                                  "short_gqa", "short_mha"])
 @pytest.mark.parametrize("partition", [0, 128, 1024, 1 << 20])
 def test_decode_tcgen05(name, partition):
     st, ref = _step_and_ref(name)
