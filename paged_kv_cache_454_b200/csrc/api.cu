@@ -111,9 +111,16 @@ using namespace pa;
 
 namespace {
 
-int partition_or_default(int partition_tokens, int kernel) {
+// Shortest default partition of the tensor-core kernel: kTcPartition tokens of
+// one KV head, i.e. the same bytes per item when an item packs several heads.
+int tc_min_partition(int item_heads) {
+  const int p = kTcPartition / item_heads;
+  return p < 128 ? 128 : p;
+}
+
+int partition_or_default(int partition_tokens, int kernel, int item_heads) {
   if (partition_tokens > 0) return partition_tokens;
-  return kernel == PA_KERNEL_TCGEN05 ? kTcPartition : kSimtPartition;
+  return kernel == PA_KERNEL_TCGEN05 ? tc_min_partition(item_heads) : kSimtPartition;
 }
 
 int max_parts_for(int max_blocks, int block_size, int partition_tokens) {
@@ -139,7 +146,16 @@ size_t pa_decode_workspace_size_ex(int32_t num_seqs, int32_t num_q_heads, pa_poo
     return 0;
   // Size for the smaller of the two defaults when the caller leaves the choice
   // to the library, so either kernel fits.
-  const int part = partition_tokens > 0 ? partition_tokens : (kSimtPartition < kTcPartition ? kSimtPartition : kTcPartition);
+  int part = partition_tokens;
+  if (part <= 0) {
+    part = kSimtPartition;
+    const int group = num_q_heads / pool.num_kv_heads;
+    if (group >= 1 && num_q_heads % pool.num_kv_heads == 0 &&
+        decode_tcgen05_supported(pool.head_dim, group)) {
+      const int tc = tc_min_partition(decode_tcgen05_heads_per_item(group, pool.num_kv_heads));
+      if (tc < part) part = tc;
+    }
+  }
   const int mp = max_parts_for(max_blocks_per_seq, pool.block_size, part);
   return decode_workspace_bytes(num_seqs, num_q_heads, pool.num_kv_heads, pool.head_dim, mp);
 }
@@ -172,7 +188,9 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
   const int kind = choose_kernel(kernel, pool.head_dim, group);
   if (kind == PA_KERNEL_TCGEN05 && !decode_tcgen05_supported(pool.head_dim, group))
     return PA_ERR_UNSUPPORTED;
-  int part = partition_or_default(partition_tokens, kind);
+  const int item_heads =
+      kind == PA_KERNEL_TCGEN05 ? decode_tcgen05_heads_per_item(group, pool.num_kv_heads) : 1;
+  int part = partition_or_default(partition_tokens, kind, item_heads);
   {
     // a partition longer than any context the table can describe is one partition
     const long long max_ctx = static_cast<long long>(max_blocks_per_seq) * pool.block_size;
@@ -202,7 +220,12 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
     a.min_part = a.max_part = part;  // the caller fixed the length
   } else {
     a.min_part = part;
-    a.max_part = kind == PA_KERNEL_TCGEN05 ? kTcMaxPartition : part;
+    if (kind == PA_KERNEL_TCGEN05) {
+      const int mx = kTcMaxPartition / item_heads;
+      a.max_part = mx > part ? mx : part;
+    } else {
+      a.max_part = part;
+    }
   }
   a.target_items = kTcItemsPerSm * num_sms();
   a.max_parts = max_parts;
@@ -211,6 +234,7 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
   a.err = device_error_word();
   a.stream = as_stream(stream);
   if (!a.err) return PA_ERR_CUDA;
+  a.item_heads = item_heads;
 
   st = launch_decode_plan(a);
   if (st != PA_OK) return st;

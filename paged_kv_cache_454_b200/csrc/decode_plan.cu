@@ -274,7 +274,8 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
 
 int launch_decode_plan(const DecodeArgs& a) {
   decode_plan_kernel<<<1, 1024, 0, a.stream>>>(
-      a.context_lens, a.block_tables, a.num_seqs, a.max_blocks, a.pool.num_kv_heads, a.min_part,
+      a.context_lens, a.block_tables, a.num_seqs, a.max_blocks,
+      a.pool.num_kv_heads / a.item_heads, a.min_part,
       a.max_part, a.target_items, num_sms(), a.ws.header, a.ws.part_base, a.ws.items,
       a.ws.merge_cnt, a.err);
   return launch_status();

@@ -1,27 +1,36 @@
-// Paged decode for grouped-query attention on the 5th-generation tensor cores.
+// Paged decode on the 5th-generation tensor cores.
 //
-// All G = Hq/Hkv query heads of one KV head read the same K/V pages, so for a
-// tile of 128 context tokens the work is two small dense products:
-//     S^T [128 tokens x 16] = K_tile [128 x D] . Q^T [D x 16]       (q heads padded to 16)
-//     O^T [D x 16]          = V_tile^T [D x 128] . P [128 x 16]
-// (for group sizes up to 8, columns 8-15 of P carry the bf16 remainder of p, so
-// the weights reach the product with about 16 significant bits)
-// each issued as 8 tcgen05.mma (M = 128, N = 16, K = 16) with fp32 accumulators
-// in tensor memory.  Every K/V byte is read from HBM once for all G heads.
+// All G = Hq/Hkv query heads of one KV head read the same K/V pages.  A tile
+// is 128 rows of the pool: HT KV heads x 16 tokens of each of 8/HT pages (the
+// HT heads of one page are adjacent in the pool, so a page of the tile moves
+// as one HT*2 KiB tensor copy per 64-dim half).  HT = 1 for large groups; for
+// small groups (MHA above all) several KV heads share a tile, which keeps the
+// copies large -- the copy engine moves 2 KiB boxes at well under the HBM
+// rate -- and fills the product's N dimension with useful columns.
+// With NH q columns per tile (the group's q heads of the tile's KV heads,
+// padded) the work is two small dense products:
+//     S^T [128 rows x 16] = K_tile [128 x D] . Q^T [D x 16]
+//     O^T [D x 2NH]       = V_tile^T [D x 128] . P [128 x 2NH]
+// where row r of the tile only scores against its own KV head's q columns
+// (the others get p = 0), and columns NH.. of P carry the bf16 remainder of p,
+// so the weights reach the product with about 16 significant bits.  Each is
+// issued as 8 tcgen05.mma (M = 128, K = 16) with fp32 accumulators in tensor
+// memory.  Every K/V byte is read from HBM once for all of its q heads.
 //
 // Roles (one CTA per SM, persistent; items handed out dynamically in the
-// plan's longest-first order):
-//   warp 6      scheduler: takes the next work item with an atomic counter,
-//               reads its block-table entries (4 tiles per fetch) and publishes
-//               one descriptor per 128-token tile (sequence, KV head, token
-//               range, physical block of each page) into an 8-slot ring.
-//   warp 0      producer: for each tile descriptor, moves the 8 pages (16 tokens
-//               x 64 dims per copy, 128-byte swizzle) with tiled tensor copies
-//               into a 3-stage ring; q of the group rides along.
-//   warp 1      allocates 64 TMEM columns; one lane issues the MMAs and commits
-//               them to mbarriers (S of tile t before O of tile t-1, so the
-//               tensor core computes scores while the softmax warps work).
-//   warps 2-5   softmax: thread r owns token r of S^T and output dimension r of
+// plan's order):
+//   warp 6      scheduler: takes the next work item (sequence, KV-head group,
+//               partition) with an atomic counter, reads its block-table entries
+//               (32 pages per fetch) and publishes one descriptor per tile
+//               (sequence, head group, token range, physical block of each
+//               page) into an 8-slot ring.
+//   warp 0      producer: q of an item into one of two q slots, then for each
+//               tile descriptor the K and V pages (128-byte swizzle) with tiled
+//               tensor copies into a 3-stage ring.
+//   warp 1      allocates the tensor memory; one lane issues the MMAs and
+//               commits them to mbarriers (S of tile t before O of tile t-1, so
+//               the tensor core computes scores while the softmax warps work).
+//   warps 2-5   softmax: thread r owns row r of S^T and output dimension r of
 //               O^T.  Online softmax in the log2 domain with one max exchange
 //               per tile; p goes to shared memory as bf16 in the operand layout
 //               of the second product; the tile's O^T is folded into registers
@@ -29,8 +38,8 @@
 //               normalised result and its log-sum-exp to the epilogue through a
 //               shared-memory buffer and move on.
 //   warps 7-10  epilogue: write the output, or the partition's partial result;
-//               the last partition of a (sequence, KV head) to finish merges all
-//               of them by log-sum-exp (one pass over the partitions).
+//               the last partition of a (sequence, head group) to finish merges
+//               all of them by log-sum-exp (one pass over the partitions).
 // Tokens past the context (and pages with a bad block id) get p = 0 and their
 // V rows are zeroed before the second product, so NaN padding is never read
 // into a result.  Every wait is bounded and the softmax warps exchange data
@@ -51,45 +60,54 @@ namespace {
 using namespace tc;
 
 constexpr int kD = 128;       // head dim
-constexpr int kN = 16;        // MMA N: q heads of one group, padded
-constexpr int kTile = 128;    // tokens per tile (8 pages)
+constexpr int kN = 16;        // N of the score product: q rows of one tile, padded
+constexpr int kRows = 128;    // pool rows per tile
 constexpr int kStages = 3;
 constexpr int kDescSlots = 8;
-constexpr int kRegion = kTile * 128;             // 128 rows x 128 B (one 64-dim half)
+constexpr int kRegion = kRows * 128;              // 128 rows x 128 B (one 64-dim half)
 constexpr int kKBytes = 2 * kRegion;              // K tile, 32 KiB
+constexpr int kStageBytes = 2 * kKBytes;          // K, V: 65536
 constexpr int kQRegion = kN * 128;                // 16 rows x 128 B
-constexpr int kStageBytes = 2 * kKBytes + 2 * kQRegion;  // K, V, Q: 69632
-constexpr int kPBytes = 2 * kN * 128;             // P: 2 token halves x 16 rows x 128 B
-constexpr int kOffP = kStages * kStageBytes;
-constexpr int kOffDesc = kOffP + 2 * kPBytes;
-constexpr int kOffRes = kOffDesc + kDescSlots * 64;  // item result handed to the epilogue
-constexpr int kResBytes = kN * 128 * 4 + kN * 4 + 32;  // res[16][128], lse2[16], meta
-constexpr int kOffBar = kOffRes + kResBytes;
-// full, empty (x stages); s_full, s_free, p_full, o_full, o_free (x2);
-// desc_full, desc_empty (x slots); drain; softmax exchange; res_full, res_empty;
-// epilogue exchange
-constexpr int kNumBars = 2 * kStages + 10 + 2 * kDescSlots + 2 + 3;
-constexpr int kOffRed = kOffBar + kNumBars * 8;
-constexpr int kRedFloats = 2 * 4 * kN + 2 * 4 * kN;  // tile max (x2), l sums (x2)
-constexpr int kOffMisc = kOffRed + kRedFloats * 4;
-constexpr int kSmemUsed = kOffMisc + 64;
-constexpr int kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-constexpr int kTmemCols = 64;                 // S x2, O x2
-constexpr int kThreads = 352;                 // 11 warps
-constexpr uint32_t kQBytes = 2 * kQRegion;
-constexpr uint32_t kPageBytes = 4 * 16 * 128;  // K and V halves of one page: 8 KiB
+constexpr uint32_t kQBytes = 2 * kQRegion;        // one q slot
+constexpr int kQSlots = 2;
+
+// Shared-memory plan for NH q columns per tile.
+template <int NH>
+struct Smem {
+  static constexpr int kNpv = 2 * NH;                       // N of the second product
+  static constexpr int kPBytes = 2 * kNpv * 128;            // 2 token halves x kNpv rows x 128 B
+  static constexpr int kOffQ = kStages * kStageBytes;
+  static constexpr int kOffP = kOffQ + kQSlots * kQBytes;
+  static constexpr int kOffDesc = kOffP + 2 * kPBytes;
+  static constexpr int kOffRes = kOffDesc + kDescSlots * 64;
+  static constexpr int kResBytes = NH * 128 * 4 + NH * 4 + 32;  // res[NH][128], lse2[NH], meta
+  static constexpr int kOffBar = kOffRes + kResBytes;
+  // full, empty (x stages); s_full, s_free, p_full, o_full, o_free, q_full,
+  // q_empty (x2); desc_full, desc_empty (x slots); drain; softmax exchange;
+  // res_full, res_empty; epilogue exchange
+  static constexpr int kNumBars = 2 * kStages + 14 + 2 * kDescSlots + 2 + 3;
+  static constexpr int kOffRed = kOffBar + kNumBars * 8;
+  // tile max (x2), l sums (x2); for single-column rows (NH = 8 only) also
+  // alpha (x2) and the final max (x2)
+  static constexpr int kRedFloats = 2 * 4 * NH + 2 * 4 * NH + (NH <= 8 ? 4 * NH : 0);
+  static constexpr int kOffMisc = kOffRed + kRedFloats * 4;
+  static constexpr int kUsed = kOffMisc + 64;
+  static constexpr int kBytes = kUsed + 1024;  // slack to align the base to 1024
+  static constexpr int kTmemCols = NH <= 8 ? 64 : 128;  // S x2 (16 columns each), O x2
+  static_assert(kBytes <= 232448, "shared memory per CTA");
+  static_assert(2 * kN + 2 * kNpv <= kTmemCols, "tensor memory columns");
+};
+constexpr int kThreads = 352;  // 11 warps
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, kN, false, false);
-constexpr uint32_t kIdescO = idesc_bf16_f32(128, kN, true, false);
 
 // Tile descriptor flags.
 constexpr int kFirst = 1, kLast = 2, kEmpty = 4, kEnd = 8;
 
 struct TileDesc {
-  int s, g, part, npart;
+  int s, g, part, npart;         // g: KV-head group of the item
   int pbase, tok0, tok1, flags;  // tok0: first token of the tile; tok1: end of the item
-  int pb[8];                     // physical block of each page, -1 = skip
+  int pb[8];                     // physical block of each page of the tile, -1 = skip
 };
 static_assert(sizeof(TileDesc) == 64, "descriptor slot size");
 
@@ -112,7 +130,10 @@ struct __align__(64) TcParams {
   int num_blocks;
   int hkv;
   int hq;
-  int group;
+  int group;     // q heads per KV head
+  int ht_shift;  // log2 of the KV heads per tile (and per item)
+  int ngroups;   // KV-head groups: hkv >> ht_shift
+  int nq;        // q columns of a tile: group << ht_shift
   float scale_log2;
 };
 
@@ -122,13 +143,31 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 }
 
 template <int NH>
+__device__ __forceinline__ void tmem_ld_o(uint32_t taddr, float (&v)[2 * NH]);
+template <>
+__device__ __forceinline__ void tmem_ld_o<8>(uint32_t taddr, float (&v)[16]) {
+  tmem_ld16(taddr, v);
+}
+template <>
+__device__ __forceinline__ void tmem_ld_o<16>(uint32_t taddr, float (&v)[32]) {
+  tmem_ld32(taddr, v);
+}
+
+// NH: q columns per tile.  GR: q columns a tile row scores against -- NH (any
+// group; every row computes all columns, masked to its own KV head's) or 1 (one
+// q head per KV head: each row has exactly one column).
+template <int NH, int GR>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ TcParams p) {
+  static_assert(GR == NH || (GR == 1 && NH <= 8), "row column modes");
+  using L = Smem<NH>;
+  constexpr int kNpv = L::kNpv;
+  constexpr uint32_t kIdescO = idesc_bf16_f32(128, kNpv, true, false);
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   unsigned char* sptr = smem_raw + (sbase - raw);
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sptr + kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sptr + L::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* s_full = bars + 2 * kStages;
@@ -136,27 +175,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   uint64_t* p_full = s_free + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* o_free = o_full + 2;
-  uint64_t* desc_full = o_free + 2;
+  uint64_t* q_full = o_free + 2;
+  uint64_t* q_empty = q_full + 2;
+  uint64_t* desc_full = q_empty + 2;
   uint64_t* desc_empty = desc_full + kDescSlots;
   uint64_t* drain = desc_empty + kDescSlots;
   uint64_t* xbar = drain + 1;       // softmax warps' exchange barrier
   uint64_t* res_full = xbar + 1;    // softmax -> epilogue: an item result is ready
   uint64_t* res_empty = res_full + 1;
   uint64_t* ebar = res_empty + 1;   // epilogue warps' exchange barrier
-  float* resbuf = reinterpret_cast<float*>(sptr + kOffRes);          // [kN][128]
-  float* reslse = resbuf + kN * 128;                                  // [kN]
-  int* resmeta = reinterpret_cast<int*>(reslse + kN);                 // s, g, part, npart, pbase
-  TileDesc* descs = reinterpret_cast<TileDesc*>(sptr + kOffDesc);
-  float* red = reinterpret_cast<float*>(sptr + kOffRed);
-  float* red_max = red;               // [2][4][kN]
-  float* red_l = red + 2 * 4 * kN;    // [2][4][kN]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sptr + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + kOffMisc + 4);
-  volatile int* merge_flag = reinterpret_cast<volatile int*>(sptr + kOffMisc + 8);  // [2]
-  (void)merge_flag;
+  float* resbuf = reinterpret_cast<float*>(sptr + L::kOffRes);        // [NH][128]
+  float* reslse = resbuf + NH * 128;                                  // [NH]
+  int* resmeta = reinterpret_cast<int*>(reslse + NH);                 // s, g, part, npart, pbase
+  TileDesc* descs = reinterpret_cast<TileDesc*>(sptr + L::kOffDesc);
+  float* red = reinterpret_cast<float*>(sptr + L::kOffRed);
+  float* red_max = red;                // [2][4][NH]
+  float* red_l = red + 2 * 4 * NH;     // [2][4][NH]
+  float* red_alpha = red_l + 2 * 4 * NH;  // [2][NH] (single-column rows)
+  float* red_mfin = red_alpha + 2 * NH;   // [2][NH] (single-column rows)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sptr + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + L::kOffMisc + 4);
+  volatile int* merge_flag = reinterpret_cast<volatile int*>(sptr + L::kOffMisc + 8);  // [2]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const int hts = p.ht_shift;
+  const int ht = 1 << hts;            // KV heads per tile
+  const int pages = 8 >> hts;         // pages per tile
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -169,6 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_init(&p_full[i], 128);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_free[i], 128);
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
     }
     for (int i = 0; i < kDescSlots; ++i) {
       mbar_init(&desc_full[i], 1);
@@ -184,10 +231,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     prefetch_tmap(&p.tm_v);
     prefetch_tmap(&p.tm_q);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
-  if (warp >= 2 && warp <= 5) {
-    // P rows >= group stay zero for the whole kernel
-    for (int i = tid - 64; i < 2 * kPBytes / 16; i += 128) sts128_zero(sbase + kOffP + i * 16);
+  if (warp == 1) tmem_alloc(tmem_slot, L::kTmemCols);
+  if (GR == 1 && warp >= 2 && warp <= 5) {
+    // Single-column rows: each row writes only its own column of P, so the rest
+    // of P stays zero for the whole kernel; a warp only writes the reduction
+    // slots of its own columns, so the others hold the identity.
+    for (int i = tid - 64; i < 2 * L::kPBytes / 16; i += 128) sts128_zero(sbase + L::kOffP + i * 16);
+    for (int i = tid - 64; i < 2 * 4 * NH; i += 128) {
+      red_max[i] = -CUDART_INF_F;
+      red_l[i] = 0.f;
+    }
     fence_proxy_async_smem();
   }
   fence_barrier_init();
@@ -205,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const int slot = d % kDescSlots;
       mbar_wait(&desc_empty[slot], ((d / kDescSlots) & 1) ^ 1, abort_flag, p.err);
       TileDesc* o = descs + slot;
-      if (lane < 8) o->pb[lane] = pbk;
+      if (lane < 8) o->pb[lane] = lane < pages ? pbk : -1;
       if (lane == 0) {
         o->s = td.s;
         o->g = td.g;
@@ -230,37 +283,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       td.s = dd.x;
       td.g = dd.y >> 16;
       td.part = dd.y & 0xffff;
-      int L = p.context_lens[td.s];
+      int Lc = p.context_lens[td.s];
       const int cap = p.max_blocks * 16;
-      L = L < 0 ? 0 : (L > cap ? cap : L);
+      Lc = Lc < 0 ? 0 : (Lc > cap ? cap : Lc);
       const int tok0 = td.part * part;
-      td.tok1 = min(L, tok0 + part);
+      td.tok1 = min(Lc, tok0 + part);
       td.pbase = p.part_base[td.s];
       td.npart = p.part_base[td.s + 1] - td.pbase;
-      const int ntiles = td.tok1 > tok0 ? (td.tok1 - tok0 + kTile - 1) / kTile : 0;
-      if (ntiles == 0) {
+      const int npages = td.tok1 > tok0 ? (td.tok1 - tok0 + 15) / 16 : 0;
+      if (npages == 0) {
         td.tok0 = tok0;
         td.flags = kFirst | kLast | kEmpty;
         publish(td, -1);
         continue;
       }
-      for (int j0 = 0; j0 < ntiles; j0 += 4) {
-        // lane l reads page l % 8 of tile j0 + l / 8
-        const int jt = j0 + (lane >> 3);
-        const int ptok = tok0 + jt * kTile + (lane & 7) * 16;
+      const int32_t* row = p.block_tables + static_cast<int64_t>(td.s) * p.max_blocks + (tok0 >> 4);
+      for (int p0 = 0; p0 < npages; p0 += 32) {
+        // lane l reads page p0 + l of the item
         int pb = -1;
-        if (jt < ntiles && ptok < td.tok1) {
-          pb = p.block_tables[static_cast<int64_t>(td.s) * p.max_blocks + (ptok >> 4)];
+        if (p0 + lane < npages) {
+          pb = row[p0 + lane];
           if (pb < 0 || pb >= p.num_blocks) {
             raise_error(p.err, PA_DEV_ERR_BLOCK_ID);
             pb = -1;
           }
         }
-        for (int k = 0; k < 4 && j0 + k < ntiles; ++k) {
-          const int pbk = __shfl_sync(0xffffffffu, pb, k * 8 + (lane & 7));
-          td.tok0 = tok0 + (j0 + k) * kTile;
-          td.flags = (j0 + k == 0 ? kFirst : 0) | (j0 + k == ntiles - 1 ? kLast : 0);
-          publish(td, pbk);
+        for (int k = 0; k < 32 && p0 + k < npages; k += pages) {
+          const int pbk = __shfl_sync(0xffffffffu, pb, (k + (lane & (pages - 1))) & 31);
+          td.tok0 = tok0 + (p0 + k) * 16;
+          td.flags = (p0 + k == 0 ? kFirst : 0) | (p0 + k + pages >= npages ? kLast : 0);
+          publish(td, p0 + k + (lane & (pages - 1)) < npages ? pbk : -1);
         }
       }
     }
@@ -274,8 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     }
   } else if (warp == 0) {
     // =========================== producer ===========================
-    uint32_t d = 0, t = 0;
+    uint32_t d = 0, t = 0, nq = 0;
     const uint64_t pol = l2_policy_evict_first();
+    const uint32_t page_bytes = 4u * 2048u * static_cast<uint32_t>(ht);  // K and V, both halves
     while (true) {
       const int slot = d % kDescSlots;
       mbar_wait(&desc_full[slot], (d / kDescSlots) & 1, abort_flag, p.err);
@@ -283,28 +336,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const int flags = td->flags;
       if (flags & kEnd) break;
       if (!(flags & kEmpty)) {
-        const int pb = lane < 8 ? td->pb[lane] : -1;
+        const int pb = lane < pages ? td->pb[lane] : -1;
         const int s = td->s, g = td->g;
+        if (flags & kFirst) {
+          // q of the item's KV-head group into the next q slot
+          const int qs = nq & 1;
+          mbar_wait(&q_empty[qs], ((nq >> 1) & 1) ^ 1, abort_flag, p.err);
+          if (!*abort_flag && lane == 0) {
+            const uint32_t q0 = sbase + L::kOffQ + qs * kQBytes;
+            mbar_arrive_expect_tx(&q_full[qs], kQBytes);
+            tma_load_3d(q0, &p.tm_q, 0, g * p.nq, s, &q_full[qs]);
+            tma_load_3d(q0 + kQRegion, &p.tm_q, 64, g * p.nq, s, &q_full[qs]);
+          }
+          ++nq;
+        }
         const unsigned vmask = __ballot_sync(0xffffffffu, pb >= 0);
         const int st = t % kStages;
         mbar_wait(&empty[st], ((t / kStages) & 1) ^ 1, abort_flag, p.err);
         if (!*abort_flag) {
           const uint32_t stage = sbase + st * kStageBytes;
-          if (lane == 0) mbar_arrive_expect_tx(&full[st], kQBytes + __popc(vmask) * kPageBytes);
+          if (lane == 0) mbar_arrive_expect_tx(&full[st], __popc(vmask) * page_bytes);
           __syncwarp();
-          if (lane == 0) {
-            const uint32_t q0 = stage + 2 * kKBytes;
-            tma_load_3d(q0, &p.tm_q, 0, g * p.group, s, &full[st]);
-            tma_load_3d(q0 + kQRegion, &p.tm_q, 64, g * p.group, s, &full[st]);
-          }
           if (pb >= 0) {
-            const int row = (pb * p.hkv + g) * 16;
-            const uint32_t kdst = stage + lane * 2048;
-            const uint32_t vdst = stage + kKBytes + lane * 2048;
-            tma_load_2d_hint(kdst, &p.tm_k, 0, row, &full[st], pol);
-            tma_load_2d_hint(kdst + kRegion, &p.tm_k, 64, row, &full[st], pol);
-            tma_load_2d_hint(vdst, &p.tm_v, 0, row, &full[st], pol);
-            tma_load_2d_hint(vdst + kRegion, &p.tm_v, 64, row, &full[st], pol);
+            const int prow = (pb * p.hkv + (g << hts)) * 16;
+            const uint32_t kdst = stage + lane * (ht * 2048);
+            const uint32_t vdst = kdst + kKBytes;
+            tma_load_2d_hint(kdst, &p.tm_k, 0, prow, &full[st], pol);
+            tma_load_2d_hint(kdst + kRegion, &p.tm_k, 64, prow, &full[st], pol);
+            tma_load_2d_hint(vdst, &p.tm_v, 0, prow, &full[st], pol);
+            tma_load_2d_hint(vdst + kRegion, &p.tm_v, 64, prow, &full[st], pol);
           }
         }
         ++t;
@@ -318,66 +378,97 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const uint32_t first = t > kStages ? t - kStages : 0;
       for (uint32_t u = first; u < t; ++u)
         mbar_wait(&full[u % kStages], (u / kStages) & 1, nullptr, p.err);
+      const uint32_t qfirst = nq > kQSlots ? nq - kQSlots : 0;
+      for (uint32_t u = qfirst; u < nq; ++u) mbar_wait(&q_full[u & 1], (u >> 1) & 1, nullptr, p.err);
     }
   } else if (warp == 1) {
     // ============================= MMA ==============================
+    // One lane issues both products as soon as each is ready: S of the next
+    // tile once its pages have landed, O of an earlier tile once its p is in
+    // shared memory.  Neither waits for the other, so a stage is released as
+    // soon as its O product is done even while the next tile's pages are still
+    // in flight.  All waits are polls with one shared limit on time without
+    // progress.
     if (lane == 0) {
-      uint32_t d = 0, t = 0, prev = 0;
-      bool have_prev = false;
-      auto issue_pv = [&](uint32_t u) {
-        const int st = u % kStages;
-        const int b = u & 1;
-        const uint32_t bph = (u >> 1) & 1;
-        mbar_wait(&p_full[b], bph, abort_flag, p.err);
-        mbar_wait(&o_free[b], bph ^ 1, abort_flag, p.err);
-        if (*abort_flag) return;
-        tc_fence_after();
-        const uint32_t vbase = sbase + st * kStageBytes + kKBytes;
-        const uint32_t pbase = sbase + kOffP + b * kPBytes;
+      uint32_t d = 0, ts = 0, tpv = 0, mq = 0;  // ts: next S tile; tpv: next O tile
+      bool have_desc = false, s_end = false;
+      int flags = 0;
+      long long last = clock64();
+      while (!*abort_flag) {
+        bool progressed = false;
+        if (tpv < ts) {
+          const int b = tpv & 1;
+          const uint32_t bph = (tpv >> 1) & 1;
+          if (mbar_try_wait(&p_full[b], bph) && mbar_try_wait(&o_free[b], bph ^ 1)) {
+            tc_fence_after();
+            const int st = tpv % kStages;
+            const uint32_t vbase = sbase + st * kStageBytes + kKBytes;
+            const uint32_t pbase = sbase + L::kOffP + b * L::kPBytes;
 #pragma unroll
-        for (int k = 0; k < kTile / 16; ++k) {
-          // A = V^T (MN-major): 16 tokens = 2 groups of 8 rows; D halves kRegion apart
-          const uint64_t a = smem_desc_sw128(vbase + k * 2048, kRegion, 1024);
-          // B = P (K-major, rows = heads): token half k/4, 32 bytes per 16 tokens
-          const uint64_t bd =
-              smem_desc_sw128(pbase + (k >> 2) * (kN * 128) + (k & 3) * 32, 16, 1024);
-          umma_ss(tmem + 2 * kN + b * kN, a, bd, kIdescO, k > 0 ? 1u : 0u);
-        }
-        umma_commit(&o_full[b]);
-        umma_commit(&empty[st]);
-      };
-      while (true) {
-        const int slot = d % kDescSlots;
-        mbar_wait(&desc_full[slot], (d / kDescSlots) & 1, abort_flag, p.err);
-        const int flags = descs[slot].flags;
-        if (flags & kEnd) break;
-        mbar_arrive(&desc_empty[slot]);
-        ++d;
-        if (flags & kEmpty) continue;
-        const int st = t % kStages;
-        const int b = t & 1;
-        mbar_wait(&full[st], (t / kStages) & 1, abort_flag, p.err);
-        mbar_wait(&s_free[b], ((t >> 1) & 1) ^ 1, abort_flag, p.err);
-        if (!*abort_flag) {
-          tc_fence_after();
-          const uint32_t kbase = sbase + st * kStageBytes;
-          const uint32_t qbase = kbase + 2 * kKBytes;
-#pragma unroll
-          for (int k = 0; k < kD / 16; ++k) {
-            const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
-            const uint64_t a = smem_desc_sw128(kbase + off, 16, 1024);
-            const uint64_t bq =
-                smem_desc_sw128(qbase + (k >> 2) * kQRegion + (k & 3) * 32, 16, 1024);
-            umma_ss(tmem + b * kN, a, bq, kIdescS, k > 0 ? 1u : 0u);
+            for (int k = 0; k < kRows / 16; ++k) {
+              // A = V^T (MN-major): 16 rows = 2 groups of 8; D halves kRegion apart
+              const uint64_t a = smem_desc_sw128(vbase + k * 2048, kRegion, 1024);
+              // B = P (K-major, kNpv rows = q columns): row half k/4, 32 bytes per 16 rows
+              const uint64_t bd =
+                  smem_desc_sw128(pbase + (k >> 2) * (kNpv * 128) + (k & 3) * 32, 16, 1024);
+              umma_ss(tmem + 2 * kN + b * kNpv, a, bd, kIdescO, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&o_full[b]);
+            umma_commit(&empty[st]);
+            ++tpv;
+            progressed = true;
           }
-          umma_commit(&s_full[b]);
         }
-        if (have_prev) issue_pv(prev);
-        prev = t;
-        have_prev = true;
-        ++t;
+        if (!s_end && !have_desc) {
+          const int slot = d % kDescSlots;
+          if (mbar_try_wait(&desc_full[slot], (d / kDescSlots) & 1)) {
+            flags = descs[slot].flags;
+            if (flags & kEnd) {
+              s_end = true;
+            } else {
+              mbar_arrive(&desc_empty[slot]);
+              ++d;
+              have_desc = !(flags & kEmpty);
+            }
+            progressed = true;
+          }
+        }
+        if (have_desc) {
+          const int st = ts % kStages;
+          const int b = ts & 1;
+          const int qs = mq & 1;
+          if ((!(flags & kFirst) || mbar_try_wait(&q_full[qs], (mq >> 1) & 1)) &&
+              mbar_try_wait(&full[st], (ts / kStages) & 1) &&
+              mbar_try_wait(&s_free[b], ((ts >> 1) & 1) ^ 1)) {
+            tc_fence_after();
+            const uint32_t kbase = sbase + st * kStageBytes;
+            const uint32_t qbase = sbase + L::kOffQ + qs * kQBytes;
+#pragma unroll
+            for (int k = 0; k < kD / 16; ++k) {
+              const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
+              const uint64_t a = smem_desc_sw128(kbase + off, 16, 1024);
+              const uint64_t bq =
+                  smem_desc_sw128(qbase + (k >> 2) * kQRegion + (k & 3) * 32, 16, 1024);
+              umma_ss(tmem + b * kN, a, bq, kIdescS, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[b]);
+            if (flags & kLast) {
+              umma_commit(&q_empty[qs]);
+              ++mq;
+            }
+            ++ts;
+            have_desc = false;
+            progressed = true;
+          }
+        }
+        if (s_end && tpv == ts) break;
+        if (progressed) {
+          last = clock64();
+        } else if (clock64() - last > kWaitLimitCycles) {
+          *abort_flag = 1;
+          raise_error(p.err, PA_DEV_ERR_TIMEOUT);
+        }
       }
-      if (have_prev) issue_pv(prev);
       // drain: every MMA issued above has completed before TMEM is freed
       umma_commit(drain);
       mbar_wait(drain, 0, nullptr, p.err);
@@ -393,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_wait(ebar, ek & 1, abort_flag, p.err);
       ++ek;
     };
+    const int nq = p.nq;
     while (!*abort_flag) {
       mbar_wait(res_full, k & 1, abort_flag, p.err);
       const int npart = resmeta[3];
@@ -401,17 +493,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       float res[NH], l2[NH];
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        res[h] = h < p.group ? resbuf[h * 128 + e] : 0.f;
+        res[h] = h < nq ? resbuf[h * 128 + e] : 0.f;
         l2[h] = reslse[h];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(res_empty);
       ++k;
+      const int qh0 = g * nq;  // first q head of the group
       if (npart == 1) {
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-          if (h < p.group) {
-            const int64_t o = static_cast<int64_t>(s) * p.hq + g * p.group + h;
+          if (h < nq) {
+            const int64_t o = static_cast<int64_t>(s) * p.hq + qh0 + h;
             p.out[o * kD + e] = f32_to_bf16_bits(res[h]);
             if (e == 0 && p.lse) p.lse[o] = l2[h] * kLn2;
           }
@@ -420,8 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       }
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        if (h < p.group) {
-          const int64_t rec = static_cast<int64_t>(pbase + part) * p.hq + g * p.group + h;
+        if (h < nq) {
+          const int64_t rec = static_cast<int64_t>(pbase + part) * p.hq + qh0 + h;
           __stcg(p.part_o + rec * kD + e, res[h]);
           if (e == 0) __stcg(p.part_lse + rec, l2[h]);
         }
@@ -430,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       eexchange();
       if (e == 0) {
         __threadfence();
-        const int old = atomicAdd(p.merge_cnt + s * p.hkv + g, 1);
+        const int old = atomicAdd(p.merge_cnt + s * p.ngroups + g, 1);
         merge_flag[k & 1] = (old == npart - 1);
       }
       eexchange();
@@ -443,12 +536,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         W[h] = 0.f;
         A[h] = 0.f;
       }
-      const int64_t rec0 = static_cast<int64_t>(pbase) * p.hq + g * p.group;
+      const int64_t rec0 = static_cast<int64_t>(pbase) * p.hq + qh0;
       for (int q = 0; q < npart; ++q) {
         float li[NH], oi[NH];
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-          if (h < p.group) {
+          if (h < nq) {
             const int64_t rec = rec0 + static_cast<int64_t>(q) * p.hq + h;
             li[h] = __ldcg(p.part_lse + rec);
             oi[h] = __ldcg(p.part_o + rec * kD + e);
@@ -456,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-          if (h < p.group && li[h] != -CUDART_INF_F) {
+          if (h < nq && li[h] != -CUDART_INF_F) {
             // one-pass log-sum-exp merge: rescale when a larger partition max appears
             if (li[h] > M[h]) {
               const float sc = exp2f(M[h] - li[h]);
@@ -473,20 +566,177 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       }
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        if (h < p.group) {
+        if (h < nq) {
           const bool live = W[h] > 0.f;
-          const int64_t o = static_cast<int64_t>(s) * p.hq + g * p.group + h;
+          const int64_t o = static_cast<int64_t>(s) * p.hq + qh0 + h;
           p.out[o * kD + e] = f32_to_bf16_bits(live ? A[h] / W[h] : 0.f);
           if (e == 0 && p.lse) p.lse[o] = live ? (M[h] + log2f(W[h])) * kLn2 : -CUDART_INF_F;
         }
       }
     }
+  } else if (GR == 1) {
+    // ===================== softmax, one column per row =====================
+    // Rows 16h..16h+15 of a page belong to KV head h of the tile, whose single
+    // q head is column h.  Lanes 0-15 and 16-31 of a warp hold one head each
+    // (the same head when the tile holds one KV head).
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const int wi = warp - 2;
+    const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
+    const int pj = r >> (4 + hts);
+    const int col = (r >> 4) & (ht - 1);          // this row's q column
+    const int col0 = (2 * q4) & (ht - 1);         // column of lanes 0-15 (S load base)
+    const bool upper = ht > 1 && lane >= 16;      // lanes 16-31 hold column col0 + 1
+    const bool col_writer = lane == 0 || (upper && lane == 16);  // one lane per (warp, column)
+    const int rtok = (pj << 4) | (r & 15);
+    uint32_t d = 0, t = 0, xk = 0, nfin = 0;
+    auto exchange = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xbar);
+      mbar_wait(xbar, xk & 1, abort_flag, p.err);
+      ++xk;
+    };
+    float m_run = -CUDART_INF_F, l_part = 0.f;
+    float acc[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) acc[h] = 0.f;
+    // O of tile u into acc; alpha of tile u comes from its column's owners
+    // (written before the exchange of tile u + 1, which every caller has passed)
+    auto fold = [&](uint32_t u) {
+      const int b = u & 1;
+      mbar_wait(&o_full[b], (u >> 1) & 1, abort_flag, p.err);
+      tc_fence_after();
+      float ov[2 * NH];
+      tmem_ld_o<NH>(tmem + lane_addr + 2 * kN + b * kNpv, ov);
+      tc_fence_before();
+      mbar_arrive(&o_free[b]);
+      const float* al = red_alpha + b * NH;
+#pragma unroll
+      for (int h = 0; h < NH; ++h) acc[h] = acc[h] * al[h] + ov[h] + ov[NH + h];
+    };
+    while (true) {
+      const int slot = d % kDescSlots;
+      mbar_wait(&desc_full[slot], (d / kDescSlots) & 1, abort_flag, p.err);
+      const TileDesc* td = descs + slot;
+      const int flags = td->flags;
+      if ((flags & kEnd) || *abort_flag) {
+        mbar_wait(res_empty, (nfin & 1) ^ 1, abort_flag, p.err);
+        if (r == 0) resmeta[3] = -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(res_full);
+        break;
+      }
+      const int s = td->s, g = td->g, part = td->part, npart = td->npart, pbase = td->pbase;
+      const int tok0 = td->tok0, tok1 = td->tok1;
+      const int mypb = td->pb[pj];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&desc_empty[slot]);
+      ++d;
+      if (flags & kFirst) {
+        m_run = -CUDART_INF_F;
+        l_part = 0.f;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) acc[h] = 0.f;
+      }
+      if (!(flags & kEmpty)) {
+        const int st = t % kStages;
+        const int b = t & 1;
+        mbar_wait(&s_full[b], (t >> 1) & 1, abort_flag, p.err);
+        tc_fence_after();
+        float sv[2];
+        tmem_ld2(tmem + lane_addr + b * kN + col0, sv);
+        tc_fence_before();
+        mbar_arrive(&s_free[b]);
+        const bool valid = tok0 + rtok < tok1 && mypb >= 0;
+        const float x = valid ? (upper ? sv[1] : sv[0]) * p.scale_log2 : -CUDART_INF_F;
+        // max over this warp's rows of the column, then over the warps
+        float v = x;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (ht == 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        float* rm = red_max + (t & 1) * 4 * NH;
+        if (col_writer) rm[wi * NH + col] = v;
+        exchange();
+        const float tmax =
+            fmaxf(fmaxf(rm[col], rm[NH + col]), fmaxf(rm[2 * NH + col], rm[3 * NH + col]));
+        const float mn = fmaxf(m_run, tmax);
+        const float alpha = (mn == -CUDART_INF_F) ? 1.f : exp2f(m_run - mn);
+        const float pr = (x == -CUDART_INF_F) ? 0.f : exp2f(x - mn);
+        l_part = l_part * alpha + pr;
+        m_run = mn;
+        if (col_writer) red_alpha[b * NH + col] = alpha;
+        // p into P[b] at row col (and its bf16 remainder at row NH + col), column r
+        const uint32_t pbuf = sbase + L::kOffP + b * L::kPBytes + (r >> 6) * (kNpv * 128);
+        const int c = r & 63;
+        const uint16_t hi = f32_to_bf16_bits(pr);
+        const float rem = pr - __uint_as_float(static_cast<uint32_t>(hi) << 16);
+        sts16(pbuf + swz(col, c >> 3) + (c & 7) * 2, hi);
+        sts16(pbuf + swz(NH + col, c >> 3) + (c & 7) * 2, f32_to_bf16_bits(rem));
+        if (!valid) {
+          const uint32_t vrow = sbase + st * kStageBytes + kKBytes + r * 128;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            sts128_zero(vrow + k * 16);
+            sts128_zero(vrow + kRegion + k * 16);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&p_full[b]);
+        if (!(flags & kFirst)) fold(t - 1);
+        ++t;
+      }
+      if (!(flags & kLast)) continue;
+      // the exchange below orders the last tile's alpha before its fold
+      float* rl = red_l + (nfin & 1) * 4 * NH;
+      float* mf = red_mfin + (nfin & 1) * NH;
+      {
+        float v = l_part;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (ht == 1) v += __shfl_xor_sync(0xffffffffu, v, 16);
+        if (col_writer) {
+          rl[wi * NH + col] = v;
+          mf[col] = m_run;
+        }
+      }
+      exchange();
+      if (!(flags & kEmpty)) fold(t - 1);
+      float res[NH], lse2[NH];
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        const float l = rl[h] + rl[NH + h] + rl[2 * NH + h] + rl[3 * NH + h];
+        const float m = mf[h];
+        const bool live = m != -CUDART_INF_F && l > 0.f;
+        res[h] = live ? acc[h] / l : 0.f;
+        lse2[h] = live ? m + log2f(l) : -CUDART_INF_F;
+      }
+      mbar_wait(res_empty, (nfin & 1) ^ 1, abort_flag, p.err);
+#pragma unroll
+      for (int h = 0; h < NH; ++h) resbuf[h * 128 + r] = res[h];
+      if (r == 0) {
+#pragma unroll
+        for (int h = 0; h < NH; ++h) reslse[h] = lse2[h];
+        resmeta[0] = s;
+        resmeta[1] = g;
+        resmeta[2] = part;
+        resmeta[3] = npart;
+        resmeta[4] = pbase;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(res_full);
+      ++nfin;
+    }
   } else {
     // ============================ softmax =============================
     const int q4 = warp & 3;          // TMEM lane quadrant of this warp
-    const int r = q4 * 32 + lane;     // token row of S^T, output dim of O^T
+    const int r = q4 * 32 + lane;     // tile row of S^T, output dim of O^T
     const int wi = warp - 2;          // index among the softmax warps
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
+    // tile row r: page j, KV head hh of the tile, token j * 16 + r % 16
+    const int pj = r >> (4 + hts);
+    const int c_lo = ((r >> 4) & (ht - 1)) * p.group;  // this row's q columns [c_lo, c_lo + G)
+    const int c_hi = c_lo + p.group;
+    const int rtok = (pj << 4) | (r & 15);
     uint32_t d = 0, t = 0, xk = 0, nfin = 0;
     // all four softmax warps have passed this point (bounded, unlike bar.sync)
     auto exchange = [&]() {
@@ -507,13 +757,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const int b = u & 1;
       mbar_wait(&o_full[b], (u >> 1) & 1, abort_flag, p.err);
       tc_fence_after();
-      float ov[16];
-      tmem_ld16(tmem + lane_addr + 2 * kN + b * kN, ov);
+      float ov[2 * NH];
+      tmem_ld_o<NH>(tmem + lane_addr + 2 * kN + b * kNpv, ov);
       tc_fence_before();
       mbar_arrive(&o_free[b]);
 #pragma unroll
-      for (int h = 0; h < NH; ++h)
-        acc[h] = acc[h] * alpha_prev[h] + ov[h] + (NH <= 8 ? ov[(h + 8) & 15] : 0.f);
+      for (int h = 0; h < NH; ++h) acc[h] = acc[h] * alpha_prev[h] + ov[h] + ov[NH + h];
     };
     while (true) {
       const int slot = d % kDescSlots;
@@ -530,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       }
       const int s = td->s, g = td->g, part = td->part, npart = td->npart, pbase = td->pbase;
       const int tok0 = td->tok0, tok1 = td->tok1;
-      const int mypb = td->pb[r >> 4];
+      const int mypb = td->pb[pj];
       __syncwarp();
       if (lane == 0) mbar_arrive(&desc_empty[slot]);
       ++d;
@@ -552,50 +801,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         tmem_ld16(tmem + lane_addr + b * kN, sv);
         tc_fence_before();
         mbar_arrive(&s_free[b]);
-        const bool valid = tok0 + r < tok1 && mypb >= 0;
+        const bool valid = tok0 + rtok < tok1 && mypb >= 0;
         float x[NH];
 #pragma unroll
-        for (int h = 0; h < NH; ++h) x[h] = valid ? sv[h] * p.scale_log2 : -CUDART_INF_F;
-        // tile max per head: warp shuffle, then across the four softmax warps
-        float* rm = red_max + (t & 1) * 4 * kN;
+        for (int h = 0; h < NH; ++h)
+          x[h] = (valid && h >= c_lo && h < c_hi) ? sv[h] * p.scale_log2 : -CUDART_INF_F;
+        // tile max per q column: warp shuffle, then across the four softmax warps
+        float* rm = red_max + (t & 1) * 4 * NH;
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
           float v = x[h];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0) rm[wi * kN + h] = v;
+          if (lane == 0) rm[wi * NH + h] = v;
         }
         exchange();
         float pr[NH], alpha[NH];
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
           const float tmax =
-              fmaxf(fmaxf(rm[h], rm[kN + h]), fmaxf(rm[2 * kN + h], rm[3 * kN + h]));
+              fmaxf(fmaxf(rm[h], rm[NH + h]), fmaxf(rm[2 * NH + h], rm[3 * NH + h]));
           const float mn = fmaxf(m_run[h], tmax);
           alpha[h] = (mn == -CUDART_INF_F) ? 1.f : exp2f(m_run[h] - mn);
           pr[h] = (x[h] == -CUDART_INF_F) ? 0.f : exp2f(x[h] - mn);
           l_part[h] = l_part[h] * alpha[h] + pr[h];
           m_run[h] = mn;
         }
-        // p into P[b]: row h (head), column r (token), K-major 128B swizzle.  For
-        // group sizes up to 8, p is split into a bf16 high part (row h) and the
-        // bf16 rounding of its remainder (row 8 + h), so the product carries p to
-        // about 16 significant bits; larger groups use the high part only.
-        const uint32_t pbuf = sbase + kOffP + b * kPBytes + (r >> 6) * (kN * 128);
+        // p into P[b]: row h (q column) and row NH + h (the bf16 remainder),
+        // column r (tile row), K-major 128B swizzle
+        const uint32_t pbuf = sbase + L::kOffP + b * L::kPBytes + (r >> 6) * (kNpv * 128);
         const int c = r & 63;
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-          if (h < p.group) {
-            const uint16_t hi = f32_to_bf16_bits(pr[h]);
-            sts16(pbuf + swz(h, c >> 3) + (c & 7) * 2, hi);
-            if (NH <= 8) {
-              const float rem = pr[h] - __uint_as_float(static_cast<uint32_t>(hi) << 16);
-              sts16(pbuf + swz(h + 8, c >> 3) + (c & 7) * 2, f32_to_bf16_bits(rem));
-            }
-          }
+          const uint16_t hi = f32_to_bf16_bits(pr[h]);
+          const float rem = pr[h] - __uint_as_float(static_cast<uint32_t>(hi) << 16);
+          sts16(pbuf + swz(h, c >> 3) + (c & 7) * 2, hi);
+          sts16(pbuf + swz(NH + h, c >> 3) + (c & 7) * 2, f32_to_bf16_bits(rem));
         }
         if (!valid) {
-          // zero this token's V row (both 64-dim halves) so padding never reaches O
+          // zero this row of V (both 64-dim halves) so padding never reaches O
           const uint32_t vrow = sbase + st * kStageBytes + kKBytes + r * 128;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
@@ -613,20 +857,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       if (!(flags & kLast)) continue;
       if (!(flags & kEmpty)) fold(t - 1);
 
-      // ---- finalize the item: l over the 128 token rows, then output dim r ----
-      float* rl = red_l + (nfin & 1) * 4 * kN;
+      // ---- finalize the item: l over the 128 tile rows, then output dim r ----
+      float* rl = red_l + (nfin & 1) * 4 * NH;
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
         float v = l_part[h];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) rl[wi * kN + h] = v;
+        if (lane == 0) rl[wi * NH + h] = v;
       }
       exchange();
       float res[NH], lse2[NH];
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        const float l = rl[h] + rl[kN + h] + rl[2 * kN + h] + rl[3 * kN + h];
+        const float l = rl[h] + rl[NH + h] + rl[2 * NH + h] + rl[3 * NH + h];
         const bool live = m_run[h] != -CUDART_INF_F && l > 0.f;
         res[h] = live ? acc[h] / l : 0.f;
         lse2[h] = live ? m_run[h] + log2f(l) : -CUDART_INF_F;
@@ -634,8 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       // hand the item's result to the epilogue warps
       mbar_wait(res_empty, (nfin & 1) ^ 1, abort_flag, p.err);
 #pragma unroll
-      for (int h = 0; h < NH; ++h)
-        if (h < p.group) resbuf[h * 128 + r] = res[h];
+      for (int h = 0; h < NH; ++h) resbuf[h * 128 + r] = res[h];
       if (r == 0) {
 #pragma unroll
         for (int h = 0; h < NH; ++h) reslse[h] = lse2[h];
@@ -655,23 +898,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int NH>
+template <int NH, int GR>
 int launch_nh(const TcParams& prm, int64_t item_bound, cudaStream_t stream) {
-  auto kern = decode_tc_kernel<NH>;
+  auto kern = decode_tc_kernel<NH, GR>;
   static KernelLaunchCache cache;
-  const int per_sm = cache.blocks_per_sm(reinterpret_cast<const void*>(kern), kThreads, kSmemBytes);
+  const int per_sm =
+      cache.blocks_per_sm(reinterpret_cast<const void*>(kern), kThreads, Smem<NH>::kBytes);
   if (per_sm < 1) return PA_ERR_CUDA;
   const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm;
   const int grid = static_cast<int>(item_bound < cap ? (item_bound < 1 ? 1 : item_bound) : cap);
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(prm);
+  kern<<<grid, kThreads, Smem<NH>::kBytes, stream>>>(prm);
   return launch_status();
+}
+
+// q columns per tile (8 or 16) and KV heads per tile for a group size.
+struct TcShape {
+  int nh;
+  int ht_shift;
+};
+
+TcShape tc_shape(int group, int hkv) {
+  TcShape sh{group <= 8 ? 8 : 16, 0};
+  // pack KV heads while their q heads fit the tile's columns and the heads
+  // divide evenly into groups
+  while ((1 << (sh.ht_shift + 1)) <= 8 && (group << (sh.ht_shift + 1)) <= sh.nh &&
+         hkv % (1 << (sh.ht_shift + 1)) == 0)
+    ++sh.ht_shift;
+  return sh;
 }
 
 }  // namespace
@@ -680,16 +940,22 @@ bool decode_tcgen05_supported(int head_dim, int group) {
   return head_dim == kD && group >= 1 && group <= kN;
 }
 
+int decode_tcgen05_heads_per_item(int group, int hkv) {
+  return 1 << tc_shape(group, hkv).ht_shift;
+}
+
 int launch_decode_tcgen05(const DecodeArgs& a) {
   const int group = a.num_q_heads / a.pool.num_kv_heads;
   if (!decode_tcgen05_supported(a.pool.head_dim, group)) return PA_ERR_UNSUPPORTED;
+  const TcShape sh = tc_shape(group, a.pool.num_kv_heads);
+  if ((1 << sh.ht_shift) != a.item_heads) return PA_ERR_ARG;  // the plan's items differ
   const int64_t rows = static_cast<int64_t>(a.pool.num_blocks) * a.pool.num_kv_heads * 16;
   if (rows >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
   TcParams p;
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(rows)};
     const uint64_t strides[1] = {kD * 2};
-    const uint32_t box[2] = {64, 16};
+    const uint32_t box[2] = {64, static_cast<uint32_t>(16 << sh.ht_shift)};
     if (!encode_bf16_map(&p.tm_k, a.k_pool, 2, dims, strides, box)) return PA_ERR_CUDA;
     if (!encode_bf16_map(&p.tm_v, a.v_pool, 2, dims, strides, box)) return PA_ERR_CUDA;
   }
@@ -716,11 +982,14 @@ int launch_decode_tcgen05(const DecodeArgs& a) {
   p.hkv = a.pool.num_kv_heads;
   p.hq = a.num_q_heads;
   p.group = group;
+  p.ht_shift = sh.ht_shift;
+  p.ngroups = a.pool.num_kv_heads >> sh.ht_shift;
+  p.nq = group << sh.ht_shift;
   p.scale_log2 = a.scale * kLog2e;
-  const int64_t bound = static_cast<int64_t>(a.num_seqs) * a.max_parts * a.pool.num_kv_heads;
-  if (group <= 4) return launch_nh<4>(p, bound, a.stream);
-  if (group <= 8) return launch_nh<8>(p, bound, a.stream);
-  return launch_nh<16>(p, bound, a.stream);
+  const int64_t bound = static_cast<int64_t>(a.num_seqs) * a.max_parts * p.ngroups;
+  if (group == 1) return launch_nh<8, 1>(p, bound, a.stream);
+  if (sh.nh == 8) return launch_nh<8, 8>(p, bound, a.stream);
+  return launch_nh<16, 16>(p, bound, a.stream);
 }
 
 }  // namespace pa

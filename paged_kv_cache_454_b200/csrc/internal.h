@@ -42,9 +42,9 @@ inline int launch_status() {
 //   header       int32[4]: total items, total partitions, dynamic item counter,
 //                partition length chosen by the plan
 //   part_base    int32[num_seqs + 1]: exclusive prefix of partitions per sequence
-//   merge_cnt    int32[num_seqs * Hkv]: partitions finished per (sequence, KV head)
-//   work list    int2[num_seqs * max_parts * Hkv]: (seq, kv_head << 16 | partition),
-//                longest items first
+//   merge_cnt    int32[num_seqs * Hkv]: partitions finished per (sequence, KV-head group)
+//   work list    int2[num_seqs * max_parts * Hkv]: (seq, head group << 16 | partition)
+//                in the plan's order; a head group is item_heads KV heads
 //   partial out  float[num_seqs * max_parts * Hq * D]
 //   partial lse  float[num_seqs * max_parts * Hq]   (base-2 log-sum-exp)
 // max_parts is the partition count of the longest possible context at the
@@ -81,6 +81,7 @@ struct DecodeArgs {
   int max_part;
   int target_items;  // the plan lengthens partitions while at least this many items remain
   int max_parts;     // workspace bound (partitions of the longest context at min_part)
+  int item_heads = 1;  // KV heads per work item (the tensor-core kernel packs small groups)
   DecodeWorkspace ws;
   unsigned int* err;
   cudaStream_t stream;
@@ -126,5 +127,8 @@ int launch_prefill_simt(const PrefillArgs& a);
 int launch_prefill_tcgen05(const PrefillArgs& a);
 bool prefill_tcgen05_supported(const PrefillArgs& a);
 bool decode_tcgen05_supported(int head_dim, int group);
+// KV heads the tensor-core decode kernel puts in one work item (a power of two
+// dividing hkv).
+int decode_tcgen05_heads_per_item(int group, int hkv);
 
 }  // namespace pa

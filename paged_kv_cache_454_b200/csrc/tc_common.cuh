@@ -96,6 +96,19 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
+// 2 consecutive fp32 columns of this thread's TMEM lane (wait included).
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, float (&v)[2]) {
+  uint32_t r0, r1;
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r0), "=r"(r1)
+      : "r"(taddr)
+      : "memory");
+  v[0] = __uint_as_float(r0);
+  v[1] = __uint_as_float(r1);
+}
+
 // 16 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes
 // 32*(w%4) .. +31); the wait is inside the same asm block so no use of the
 // registers can be scheduled before the data has arrived.
