@@ -72,6 +72,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the same (try_wait may suspend the thread for a while
+// when the phase is not complete; a thread polling several barriers in turn
+// uses this instead).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with parity `parity` to complete.  Returns false if the
 // CTA-wide abort flag is (or becomes) set or the wait exceeds the limit; in the
 // latter case it sets the abort flag and PA_DEV_ERR_TIMEOUT.

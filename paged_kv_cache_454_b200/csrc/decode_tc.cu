@@ -387,9 +387,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     // tile once its pages have landed, O of an earlier tile once its p is in
     // shared memory.  Neither waits for the other, so a stage is released as
     // soon as its O product is done even while the next tile's pages are still
-    // in flight.  All waits are polls with one shared limit on time without
-    // progress.
+    // in flight.  All waits are non-blocking polls with one shared limit on
+    // time without progress.
     if (lane == 0) {
+      // Operand descriptors of every stage and buffer, computed once: issuing
+      // a product then costs only constant adds (the single issuing thread is
+      // otherwise bound by its own address arithmetic).
+      const uint64_t desc_k0 = smem_desc_sw128(sbase, 16, 1024);
+      const uint64_t desc_v0 = smem_desc_sw128(sbase + kKBytes, kRegion, 1024);
+      const uint64_t desc_q0 = smem_desc_sw128(sbase + L::kOffQ, 16, 1024);
+      const uint64_t desc_p0 = smem_desc_sw128(sbase + L::kOffP, 16, 1024);
       uint32_t d = 0, ts = 0, tpv = 0, mq = 0;  // ts: next S tile; tpv: next O tile
       bool have_desc = false, s_end = false;
       int flags = 0;
@@ -399,19 +406,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         if (tpv < ts) {
           const int b = tpv & 1;
           const uint32_t bph = (tpv >> 1) & 1;
-          if (mbar_try_wait(&p_full[b], bph) && mbar_try_wait(&o_free[b], bph ^ 1)) {
+          if (mbar_test_wait(&p_full[b], bph) && mbar_test_wait(&o_free[b], bph ^ 1)) {
             tc_fence_after();
             const int st = tpv % kStages;
-            const uint32_t vbase = sbase + st * kStageBytes + kKBytes;
-            const uint32_t pbase = sbase + L::kOffP + b * L::kPBytes;
+            const uint64_t a0 = desc_add(desc_v0, st * kStageBytes);
+            const uint64_t b0 = desc_add(desc_p0, b * L::kPBytes);
+            const uint32_t dt = tmem + 2 * kN + b * kNpv;
 #pragma unroll
             for (int k = 0; k < kRows / 16; ++k) {
               // A = V^T (MN-major): 16 rows = 2 groups of 8; D halves kRegion apart
-              const uint64_t a = smem_desc_sw128(vbase + k * 2048, kRegion, 1024);
               // B = P (K-major, kNpv rows = q columns): row half k/4, 32 bytes per 16 rows
-              const uint64_t bd =
-                  smem_desc_sw128(pbase + (k >> 2) * (kNpv * 128) + (k & 3) * 32, 16, 1024);
-              umma_ss(tmem + 2 * kN + b * kNpv, a, bd, kIdescO, k > 0 ? 1u : 0u);
+              umma_ss(dt, desc_add(a0, k * 2048), desc_add(b0, (k >> 2) * (kNpv * 128) + (k & 3) * 32),
+                      kIdescO, k > 0 ? 1u : 0u);
             }
             umma_commit(&o_full[b]);
             umma_commit(&empty[st]);
@@ -421,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         if (!s_end && !have_desc) {
           const int slot = d % kDescSlots;
-          if (mbar_try_wait(&desc_full[slot], (d / kDescSlots) & 1)) {
+          if (mbar_test_wait(&desc_full[slot], (d / kDescSlots) & 1)) {
             flags = descs[slot].flags;
             if (flags & kEnd) {
               s_end = true;
@@ -437,20 +443,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           const int st = ts % kStages;
           const int b = ts & 1;
           const int qs = mq & 1;
-          if ((!(flags & kFirst) || mbar_try_wait(&q_full[qs], (mq >> 1) & 1)) &&
-              mbar_try_wait(&full[st], (ts / kStages) & 1) &&
-              mbar_try_wait(&s_free[b], ((ts >> 1) & 1) ^ 1)) {
+          if ((!(flags & kFirst) || mbar_test_wait(&q_full[qs], (mq >> 1) & 1)) &&
+              mbar_test_wait(&full[st], (ts / kStages) & 1) &&
+              mbar_test_wait(&s_free[b], ((ts >> 1) & 1) ^ 1)) {
             tc_fence_after();
-            const uint32_t kbase = sbase + st * kStageBytes;
-            const uint32_t qbase = sbase + L::kOffQ + qs * kQBytes;
+            const uint64_t a0 = desc_add(desc_k0, st * kStageBytes);
+            const uint64_t b0 = desc_add(desc_q0, qs * kQBytes);
+            const uint32_t dt = tmem + b * kN;
 #pragma unroll
-            for (int k = 0; k < kD / 16; ++k) {
-              const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
-              const uint64_t a = smem_desc_sw128(kbase + off, 16, 1024);
-              const uint64_t bq =
-                  smem_desc_sw128(qbase + (k >> 2) * kQRegion + (k & 3) * 32, 16, 1024);
-              umma_ss(tmem + b * kN, a, bq, kIdescS, k > 0 ? 1u : 0u);
-            }
+            for (int k = 0; k < kD / 16; ++k)
+              umma_ss(dt, desc_add(a0, (k >> 2) * kRegion + (k & 3) * 32),
+                      desc_add(b0, (k >> 2) * kQRegion + (k & 3) * 32), kIdescS, k > 0 ? 1u : 0u);
             umma_commit(&s_full[b]);
             if (flags & kLast) {
               umma_commit(&q_empty[qs]);

@@ -129,6 +129,57 @@ __device__ __forceinline__ PfItem pf_item(const PfParams& p, int v, bool flag_er
   return it;
 }
 
+// The same in two steps for a thread that must not stall on the loads: the
+// three loads of item v are issued early (volatile, so they stay where they
+// are written) and the item is decoded when it is needed.
+struct PfRaw {
+  int v, q0, q1, L;
+};
+
+__device__ __forceinline__ int ld_early(const int32_t* ptr) {
+  int x;
+  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(x) : "l"(ptr));
+  return x;
+}
+
+__device__ __forceinline__ PfRaw pf_fetch(const PfParams& p, int v) {
+  PfRaw r;
+  r.v = v;
+  const int s = (v / p.hkv) % p.num_seqs;
+  r.q0 = ld_early(p.cu_q + s);
+  r.q1 = ld_early(p.cu_q + s + 1);
+  r.L = ld_early(p.context_lens + s);
+  return r;
+}
+
+__device__ __forceinline__ PfItem pf_decode(const PfParams& p, const PfRaw& r) {
+  PfItem it;
+  it.g = r.v % p.hkv;
+  const int rest = r.v / p.hkv;
+  it.s = rest % p.num_seqs;
+  const int mt = p.mt_max - 1 - rest / p.num_seqs;
+  it.q0 = r.q0;
+  const int n = r.q1 - r.q0;
+  it.i0 = mt * p.tpt;
+  it.valid = it.i0 < n;
+  if (!it.valid) return it;
+  it.ntok = min(p.tpt, n - it.i0);
+  int L = r.L;
+  const int cap = p.max_blocks * 16;
+  if (L < n || L > cap) {
+    L = L > cap ? cap : L;
+    if (L < n) {
+      it.valid = false;
+      return it;
+    }
+  }
+  it.ctx = L;
+  it.c = L - n;
+  it.kv_end = min(L, it.c + it.i0 + it.ntok);
+  it.ntiles = (it.kv_end + 127) / 128;
+  return it;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return static_cast<uint32_t>(f32_to_bf16_bits(lo)) |
          (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
@@ -276,62 +327,104 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         mbar_wait(&v_full[u % kVSlots], (u / kVSlots) & 1, nullptr, p.err);
   } else if (warp == 1) {
     // ============================= MMA ==============================
+    // One lane issues S of the next key tile and P.V of an earlier one, each as
+    // soon as its inputs are ready (non-blocking polls, one shared limit on time
+    // without progress).  Operand descriptors are computed once; an issue is
+    // then a constant add.  The next item's indices are loaded while the
+    // current one runs.
     if (lane == 0) {
-      uint32_t t = 0, it = 0, prev = 0, items_pv = 0;
-      bool have_prev = false, prev_first = false;
-      auto issue_pv = [&](uint32_t u, bool first) {
-        const int sb = u % kSP, vs = u % kVSlots;
-        mbar_wait(&v_full[vs], (u / kVSlots) & 1, abort_flag, p.err);
-        mbar_wait(&p_full[sb], (u / kSP) & 1, abort_flag, p.err);
-        if (first) {  // O of the previous item has been read out
-          mbar_wait(o_free, (items_pv & 1) ^ 1, abort_flag, p.err);
-          ++items_pv;
-        }
-        if (*abort_flag) return;
-        tc_fence_after();
-        const uint32_t vb = sbase + kOffV + vs * kTileBytes;
-        const uint32_t sp = tmem + sb * 128;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t bd = smem_desc_sw128(vb + k * 2048, kRegion, 1024);
-          umma_ts(tmem + kOcol, sp + 16 * k, bd, kIdescO, (first && k == 0) ? 0u : 1u);
-          umma_ts(tmem + kOcol, sp + 16 * k + 8, bd, kIdescO, 1u);
-        }
-        umma_commit(&pv_done[sb]);
-        umma_commit(&v_empty[vs]);
-      };
-      for (int v = blockIdx.x; v < p.total; v += gridDim.x) {
-        const PfItem I = pf_item(p, v, false);
-        if (!I.valid) continue;
-        const int qs = it % kQSlots;
-        mbar_wait(&q_full[qs], (it / kQSlots) & 1, abort_flag, p.err);
-        const uint32_t qa = sbase + kOffQ + qs * kTileBytes;
-        for (int j = 0; j < I.ntiles; ++j, ++t) {
-          const int sb = t % kSP, ks = t % kKSlots;
-          mbar_wait(&k_full[ks], (t / kKSlots) & 1, abort_flag, p.err);
-          // S/P buffer sb is free once the P.V of tile t-3 is done
-          mbar_wait(&pv_done[sb], ((t / kSP) & 1) ^ 1, abort_flag, p.err);
-          if (!*abort_flag) {
+      const uint64_t dq0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(sbase + kOffK, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sbase + kOffV, kRegion, 1024);
+      uint32_t ts = 0, tpv = 0, it = 0, items_pv = 0;
+      uint32_t first_bits = 0;  // bit t % 8: tile t is the first of its item
+      PfItem I{};
+      int j = 0;
+      bool have = false, s_end = false;
+      PfRaw nxt = pf_fetch(p, blockIdx.x < p.total ? blockIdx.x : 0);
+      bool nxt_ok = blockIdx.x < p.total;
+      long long last = clock64();
+      while (!*abort_flag) {
+        bool prog = false;
+        if (tpv < ts) {
+          const int sb = tpv % kSP, vs = tpv % kVSlots;
+          const bool first = (first_bits >> (tpv & 7)) & 1u;
+          if (mbar_test_wait(&v_full[vs], (tpv / kVSlots) & 1) &&
+              mbar_test_wait(&p_full[sb], (tpv / kSP) & 1) &&
+              (!first || mbar_test_wait(o_free, (items_pv & 1) ^ 1))) {
+            if (first) ++items_pv;  // O of the previous item has been read out
             tc_fence_after();
-            const uint32_t kb = sbase + kOffK + ks * kTileBytes;
+            const uint64_t vb = desc_add(dv0, vs * kTileBytes);
+            const uint32_t sp = tmem + sb * 128;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint64_t bd = desc_add(vb, k * 2048);
+              umma_ts(tmem + kOcol, sp + 16 * k, bd, kIdescO, (first && k == 0) ? 0u : 1u);
+              umma_ts(tmem + kOcol, sp + 16 * k + 8, bd, kIdescO, 1u);
+            }
+            umma_commit(&pv_done[sb]);
+            umma_commit(&v_empty[vs]);
+            ++tpv;
+            prog = true;
+          }
+        }
+        if (!have && !s_end) {
+          // the next valid item: the prefetched one, else load in place
+          while (nxt_ok) {
+            I = pf_decode(p, nxt);
+            const int vn = nxt.v + gridDim.x;
+            nxt_ok = vn < p.total;
+            if (I.valid) {
+              if (nxt_ok) nxt = pf_fetch(p, vn);
+              break;
+            }
+            if (nxt_ok) nxt = pf_fetch(p, vn);
+          }
+          if (I.valid) {
+            have = true;
+            j = 0;
+          } else {
+            s_end = true;
+          }
+          I.valid = false;  // consumed
+          prog = true;
+        }
+        if (have) {
+          const int sb = ts % kSP, ks = ts % kKSlots, qs = it % kQSlots;
+          // S/P buffer sb is free once the P.V of tile ts - 3 is done
+          if ((j > 0 || mbar_test_wait(&q_full[qs], (it / kQSlots) & 1)) &&
+              mbar_test_wait(&k_full[ks], (ts / kKSlots) & 1) &&
+              mbar_test_wait(&pv_done[sb], ((ts / kSP) & 1) ^ 1)) {
+            tc_fence_after();
+            const uint64_t qa = desc_add(dq0, qs * kTileBytes);
+            const uint64_t kb = desc_add(dk0, ks * kTileBytes);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
-              umma_ss(tmem + sb * 128, smem_desc_sw128(qa + off, 16, 1024),
-                      smem_desc_sw128(kb + off, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+              umma_ss(tmem + sb * 128, desc_add(qa, off), desc_add(kb, off), kIdescS,
+                      k > 0 ? 1u : 0u);
             }
             umma_commit(&s_full[sb]);
             umma_commit(&k_empty[ks]);
-            if (j == I.ntiles - 1) umma_commit(&q_empty[qs]);
+            if (j == 0) first_bits |= 1u << (ts & 7);
+            else first_bits &= ~(1u << (ts & 7));
+            ++ts;
+            if (++j == I.ntiles) {
+              umma_commit(&q_empty[qs]);
+              ++it;
+              have = false;
+            }
+            prog = true;
           }
-          if (have_prev) issue_pv(prev, prev_first);
-          prev = t;
-          prev_first = j == 0;
-          have_prev = true;
         }
-        ++it;
+        if (s_end && tpv == ts) break;
+        if (prog) {
+          last = clock64();
+        } else if (clock64() - last > kWaitLimitCycles) {
+          *abort_flag = 1;
+          raise_error(p.err, PA_DEV_ERR_TIMEOUT);
+        }
       }
-      if (have_prev) issue_pv(prev, prev_first);
       umma_commit(drain);
       mbar_wait(drain, 0, nullptr, p.err);
     }
@@ -382,14 +475,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             vis[w] = lead & pg;
           }
         }
+        // Row maximum of the scaled scores.  Scaling is folded into the
+        // exponent's FMA below, so the maximum is taken on the raw scores (the
+        // largest for a positive scale, the smallest for a negative one).  A
+        // warp whose rows see all 64 keys skips the per-key visibility test.
+        const bool all_vis = __all_sync(0xffffffffu, (vis[0] & vis[1]) == 0xffffffffu);
+        const float sc = p.scale_log2;
+        const float sgn = sc < 0.f ? -1.f : 1.f;  // max of sgn * raw score
         float mx4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+        if (all_vis) {
 #pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          sv[k] *= p.scale_log2;
-          const bool on = (vis[k >> 5] >> (k & 31)) & 1u;
-          mx4[k & 3] = fmaxf(mx4[k & 3], on ? sv[k] : -CUDART_INF_F);
+          for (int k = 0; k < 64; ++k) mx4[k & 3] = fmaxf(mx4[k & 3], sgn * sv[k]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) {
+            const bool on = (vis[k >> 5] >> (k & 31)) & 1u;
+            mx4[k & 3] = fmaxf(mx4[k & 3], on ? sgn * sv[k] : -CUDART_INF_F);
+          }
         }
         float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        mx = mx == -CUDART_INF_F ? mx : mx * (sgn * sc);  // scaled maximum
         float* px = xbuf + (xk & 1) * 256;
         px[half * 128 + r] = mx;
         exchange();
@@ -413,7 +518,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           l *= f;
         }
         if (raise) m = mx;
-        // exponentials written back over the scores as P_hi / P_lo
+        // Exponentials written back over the scores as P_hi / P_lo.  P_hi is
+        // p with its mantissa cut to bf16, P_lo the same cut of the remainder
+        // (p = P_hi + P_lo to within 2^-15 of p); both are formed with integer
+        // masks and byte permutes, leaving the multi-function unit to ex2.
+        const float negm = m == -CUDART_INF_F ? 0.f : -m;
         float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -421,16 +530,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
           for (int k = 0; k < 16; k += 2) {
             const int kk = c * 16 + k;
-            const float e0 = exp2f(sv[kk] - m);
-            const float e1 = exp2f(sv[kk + 1] - m);
-            const float p0 = ((vis[kk >> 5] >> (kk & 31)) & 1u) ? e0 : 0.f;
-            const float p1 = ((vis[kk >> 5] >> ((kk + 1) & 31)) & 1u) ? e1 : 0.f;
+            float p0 = exp2f(fmaf(sv[kk], sc, negm));
+            float p1 = exp2f(fmaf(sv[kk + 1], sc, negm));
+            if (!all_vis) {
+              p0 = ((vis[kk >> 5] >> (kk & 31)) & 1u) ? p0 : 0.f;
+              p1 = ((vis[kk >> 5] >> ((kk + 1) & 31)) & 1u) ? p1 : 0.f;
+            }
             rs4[(k >> 1) & 3] += p0 + p1;
-            const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-            const float2 hf = __bfloat1622float2(hb);
-            const __nv_bfloat162 lb = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
-            pw[k >> 1] = *reinterpret_cast<const uint32_t*>(&hb);
-            pw[8 + (k >> 1)] = *reinterpret_cast<const uint32_t*>(&lb);
+            const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+            const float l0 = p0 - __uint_as_float(b0 & 0xffff0000u);
+            const float l1 = p1 - __uint_as_float(b1 & 0xffff0000u);
+            pw[k >> 1] = __byte_perm(b0, b1, 0x7632);
+            pw[8 + (k >> 1)] = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
           }
           tmem_st16_nowait(tmem + lane_addr + sb * 128 + cofs + c * 16, pw);
         }

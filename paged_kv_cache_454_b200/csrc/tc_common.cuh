@@ -35,6 +35,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The descriptor of the same operand `bytes` further on (bytes a multiple of
+// 16; the 14-bit address field cannot carry for shared-memory addresses).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 x bf16 -> fp32.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
 //   15 A major (1 = MN), 16 B major, 17-22 N >> 3, 24-28 M >> 4.
