@@ -39,6 +39,7 @@ __device__ __forceinline__ int bucket_of(int ntiles) {
 }
 
 constexpr int kSortMax = 1024;  // sequences the locality order sorts (one per thread)
+constexpr int kLensCache = 2048;  // sequences whose lengths the plan keeps in shared memory
 
 // Inclusive block-wide scan (sum or max) of one value per thread, 1024 threads.
 template <bool kMax>
@@ -82,7 +83,21 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   __shared__ unsigned long long skey[kSortMax];  // (first block << 32 | sequence), sorted
   __shared__ int run_tab[2 * kSortMax];           // per run start: partition prefix, run total
   __shared__ int sflag[4];                        // [0] any sharing, [1] max item tiles, [2] total tiles x KV heads
+  __shared__ int slens[kLensCache];               // context lengths as given (S <= kLensCache)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // The decode kernel that follows may start its prologue now; it waits for
+  // this grid's results before reading them.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // Context lengths are read once into shared memory when they fit; every pass
+  // below reads them through `lens`.
+  const int32_t* lens = context_lens;
+  if (S <= kLensCache) {
+    for (int s = tid; s < S; s += 1024) slens[s] = context_lens[s];
+    __syncthreads();
+    lens = slens;
+  }
 
   // ---- partition length ----
   int ncand = 1;
@@ -92,7 +107,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   if (ncand > 1) {
     int cnt[4] = {0, 0, 0, 0};
     for (int s = tid; s < S; s += 1024) {
-      const int L = clamp_len(context_lens[s], max_blocks, nullptr);
+      const int L = clamp_len(lens[s], max_blocks, nullptr);
       for (int k = 0; k < ncand; ++k) {
         const int pk = min_part << k;
         const int n = (L + pk - 1) / pk;
@@ -122,7 +137,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     const int s = base + tid;
     int np = 0;
     if (s < S) {
-      const int L = clamp_len(context_lens[s], max_blocks, err);
+      const int L = clamp_len(lens[s], max_blocks, err);
       np = (L + part - 1) / part;
       if (np < 1) np = 1;
       // bucket counts: full partitions, the tail, or an empty context
@@ -178,7 +193,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     for (int i = tid; i < n2; i += 1024) {
       unsigned long long k = ~0ull;
       if (i < S) {
-        const int L = clamp_len(context_lens[i], max_blocks, nullptr);
+        const int L = clamp_len(lens[i], max_blocks, nullptr);
         const unsigned first =
             L > 0 ? static_cast<unsigned>(block_tables[static_cast<int64_t>(i) * max_blocks])
                   : 0xffffffffu;
@@ -206,7 +221,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
       const unsigned first = static_cast<unsigned>(skey[tid] >> 32);
       const bool shared = tid > 0 && first != 0xffffffffu &&
                           first == static_cast<unsigned>(skey[tid - 1] >> 32);
-      const int L = clamp_len(context_lens[tid], max_blocks, nullptr);
+      const int L = clamp_len(lens[tid], max_blocks, nullptr);
       if (shared) atomicOr(&sflag[0], 1);
       atomicMax(&sflag[1], (min(L, part) + 127) / 128);
       atomicAdd(&sflag[2], ((L + 127) / 128) * hkv);
@@ -224,7 +239,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     bool last = false;
     if (i < S) {
       s = static_cast<int>(skey[i] & 0xffffffffull);
-      const int L = clamp_len(context_lens[s], max_blocks, nullptr);
+      const int L = clamp_len(lens[s], max_blocks, nullptr);
       np = max(1, (L + part - 1) / part);
       const unsigned long long f = skey[i] >> 32;
       const bool st = i == 0 || f == 0xffffffffull || f != (skey[i - 1] >> 32);
@@ -251,7 +266,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
 
   // ---- the work list, longest items first ----
   for (int s = tid; s < S && !locality; s += 1024) {
-    const int L = clamp_len(context_lens[s], max_blocks, nullptr);
+    const int L = clamp_len(lens[s], max_blocks, nullptr);
     const int full = L / part, rem = L - full * part;
     if (full) {
       int at = atomicAdd(&cursor[full_bucket], full * hkv);

@@ -248,6 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The kernel may be launched while the plan kernel before it still runs (a
+  // programmatic dependent launch): the set-up above overlaps it, and nothing
+  // below reads the plan's results before the plan grid has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 6) {
     // =========================== scheduler ===========================
@@ -917,7 +921,22 @@ int launch_nh(const TcParams& prm, int64_t item_bound, cudaStream_t stream) {
   if (per_sm < 1) return PA_ERR_CUDA;
   const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm;
   const int grid = static_cast<int>(item_bound < cap ? (item_bound < 1 ? 1 : item_bound) : cap);
-  kern<<<grid, kThreads, Smem<NH>::kBytes, stream>>>(prm);
+  // programmatic dependent launch: the CTAs start and set up while the plan
+  // kernel (launched just before on the same stream) finishes
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Smem<NH>::kBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, prm) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
   return launch_status();
 }
 

@@ -180,6 +180,31 @@ __device__ __forceinline__ PfItem pf_decode(const PfParams& p, const PfRaw& r) {
   return it;
 }
 
+// 2^x on the FMA pipe, for the share of the softmax exponentials taken off the
+// multi-function unit.  x = j + f with j = rint(x) (by the 1.5 * 2^23 rounding
+// trick) and |f| <= 1/2; 2^f = e^(f ln 2) by its Taylor series to degree 5
+// (relative error below 3.3e-6 on |f| <= 1/2); j is added to the exponent
+// field.  x is clamped below at -126; callers pass x <= 8.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
+  float y = 1.3333558146428441e-3f;       // (ln 2)^5 / 5!
+  y = fmaf(y, f, 9.618129107628477e-3f);  // (ln 2)^4 / 4!
+  y = fmaf(y, f, 5.5504108664821576e-2f); // (ln 2)^3 / 3!
+  y = fmaf(y, f, 2.402265069591007e-1f);  // (ln 2)^2 / 2!
+  y = fmaf(y, f, 6.931471805599453e-1f);  // ln 2
+  y = fmaf(y, f, 1.f);
+  return __int_as_float(__float_as_int(y) + (__float_as_int(t) << 23));
+}
+
+#ifndef PA_PREFILL_EXP_FMA_EVERY
+#define PA_PREFILL_EXP_FMA_EVERY 0
+#endif
+// Every kExpFmaEvery-th exponential of the softmax is computed with exp2_fma
+// (0: none), balancing the multi-function unit against the FMA pipe.
+constexpr int kExpFmaEvery = PA_PREFILL_EXP_FMA_EVERY;
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return static_cast<uint32_t>(f32_to_bf16_bits(lo)) |
          (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
@@ -481,20 +506,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // warp whose rows see all 64 keys skips the per-key visibility test.
         const bool all_vis = __all_sync(0xffffffffu, (vis[0] & vis[1]) == 0xffffffffu);
         const float sc = p.scale_log2;
-        const float sgn = sc < 0.f ? -1.f : 1.f;  // max of sgn * raw score
-        float mx4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-        if (all_vis) {
+        float mx;
+        if (sc >= 0.f) {
+          float mx4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+          if (all_vis) {
 #pragma unroll
-          for (int k = 0; k < 64; ++k) mx4[k & 3] = fmaxf(mx4[k & 3], sgn * sv[k]);
-        } else {
+            for (int k = 0; k < 64; ++k) mx4[k & 3] = fmaxf(mx4[k & 3], sv[k]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 64; ++k) {
+              const bool on = (vis[k >> 5] >> (k & 31)) & 1u;
+              mx4[k & 3] = fmaxf(mx4[k & 3], on ? sv[k] : -CUDART_INF_F);
+            }
+          }
+          mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        } else {  // a negative scale turns the smallest raw score into the largest
+          float mn4[4] = {CUDART_INF_F, CUDART_INF_F, CUDART_INF_F, CUDART_INF_F};
 #pragma unroll
           for (int k = 0; k < 64; ++k) {
             const bool on = (vis[k >> 5] >> (k & 31)) & 1u;
-            mx4[k & 3] = fmaxf(mx4[k & 3], on ? sgn * sv[k] : -CUDART_INF_F);
+            mn4[k & 3] = fminf(mn4[k & 3], on ? sv[k] : CUDART_INF_F);
           }
+          mx = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
+          mx = mx == CUDART_INF_F ? -CUDART_INF_F : mx;
         }
-        float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        mx = mx == -CUDART_INF_F ? mx : mx * (sgn * sc);  // scaled maximum
+        mx = mx == -CUDART_INF_F ? mx : mx * sc;  // scaled maximum
         float* px = xbuf + (xk & 1) * 256;
         px[half * 128 + r] = mx;
         exchange();
@@ -523,29 +559,38 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // (p = P_hi + P_lo to within 2^-15 of p); both are formed with integer
         // masks and byte permutes, leaving the multi-function unit to ex2.
         const float negm = m == -CUDART_INF_F ? 0.f : -m;
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+        // pairs of keys go through the packed fp32x2 FMA/add instructions
+        const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(negm, negm);
+        const float2 neg1 = make_float2(-1.f, -1.f);
+        float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pw[16];
 #pragma unroll
           for (int k = 0; k < 16; k += 2) {
             const int kk = c * 16 + k;
-            float p0 = exp2f(fmaf(sv[kk], sc, negm));
-            float p1 = exp2f(fmaf(sv[kk + 1], sc, negm));
+            const float2 x = __ffma2_rn(make_float2(sv[kk], sv[kk + 1]), sc2, nm2);
+            float p0 = (kExpFmaEvery > 0 && kk % kExpFmaEvery == kExpFmaEvery - 1) ? exp2_fma(x.x)
+                                                                                   : exp2f(x.x);
+            float p1 = (kExpFmaEvery > 0 && (kk + 1) % kExpFmaEvery == kExpFmaEvery - 1)
+                           ? exp2_fma(x.y)
+                           : exp2f(x.y);
             if (!all_vis) {
               p0 = ((vis[kk >> 5] >> (kk & 31)) & 1u) ? p0 : 0.f;
               p1 = ((vis[kk >> 5] >> ((kk + 1) & 31)) & 1u) ? p1 : 0.f;
             }
-            rs4[(k >> 1) & 3] += p0 + p1;
+            const float2 pp = make_float2(p0, p1);
+            rs2[(k >> 1) & 1] = __fadd2_rn(rs2[(k >> 1) & 1], pp);
             const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-            const float l0 = p0 - __uint_as_float(b0 & 0xffff0000u);
-            const float l1 = p1 - __uint_as_float(b1 & 0xffff0000u);
+            const float2 hi =
+                make_float2(__uint_as_float(b0 & 0xffff0000u), __uint_as_float(b1 & 0xffff0000u));
+            const float2 lo = __ffma2_rn(hi, neg1, pp);  // p - P_hi, exact
             pw[k >> 1] = __byte_perm(b0, b1, 0x7632);
-            pw[8 + (k >> 1)] = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
+            pw[8 + (k >> 1)] = __byte_perm(__float_as_uint(lo.x), __float_as_uint(lo.y), 0x7632);
           }
           tmem_st16_nowait(tmem + lane_addr + sb * 128 + cofs + c * 16, pw);
         }
-        const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        const float rs = (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
         tmem_wait_st();
         l += rs;
         // key rows past the context or in an unloaded page: zero this half of them in V
