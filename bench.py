@@ -470,17 +470,24 @@ def main():
 # 1,755,018,024 algorithmic bytes) scaled by algorithmic bytes to the full
 # 128-sequence batch; see profiles/decode_tc_gqa70b_long.md.
 TRAFFIC = {
-    "gqa70b_long": {"bytes": 4785697610, "sources": "b4a9199e941a"},
+    # 48-sequence capture of the same shape (1.0054 x its algorithmic bytes), scaled
+    "gqa70b_long": {"bytes": 4786146198, "sources": "f6f09991b9fa"},
+    # full-size captures
+    "llama13b_sampling": {"bytes": 2208505344, "sources": "f6f09991b9fa"},
+    "llama7b_decode": {"bytes": 1124766464, "sources": "f6f09991b9fa"},
 }
+
+
+# the sources the decode path's two kernels (plan, tensor-core decode) are built from
+DECODE_SOURCES = ("decode_plan.cu", "decode_tc.cu", "common.cuh", "tc_common.cuh")
 
 
 def kernel_source_digest():
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "paged_kv_cache_454_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        if f.startswith("decode") or f.endswith((".cuh", ".h")):
-            h.update(open(os.path.join(d, f), "rb").read())
+    for f in DECODE_SOURCES:
+        h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:12]
 
 
