@@ -23,3 +23,4 @@ from .paged_attention import (  # noqa: F401
     copy_blocks,
     CopyBlocksError,
 )
+from .kv_manager import KvManager, KvManagerError, NoBlocks  # noqa: F401,E402

@@ -14,7 +14,7 @@ Sources, by page title and section:
 * "vLLM 定位与核心机制详解", section 六.4 (chunked prefill: a long prompt is read
   a chunk per round; each chunk's tokens attend causally).
 
-Readings taken where the pages are silent (each is restated in the design doc):
+Readings taken where the pages are silent:
 
 * GQA: q head ``h`` reads KV head ``h // (Hq / Hkv)`` (contiguous groups).
 * A decode step's own new token is part of its context (``context_lens``
