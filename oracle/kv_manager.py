@@ -35,9 +35,9 @@ Readings taken where the pages are silent or leave a choice:
 * A cached block's identity is the full token sequence from position 0 to its
   last token.  Prefix-cache hits form a contiguous run from block 0 and stop
   at the first miss.  A full block is registered when it becomes full (at
-  allocation for a prompt, when its last slot is reserved during decode);
-  if that prefix is already cached by another block, the new block stays
-  unregistered.  The caller runs each step's prefill before the next step's
+  allocation for a prompt, when its last slot is reserved during decode) if
+  the prefix before it is cached (or it is block 0); if its own prefix is
+  already cached by another block, the new block stays unregistered.  The caller runs each step's prefill before the next step's
   lookups.
 * Prompt tokens found in the cache get slot -1 (nothing to write: the block is
   shared), the others their slot ``block * block_size + offset``.
@@ -126,9 +126,14 @@ class KvManager:
         self.ref[b] += 1
 
     def _register(self, b, prefix):
-        if self.prefix_caching and prefix not in self.cache:
-            self.cache[prefix] = b
-            self.prefix_of[b] = prefix
+        # only a block whose whole prefix is cached can ever be found (lookups
+        # start at position 0), so only such a block is registered
+        if not self.prefix_caching or prefix in self.cache:
+            return
+        if len(prefix) > self.bs and prefix[:-self.bs] not in self.cache:
+            return
+        self.cache[prefix] = b
+        self.prefix_of[b] = prefix
 
     def _need(self, n):
         if n > self.num_free_blocks():

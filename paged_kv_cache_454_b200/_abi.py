@@ -18,6 +18,7 @@ PA_ERR_SHAPE = 2
 PA_ERR_UNSUPPORTED = 3
 PA_ERR_WORKSPACE = 4
 PA_ERR_CUDA = 5
+PA_ERR_NO_BLOCKS = 6
 
 PA_DEV_ERR_BLOCK_ID = 0x1
 PA_DEV_ERR_SLOT = 0x2
@@ -58,6 +59,20 @@ SIGNATURES = {
     "pa_get_device_error": (c_int, [ctypes.POINTER(ctypes.c_uint32), c_vp]),
     "pa_status_string": (ctypes.c_char_p, [c_int]),
     "pa_abi_version": (c_int, []),
+    # host KV-cache block manager (include/pa_kv_manager.h)
+    "pa_kvm_create": (c_vp, [c_i32, c_i32, c_i32]),
+    "pa_kvm_destroy": (None, [c_vp]),
+    "pa_kvm_num_free_blocks": (c_i32, [c_vp]),
+    "pa_kvm_add_sequence": (c_int, [c_vp, c_i64, c_vp, c_i32, c_vp, c_vp]),
+    "pa_kvm_append_tokens": (c_int, [c_vp, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp]),
+    "pa_kvm_fork": (c_int, [c_vp, c_i64, c_i64]),
+    "pa_kvm_share_prefix": (c_int, [c_vp, c_i64, c_i64, c_i32]),
+    "pa_kvm_share_blocks": (c_int, [c_vp, c_i64, c_i64, c_vp, c_i32]),
+    "pa_kvm_free_sequence": (c_int, [c_vp, c_i64]),
+    "pa_kvm_sequence_info": (c_int, [c_vp, c_i64, c_vp, c_vp]),
+    "pa_kvm_block_table": (c_int, [c_vp, c_i64, c_vp, c_i32]),
+    "pa_kvm_batch": (c_int, [c_vp, c_vp, c_i32, c_i32, c_vp, c_vp]),
+    "pa_kvm_ref_count": (c_i32, [c_vp, c_i32]),
 }
 
 _lib = None

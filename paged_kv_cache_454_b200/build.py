@@ -33,12 +33,13 @@ def nvcc() -> str:
 
 
 def _sources():
-    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cpp")))
 
 
 def _headers():
     hs = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
-    hs.append(os.path.join(ROOT, "include", "pa.h"))
+    inc = os.path.join(ROOT, "include")
+    hs += [os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h")]
     return sorted(hs)
 
 
@@ -53,7 +54,8 @@ def _digest(src: str, extra: list) -> str:
 
 def _compile(src: str, ptxas_info: bool, verbose: bool) -> str:
     extra = ARCH + NVCC_FLAGS + (["-Xptxas", "-v"] if ptxas_info else [])
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + "-" + _digest(src, extra) + ".o")
+    obj = os.path.join(BUILD, os.path.splitext(os.path.basename(src))[0] + "-" +
+                       _digest(src, extra) + ".o")
     if os.path.exists(obj) and not ptxas_info:
         return obj
     cmd = [nvcc(), "-c", src, "-o", obj] + extra

@@ -4,6 +4,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "../../include/pa_kv_manager.h"
 
 namespace pa {
 
@@ -319,6 +320,7 @@ const char* pa_status_string(int status) {
     case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: size not compiled";
     case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace missing or too small";
     case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime or launch failure";
+    case PA_ERR_NO_BLOCKS: return "PA_ERR_NO_BLOCKS: too few free blocks in the pool";
     default: return "unknown status";
   }
 }

@@ -1,0 +1,126 @@
+"""Python handle on the library's host KV-cache block manager (``pa_kvm_*``,
+declared in ``include/pa_kv_manager.h``).
+
+Argument marshalling only: every decision (allocation, reference counts,
+copy-on-write pairs, prefix-cache lookups) is made by the C++ manager in
+``libpa.so``.  Method names follow the C calls without the prefix.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import _abi
+
+
+class KvManagerError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = _abi.load().pa_status_string(status)
+        super().__init__(f"{fn} failed: {msg.decode() if msg else status}")
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+class KvManager:
+    """One pool of ``num_blocks`` blocks of ``block_size`` token slots."""
+
+    def __init__(self, num_blocks: int, block_size: int = 16, prefix_caching: bool = False):
+        self._lib = _abi.load()
+        self._h = self._lib.pa_kvm_create(num_blocks, block_size, 1 if prefix_caching else 0)
+        if not self._h:
+            raise ValueError("pa_kvm_create failed (bad sizes or out of memory)")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        self.prefix_caching = prefix_caching
+
+    def close(self):
+        if self._h:
+            self._lib.pa_kvm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 -- interpreter shutdown
+            pass
+
+    def _check(self, fn, st):
+        if st != _abi.PA_OK:
+            raise KvManagerError(fn, st)
+
+    # ------------------------------------------------------------------ calls
+    def num_free_blocks(self) -> int:
+        return self._lib.pa_kvm_num_free_blocks(self._h)
+
+    def add_sequence(self, seq_id: int, tokens):
+        """Returns (slots int64[n], cached_tokens)."""
+        t = _i32(tokens)
+        slots = np.empty(len(t), np.int64)
+        cached = ctypes.c_int32(0)
+        self._check("pa_kvm_add_sequence",
+                    self._lib.pa_kvm_add_sequence(self._h, seq_id, _p(t), len(t), _p(slots),
+                                                  ctypes.byref(cached)))
+        return slots, cached.value
+
+    def append_tokens(self, seq_id: int, tokens):
+        """Returns (slots int64[n], copy pairs as a list of (src, dst))."""
+        t = _i32(tokens)
+        slots = np.empty(len(t), np.int64)
+        pair = np.empty(2, np.int64)
+        npairs = ctypes.c_int32(0)
+        self._check("pa_kvm_append_tokens",
+                    self._lib.pa_kvm_append_tokens(self._h, seq_id, _p(t), len(t), _p(slots),
+                                                   _p(pair), ctypes.byref(npairs)))
+        return slots, [(int(pair[0]), int(pair[1]))] if npairs.value else []
+
+    def fork(self, parent: int, child: int):
+        self._check("pa_kvm_fork", self._lib.pa_kvm_fork(self._h, parent, child))
+
+    def share_prefix(self, src: int, dst: int, n_blocks: int):
+        self._check("pa_kvm_share_prefix", self._lib.pa_kvm_share_prefix(self._h, src, dst, n_blocks))
+
+    def share_blocks(self, src: int, dst: int, idx):
+        i = _i32(idx)
+        self._check("pa_kvm_share_blocks",
+                    self._lib.pa_kvm_share_blocks(self._h, src, dst, _p(i), len(i)))
+
+    def free_sequence(self, seq_id: int):
+        self._check("pa_kvm_free_sequence", self._lib.pa_kvm_free_sequence(self._h, seq_id))
+
+    def sequence_info(self, seq_id: int):
+        """Returns (context_len, num_blocks)."""
+        L, nb = ctypes.c_int32(0), ctypes.c_int32(0)
+        self._check("pa_kvm_sequence_info",
+                    self._lib.pa_kvm_sequence_info(self._h, seq_id, ctypes.byref(L),
+                                                   ctypes.byref(nb)))
+        return L.value, nb.value
+
+    def context_len(self, seq_id: int) -> int:
+        return self.sequence_info(seq_id)[0]
+
+    def block_table(self, seq_id: int) -> list:
+        _, nb = self.sequence_info(seq_id)
+        t = np.empty(max(nb, 1), np.int32)
+        self._check("pa_kvm_block_table", self._lib.pa_kvm_block_table(self._h, seq_id, _p(t), nb))
+        return [int(x) for x in t[:nb]]
+
+    def batch(self, seq_ids, max_blocks: int):
+        """Decode inputs of a batch: (block_tables int32[S, max_blocks], context_lens int32[S])."""
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+        tables = np.empty((len(ids), max_blocks), np.int32)
+        lens = np.empty(len(ids), np.int32)
+        self._check("pa_kvm_batch",
+                    self._lib.pa_kvm_batch(self._h, _p(ids), len(ids), max_blocks, _p(tables),
+                                           _p(lens)))
+        return tables, lens
+
+    def ref_count(self, block: int) -> int:
+        return self._lib.pa_kvm_ref_count(self._h, block)

@@ -1,4 +1,4 @@
-"""The C-ABI library loads without a GPU, exports every symbol ``include/pa.h``
+"""The C-ABI library loads without a GPU, exports every symbol ``include/*.h``
 declares, and rejects bad arguments on the host before any CUDA call."""
 import ctypes
 import os
@@ -10,12 +10,16 @@ import pytest
 from paged_kv_cache_454_b200 import _abi
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "pa.h")
+INCLUDE = os.path.join(ROOT, "include")
 
 
 def declared_symbols():
-    text = open(HEADER).read()
-    return sorted(set(re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text)))
+    names = set()
+    for f in sorted(os.listdir(INCLUDE)):
+        if f.endswith(".h"):
+            text = open(os.path.join(INCLUDE, f)).read()
+            names |= set(re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
@@ -26,7 +30,8 @@ def lib():
 def test_header_declares_the_boundary():
     names = declared_symbols()
     for n in ("pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
-              "pa_chunked_prefill", "pa_gather_kv", "pa_get_device_error"):
+              "pa_chunked_prefill", "pa_gather_kv", "pa_get_device_error", "pa_kvm_create",
+              "pa_kvm_add_sequence", "pa_kvm_append_tokens", "pa_kvm_batch"):
         assert n in names
 
 
