@@ -206,6 +206,38 @@ class Workload:
         return n
 
 
+def host_manager_timing(w: Workload, steps: int = 100):
+    """Host time of the C++ block manager for this batch's decode steps,
+    through the Python binding: every step reserves one new token's slot for
+    each decode sequence (``pa_kvm_decode_step``) and brings the batch's block
+    tables and lengths up to date (``pa_kvm_batch_update``; the full tables are
+    built once before).  No device work."""
+    from paged_kv_cache_454_b200.kv_manager import KvManager
+    lay = w.layout
+    if not len(w.dec):
+        return None
+    lens = lay.context_lens[w.dec].astype(np.int64)
+    S = len(lens)
+    max_blocks = int(-(-(int(lens.max()) + steps) // lay.block_size))
+    blocks = int(sum(-(-(int(x) + steps) // lay.block_size) for x in lens))
+    m = KvManager(blocks, lay.block_size, prefix_caching=False)
+    ids = np.arange(S, dtype=np.int64)
+    for i in range(S):
+        m.add_sequence(i, np.zeros(max(int(lens[i]) - 1, 0), np.int32))
+    toks = np.zeros(S, np.int32)
+    slots = np.empty(S, np.int64)
+    out = (np.empty((S, max_blocks), np.int32), np.empty(S, np.int32))
+    m.batch(ids, max_blocks, out=out)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        m.decode_step(ids, toks, slots=slots)
+        m.batch_update(ids, out)
+    us = (time.perf_counter() - t0) / steps * 1e6
+    m.close()
+    return {"us_per_step": round(us, 2), "num_seqs": S, "steps": steps,
+            "calls": "pa_kvm_decode_step + pa_kvm_batch_update", "threads": 1}
+
+
 def e2e_run(w: Workload, stream, steps, warmup):
     """The same step through the public API with host buffers: per step, pinned
     host -> device copies of the step's inputs (q, new K/V, slot mapping, block
@@ -455,6 +487,7 @@ def main():
         "e2e": e2e,
         "gpu_launches": w.launches_per_step() * a.steps,
         "clocks": clk,
+        "host_block_manager": host_manager_timing(w) if rank == 0 else None,
     }
     if rank == 0:
         print(json.dumps(res), flush=True)
@@ -466,9 +499,9 @@ def main():
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # decode kernel from an ncu capture, keyed by workload and the kernel sources
 # it was taken with (reported as null once those sources change).  The
-# gqa70b_long figure is the 48-sequence capture (1,764,291,328 bytes for
+# gqa70b_long figure is the 48-sequence capture (1,764,456,704 bytes for
 # 1,755,018,024 algorithmic bytes) scaled by algorithmic bytes to the full
-# 128-sequence batch; see profiles/decode_tc_gqa70b_long.md.
+# 128-sequence batch; the captures are summarised in profiles/.
 TRAFFIC = {
     # 48-sequence capture of the same shape (1.0054 x its algorithmic bytes), scaled
     "gqa70b_long": {"bytes": 4786146198, "sources": "f6f09991b9fa"},

@@ -96,6 +96,20 @@ PA_API int pa_kvm_add_sequence(pa_kvm* m, int64_t seq_id, const int32_t* tokens,
 PA_API int pa_kvm_append_tokens(pa_kvm* m, int64_t seq_id, const int32_t* tokens, int32_t n,
                                 int64_t* slots, int64_t* copy_pair, int32_t* num_pairs);
 
+/*
+ * pa_kvm_decode_step -- one new token for each of num_seqs sequences, in order
+ * (the same as pa_kvm_append_tokens with n = 1 for each), all or nothing for
+ * the whole batch.
+ *   tokens      int32 [num_seqs] (may be NULL when prefix caching is off).
+ *   slots       int64 [num_seqs], out: pa_reshape_and_cache's slot_mapping.
+ *   copy_pairs  int64 [num_seqs][2], out: the copies to run first, packed;
+ *               *num_pairs of them.
+ * PA_ERR_ARG also for a sequence listed twice.
+ */
+PA_API int pa_kvm_decode_step(pa_kvm* m, const int64_t* seq_ids, int32_t num_seqs,
+                              const int32_t* tokens, int64_t* slots, int64_t* copy_pairs,
+                              int32_t* num_pairs);
+
 /* pa_kvm_fork -- new sequence `child` sharing every block of `parent`. */
 PA_API int pa_kvm_fork(pa_kvm* m, int64_t parent, int64_t child);
 
@@ -132,6 +146,15 @@ PA_API int pa_kvm_block_table(const pa_kvm* m, int64_t seq_id, int32_t* table, i
  */
 PA_API int pa_kvm_batch(const pa_kvm* m, const int64_t* seq_ids, int32_t num_seqs,
                         int32_t max_blocks, int32_t* block_tables, int32_t* context_lens);
+
+/*
+ * pa_kvm_batch_update -- the same for arrays that already hold this batch's
+ * tables as they were before the last pa_kvm_decode_step of these sequences
+ * (same order): a decode step changes only a sequence's last table entry (a
+ * new block, or its copy), so only that entry and the length are written.
+ */
+PA_API int pa_kvm_batch_update(const pa_kvm* m, const int64_t* seq_ids, int32_t num_seqs,
+                               int32_t max_blocks, int32_t* block_tables, int32_t* context_lens);
 
 /* Tables referencing `block`, or -1 when it is out of range. */
 PA_API int32_t pa_kvm_ref_count(const pa_kvm* m, int32_t block);

@@ -208,6 +208,30 @@ class KvManager:
         s["len"] = L
         return slots, pairs
 
+    def decode_step(self, sids, tokens):
+        """One new token for each of ``sids`` (in order), all or nothing.
+        Returns (slots, copy_pairs)."""
+        if len(set(sids)) != len(sids):
+            raise KvManagerError("a sequence listed twice")
+        need, drops = 0, {}
+        for sid in sids:
+            st = self._seq(sid)
+            L = st["len"]
+            if L % self.bs == 0:
+                need += 1
+            else:
+                b = st["table"][-1]
+                if self.ref[b] - drops.get(b, 0) > 1:   # shared: a copy
+                    need += 1
+                    drops[b] = drops.get(b, 0) + 1
+        self._need(need)
+        slots, pairs = [], []
+        for sid, t in zip(sids, tokens):
+            sl, pr = self.append_tokens(sid, [t])
+            slots += sl
+            pairs += pr
+        return slots, pairs
+
     def fork(self, parent, child):
         """Whole-sequence sharing: ``child`` holds every block of ``parent``."""
         p = self._seq(parent)

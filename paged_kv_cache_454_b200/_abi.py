@@ -65,6 +65,7 @@ SIGNATURES = {
     "pa_kvm_num_free_blocks": (c_i32, [c_vp]),
     "pa_kvm_add_sequence": (c_int, [c_vp, c_i64, c_vp, c_i32, c_vp, c_vp]),
     "pa_kvm_append_tokens": (c_int, [c_vp, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp]),
+    "pa_kvm_decode_step": (c_int, [c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "pa_kvm_fork": (c_int, [c_vp, c_i64, c_i64]),
     "pa_kvm_share_prefix": (c_int, [c_vp, c_i64, c_i64, c_i32]),
     "pa_kvm_share_blocks": (c_int, [c_vp, c_i64, c_i64, c_vp, c_i32]),
@@ -72,6 +73,7 @@ SIGNATURES = {
     "pa_kvm_sequence_info": (c_int, [c_vp, c_i64, c_vp, c_vp]),
     "pa_kvm_block_table": (c_int, [c_vp, c_i64, c_vp, c_i32]),
     "pa_kvm_batch": (c_int, [c_vp, c_vp, c_i32, c_i32, c_vp, c_vp]),
+    "pa_kvm_batch_update": (c_int, [c_vp, c_vp, c_i32, c_i32, c_vp, c_vp]),
     "pa_kvm_ref_count": (c_i32, [c_vp, c_i32]),
 }
 

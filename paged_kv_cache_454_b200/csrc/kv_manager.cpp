@@ -85,6 +85,7 @@ class IdSet {
 struct Seq {
   std::vector<int32_t> table;
   int32_t len = 0;
+  uint64_t stamp = 0;           // last batch call that listed this sequence
   std::vector<int32_t> tokens;  // kept only with prefix caching
   std::vector<uint64_t> hash;   // chain hash of each full block (prefix caching)
 };
@@ -106,6 +107,7 @@ struct pa_kvm {
   std::vector<uint64_t> bhash, bparent;
   std::vector<std::vector<int32_t>> btokens, children;
   std::unordered_map<int64_t, Seq> seqs;
+  uint64_t calls = 0;  // batch-call counter (duplicate detection)
 
   pa_kvm(int32_t n, int32_t b, bool p)
       : nb(n), bs(b), pc(p), ref(n, 0), free_set(n), prev(n, -1), next(n, -1), in_lru(n, 0),
@@ -208,6 +210,42 @@ struct pa_kvm {
 
   uint64_t parent_hash(const Seq& s, int32_t i) const { return i == 0 ? kRoot : s.hash[i - 1]; }
 
+  // Blocks appending n tokens to s takes from the pool (a copy of a shared
+  // partial last block, then fresh blocks).
+  int32_t blocks_needed(const Seq& s, int32_t n, bool* cow) const {
+    *cow = n > 0 && s.len % bs != 0 && ref[s.table.back()] > 1;
+    return (s.len + n + bs - 1) / bs - (s.len + bs - 1) / bs + (*cow ? 1 : 0);
+  }
+
+  // Append n tokens to s; the caller has checked the pool can supply the blocks.
+  void append(Seq& s, const int32_t* tokens, int32_t n, bool cow, int64_t* slots,
+              int64_t* pair, int32_t* num_pairs) {
+    int32_t L = s.len;
+    if (cow) {
+      const int32_t old = s.table.back();
+      const int32_t fresh = alloc();
+      release(old);
+      s.table.back() = fresh;
+      pair[0] = old;
+      pair[1] = fresh;
+      ++*num_pairs;
+    }
+    for (int32_t t = 0; t < n; ++t) {
+      if (L % bs == 0) s.table.push_back(alloc());
+      slots[t] = static_cast<int64_t>(s.table[L / bs]) * bs + L % bs;
+      if (pc) s.tokens.push_back(tokens[t]);
+      ++L;
+      if (pc && L % bs == 0) {
+        const int32_t k = L / bs - 1;
+        const uint64_t parent = parent_hash(s, k);
+        const uint64_t h = chain_hash(parent, s.tokens.data() + k * bs, bs);
+        s.hash.push_back(h);
+        reg(s.table[k], k, h, parent, s.tokens.data() + k * bs);
+      }
+    }
+    s.len = L;
+  }
+
   // Chain hashes of s's full blocks from block `from` on (after its tokens changed).
   void rehash(Seq& s, int32_t from) {
     if (!pc) return;
@@ -286,37 +324,53 @@ PA_API int pa_kvm_append_tokens(pa_kvm* m, int64_t seq_id, const int32_t* tokens
   auto it = m->seqs.find(seq_id);
   if (it == m->seqs.end()) return PA_ERR_ARG;
   Seq& s = it->second;
-  const int32_t bs = m->bs;
-  int32_t L = s.len;
   *num_pairs = 0;
   if (n == 0) return PA_OK;
-  const bool cow = L % bs != 0 && m->ref[s.table.back()] > 1;
+  bool cow = false;
+  const int32_t need = m->blocks_needed(s, n, &cow);
   if (cow && !copy_pair) return PA_ERR_ARG;
-  const int32_t new_blocks = (L + n + bs - 1) / bs - (L + bs - 1) / bs;
-  if (new_blocks + (cow ? 1 : 0) > m->num_free()) return PA_ERR_NO_BLOCKS;
-  if (cow) {
-    const int32_t old = s.table.back();
-    const int32_t fresh = m->alloc();
-    m->release(old);
-    s.table.back() = fresh;
-    copy_pair[0] = old;
-    copy_pair[1] = fresh;
-    *num_pairs = 1;
-  }
-  for (int32_t t = 0; t < n; ++t) {
-    if (L % bs == 0) s.table.push_back(m->alloc());
-    slots[t] = static_cast<int64_t>(s.table[L / bs]) * bs + L % bs;
-    if (m->pc) s.tokens.push_back(tokens[t]);
-    ++L;
-    if (m->pc && L % bs == 0) {
-      const int32_t k = L / bs - 1;
-      const uint64_t parent = m->parent_hash(s, k);
-      const uint64_t h = chain_hash(parent, s.tokens.data() + k * bs, bs);
-      s.hash.push_back(h);
-      m->reg(s.table[k], k, h, parent, s.tokens.data() + k * bs);
+  if (need > m->num_free()) return PA_ERR_NO_BLOCKS;
+  m->append(s, tokens, n, cow, slots, copy_pair, num_pairs);
+  return PA_OK;
+}
+
+PA_API int pa_kvm_decode_step(pa_kvm* m, const int64_t* seq_ids, int32_t num_seqs,
+                              const int32_t* tokens, int64_t* slots, int64_t* copy_pairs,
+                              int32_t* num_pairs) {
+  if (!m || num_seqs < 0 || !num_pairs ||
+      (num_seqs > 0 && (!seq_ids || !slots || !copy_pairs || (m->pc && !tokens))))
+    return PA_ERR_ARG;
+  *num_pairs = 0;
+  std::vector<Seq*> ss(num_seqs);
+  std::unordered_map<int32_t, int32_t> drops;  // references an earlier copy in the batch drops
+  const uint64_t stamp = ++m->calls;
+  int32_t need = 0;
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    auto it = m->seqs.find(seq_ids[i]);
+    if (it == m->seqs.end() || it->second.stamp == stamp) return PA_ERR_ARG;
+    Seq& s = it->second;
+    s.stamp = stamp;
+    ss[i] = &s;
+    if (s.len % m->bs == 0) {
+      ++need;
+    } else {
+      const int32_t b = s.table.back();
+      if (m->ref[b] > 1) {  // shared: copied unless earlier copies left one holder
+        int32_t& d = drops[b];
+        if (m->ref[b] - d > 1) {
+          ++need;
+          ++d;
+        }
+      }
     }
   }
-  s.len = L;
+  if (need > m->num_free()) return PA_ERR_NO_BLOCKS;
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    bool cow = false;
+    m->blocks_needed(*ss[i], 1, &cow);
+    m->append(*ss[i], tokens ? tokens + i : nullptr, 1, cow, slots + i,
+              copy_pairs + 2 * *num_pairs, num_pairs);
+  }
   return PA_OK;
 }
 
@@ -424,6 +478,23 @@ PA_API int pa_kvm_batch(const pa_kvm* m, const int64_t* seq_ids, int32_t num_seq
     const int32_t nt = static_cast<int32_t>(s.table.size());
     std::copy(s.table.begin(), s.table.end(), row);
     for (int32_t j = nt; j < max_blocks; ++j) row[j] = -1;
+    context_lens[i] = s.len;
+  }
+  return PA_OK;
+}
+
+PA_API int pa_kvm_batch_update(const pa_kvm* m, const int64_t* seq_ids, int32_t num_seqs,
+                               int32_t max_blocks, int32_t* block_tables, int32_t* context_lens) {
+  if (!m || num_seqs < 0 || max_blocks < 0 ||
+      (num_seqs > 0 && (!seq_ids || !context_lens || (max_blocks > 0 && !block_tables))))
+    return PA_ERR_ARG;
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    auto it = m->seqs.find(seq_ids[i]);
+    if (it == m->seqs.end()) return PA_ERR_ARG;
+    const Seq& s = it->second;
+    const int32_t nt = static_cast<int32_t>(s.table.size());
+    if (nt > max_blocks) return PA_ERR_SHAPE;
+    if (nt > 0) block_tables[static_cast<int64_t>(i) * max_blocks + nt - 1] = s.table.back();
     context_lens[i] = s.len;
   }
   return PA_OK;

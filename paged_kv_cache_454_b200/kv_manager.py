@@ -81,6 +81,22 @@ class KvManager:
                                                    _p(pair), ctypes.byref(npairs)))
         return slots, [(int(pair[0]), int(pair[1]))] if npairs.value else []
 
+    def decode_step(self, seq_ids, tokens, slots=None):
+        """One new token per sequence, all or nothing.  Returns (slots int64[S],
+        copy pairs as a list of (src, dst)); ``slots`` may be given to fill."""
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+        t = _i32(tokens)
+        if slots is None:
+            slots = np.empty(len(ids), np.int64)
+        elif slots.shape != (len(ids),) or slots.dtype != np.int64:
+            raise ValueError("slots does not match the batch")
+        pairs = np.empty((max(len(ids), 1), 2), np.int64)
+        npairs = ctypes.c_int32(0)
+        self._check("pa_kvm_decode_step",
+                    self._lib.pa_kvm_decode_step(self._h, _p(ids), len(ids), _p(t), _p(slots),
+                                                 _p(pairs), ctypes.byref(npairs)))
+        return slots, [(int(a), int(b)) for a, b in pairs[:npairs.value]]
+
     def fork(self, parent: int, child: int):
         self._check("pa_kvm_fork", self._lib.pa_kvm_fork(self._h, parent, child))
 
@@ -112,14 +128,37 @@ class KvManager:
         self._check("pa_kvm_block_table", self._lib.pa_kvm_block_table(self._h, seq_id, _p(t), nb))
         return [int(x) for x in t[:nb]]
 
-    def batch(self, seq_ids, max_blocks: int):
-        """Decode inputs of a batch: (block_tables int32[S, max_blocks], context_lens int32[S])."""
+    def batch(self, seq_ids, max_blocks: int, out=None):
+        """Decode inputs of a batch: (block_tables int32[S, max_blocks], context_lens int32[S]).
+        ``out``: optional (tables, lens) arrays of those shapes to fill instead."""
         ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
-        tables = np.empty((len(ids), max_blocks), np.int32)
-        lens = np.empty(len(ids), np.int32)
+        if out is None:
+            tables = np.empty((len(ids), max_blocks), np.int32)
+            lens = np.empty(len(ids), np.int32)
+        else:
+            tables, lens = out
+            if (tables.shape != (len(ids), max_blocks) or tables.dtype != np.int32
+                    or not tables.flags.c_contiguous or lens.shape != (len(ids),)
+                    or lens.dtype != np.int32):
+                raise ValueError("out arrays do not match the batch")
         self._check("pa_kvm_batch",
                     self._lib.pa_kvm_batch(self._h, _p(ids), len(ids), max_blocks, _p(tables),
                                            _p(lens)))
+        return tables, lens
+
+    def batch_update(self, seq_ids, out):
+        """Bring ``out`` = (tables, lens) from ``batch`` up to date after a
+        ``decode_step`` of the same sequences in the same order (writes only
+        each sequence's last table entry and its length)."""
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+        tables, lens = out
+        if (tables.ndim != 2 or tables.shape[0] != len(ids) or tables.dtype != np.int32
+                or not tables.flags.c_contiguous or lens.shape != (len(ids),)
+                or lens.dtype != np.int32):
+            raise ValueError("out arrays do not match the batch")
+        self._check("pa_kvm_batch_update",
+                    self._lib.pa_kvm_batch_update(self._h, _p(ids), len(ids), tables.shape[1],
+                                                  _p(tables), _p(lens)))
         return tables, lens
 
     def ref_count(self, block: int) -> int:

@@ -64,6 +64,30 @@ def lay_shared_many():
     return lay
 
 
+def lay_gqa4():
+    # group 4: two KV heads share a tile (4 KiB copies)
+    return synth.build_layout("gqa4", 113, [1, 40, 700, 1500, 3000], num_q_heads=16,
+                              num_kv_heads=4, head_dim=128)
+
+
+def lay_gqa2_h6():
+    # group 2 over 6 KV heads: tiles of 2 heads (4 does not divide 6)
+    return synth.build_layout("gqa2_h6", 114, [3, 129, 900, 2100], num_q_heads=12,
+                              num_kv_heads=6, head_dim=128)
+
+
+def lay_mha_h5():
+    # one q head per KV head, 5 KV heads: one head per tile
+    return synth.build_layout("mha_h5", 115, [2, 17, 300, 1300], num_q_heads=5,
+                              num_kv_heads=5, head_dim=128)
+
+
+def lay_mha_h16():
+    # 16 KV heads: two tiles of 8 heads per page
+    return synth.build_layout("mha_h16", 116, [1, 16, 33, 1000, 2500], num_q_heads=16,
+                              num_kv_heads=16, head_dim=128)
+
+
 def lay_mixed(hq=10, hkv=2, d=128):
     # prefill chunks: fresh prompt, short cache, long cache with a ragged chunk;
     # plus two decode sequences
@@ -94,6 +118,10 @@ DECODE_LAYOUTS = {
     "g16": lay_g16,
     "shared_prefix": lay_shared,
     "shared_many": lay_shared_many,
+    "gqa4": lay_gqa4,
+    "gqa2_h6": lay_gqa2_h6,
+    "mha_h5": lay_mha_h5,
+    "mha_h16": lay_mha_h16,
     "short_gqa": lay_short_gqa,
     "short_mha": lay_short_mha,
 }
@@ -191,7 +219,8 @@ def test_decode_simt(name, partition):
 
 
 @pytest.mark.parametrize("name", ["gqa8", "gqa5", "g16", "shared_prefix", "shared_many", "mha128",
-                                  "short_gqa", "short_mha"])
+                                  "short_gqa", "short_mha", "gqa4", "gqa2_h6", "mha_h5",
+                                  "mha_h16"])
 @pytest.mark.parametrize("partition", [0, 128, 1024, 1 << 20])
 def test_decode_tcgen05(name, partition):
     st, ref = _step_and_ref(name)

@@ -25,6 +25,9 @@ def run(target, op):
         if kind == "append":
             slots, pairs = target.append_tokens(op[1], op[2])
             return ("ok", [int(s) for s in slots], [tuple(map(int, p)) for p in pairs])
+        if kind == "step":
+            slots, pairs = target.decode_step(op[1], op[2])
+            return ("ok", [int(s) for s in slots], [tuple(map(int, p)) for p in pairs])
         if kind == "fork":
             target.fork(op[1], op[2])
         elif kind == "share_prefix":
@@ -131,3 +134,20 @@ def test_without_prefix_caching_tokens_may_be_omitted():
         assert list(slots)[:3] == [6, 7, 8] and npairs.value == 0
     finally:
         lib.pa_kvm_destroy(h)
+
+
+def test_batch_update_tracks_decode_steps():
+    m = KvManager(400, 16, prefix_caching=False)
+    rng = np.random.default_rng(3)
+    ids = list(range(12))
+    for i in ids:
+        m.add_sequence(i, np.zeros(int(rng.integers(1, 60)), np.int32))
+    for i in (1, 2, 3):
+        m.fork(0, 100 + i)          # shared partial blocks: steps copy them
+    ids += [101, 102, 103]
+    out = m.batch(ids, 12)
+    for step in range(40):
+        _, pairs = m.decode_step(ids, np.zeros(len(ids), np.int32))
+        m.batch_update(ids, out)
+        full = m.batch(ids, 12)
+        assert np.array_equal(out[0], full[0]) and np.array_equal(out[1], full[1]), step

@@ -49,6 +49,14 @@ class Sim:
         self.expect[sid] += list(tokens)
         return slots, pairs
 
+    def step(self, sids, tokens):
+        slots, pairs = self.m.decode_step(sids, tokens)
+        self._copy(pairs)
+        self._write(slots, tokens)
+        for sid, t in zip(sids, tokens):
+            self.expect[sid].append(t)
+        return slots, pairs
+
     def fork(self, p, c):
         self.m.fork(p, c)
         self.expect[c] = list(self.expect[p])
@@ -250,6 +258,11 @@ def random_ops(seed, n_ops, num_blocks, bs, prefix_caching):
         elif r < 0.6:
             ops.append(("append", rng.choice(live),
                         [rng.randrange(4) for _ in range(rng.choice([1, 1, 1, 3, bs + 1]))]))
+        elif r < 0.66:
+            ids = rng.sample(live, rng.randrange(1, len(live) + 1))
+            if rng.random() < 0.1:
+                ids.append(ids[0])            # a duplicate: rejected
+            ops.append(("step", ids, [rng.randrange(4) for _ in ids]))
         elif r < 0.7:
             ops.append(("fork", rng.choice(live), next_id))
             live.append(next_id)
@@ -276,6 +289,8 @@ def apply_op(target, op):
             return target.add(op[1], op[2])
         if kind == "append":
             return target.append(op[1], op[2])
+        if kind == "step":
+            return target.step(op[1], op[2])
         if kind == "fork":
             return target.fork(op[1], op[2])
         if kind == "share_prefix":
