@@ -24,3 +24,4 @@ from .paged_attention import (  # noqa: F401
     CopyBlocksError,
 )
 from .kv_manager import KvManager, KvManagerError, NoBlocks  # noqa: F401,E402
+from . import sampler  # noqa: F401,E402
