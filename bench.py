@@ -238,6 +238,38 @@ def host_manager_timing(w: Workload, steps: int = 100):
             "calls": "pa_kvm_decode_step + pa_kvm_batch_update", "threads": 1}
 
 
+def sampler_timing(w: Workload, stream, reps: int = 50):
+    """Device time of the fused sampler (``pa_sample``) for this batch's decode
+    rows at two vocabulary sizes (32000, 152064), temperature 0.7, top-k 50,
+    top-p 0.9; CUDA events over ``reps`` back-to-back calls after warm-up."""
+    torch = w.torch
+    rows = len(w.dec) if len(w.dec) else 1
+    res = {}
+    g = torch.Generator(device=w.dev)
+    g.manual_seed(0)
+    for vocab in (32000, 152064):
+        x = torch.randn(rows, vocab, device=w.dev, generator=g) * 3
+        T = torch.full((rows,), 0.7, device=w.dev)
+        K = torch.full((rows,), 50, dtype=torch.int32, device=w.dev)
+        P = torch.full((rows,), 0.9, device=w.dev)
+        u = torch.rand(rows, device=w.dev, generator=g)
+        out = torch.empty(rows, dtype=torch.int32, device=w.dev)
+        with torch.cuda.stream(stream):
+            for _ in range(5):
+                w.pa.pa_sample(x, T, K, P, u, out=out, stream=stream)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                w.pa.pa_sample(x, T, K, P, u, out=out, stream=stream)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        res[str(vocab)] = round(e0.elapsed_time(e1) / reps * 1e3, 2)
+    return {"us_per_call": res, "rows": rows, "temperature": 0.7, "top_k": 50, "top_p": 0.9,
+            "logits_gb_per_s": {k: round(rows * int(k) * 4 / (v * 1e-6) / 1e9, 1)
+                                for k, v in res.items()}}
+
+
 def e2e_run(w: Workload, stream, steps, warmup):
     """The same step through the public API with host buffers: per step, pinned
     host -> device copies of the step's inputs (q, new K/V, slot mapping, block
@@ -488,6 +520,7 @@ def main():
         "gpu_launches": w.launches_per_step() * a.steps,
         "clocks": clk,
         "host_block_manager": host_manager_timing(w) if rank == 0 else None,
+        "fused_sampler": sampler_timing(w, stream) if rank == 0 else None,
     }
     if rank == 0:
         print(json.dumps(res), flush=True)

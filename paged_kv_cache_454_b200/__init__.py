@@ -19,7 +19,7 @@ from ._abi import (PA_DEV_ERR_BLOCK_ID, PA_DEV_ERR_CONTEXT, PA_DEV_ERR_SLOT,  # 
 __all__ = [
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
     "pa_decode_noalloc",
-    "pa_chunked_prefill", "pa_gather_kv", "pa_get_device_error", "pool_desc", "lib",
+    "pa_chunked_prefill", "pa_gather_kv", "pa_get_device_error", "pa_sample", "pool_desc", "lib",
     "PaError", "PA_KERNEL_AUTO", "PA_KERNEL_SIMT", "PA_KERNEL_TCGEN05",
 ]
 
@@ -216,3 +216,26 @@ def pa_get_device_error(stream=None) -> int:
     v = ctypes.c_uint32(0)
     _abi.check("pa_get_device_error", lib().pa_get_device_error(ctypes.byref(v), _stream(stream)))
     return int(v.value)
+
+
+def pa_sample(logits, temperature, top_k, top_p, uniform, out=None, stream=None):
+    """Fused temperature / Top-K / Top-P sampling, one token per row of ``logits``
+    (fp32 [rows, vocab], rows contiguous).  ``temperature``, ``top_p``, ``uniform``:
+    fp32 [rows]; ``top_k``: int32 [rows]; all CUDA tensors.  Returns int32 [rows]."""
+    torch = _torch()
+    _need_cuda("logits", logits, torch.float32, contiguous=False)
+    if logits.dim() != 2 or logits.stride(1) != 1:
+        raise ValueError("logits must be [rows, vocab] with unit stride along the vocabulary")
+    rows, vocab = logits.shape
+    for name, t, dt in (("temperature", temperature, torch.float32), ("top_k", top_k, torch.int32),
+                        ("top_p", top_p, torch.float32), ("uniform", uniform, torch.float32)):
+        _need_cuda(name, t, dt)
+        if t.shape != (rows,):
+            raise ValueError(f"{name} must have shape ({rows},)")
+    if out is None:
+        out = torch.empty(rows, dtype=torch.int32, device=logits.device)
+    _need_cuda("out", out, torch.int32)
+    _abi.check("pa_sample", lib().pa_sample(
+        _ptr(logits), logits.stride(0), rows, vocab, _ptr(temperature), _ptr(top_k),
+        _ptr(top_p), _ptr(uniform), _ptr(out), _stream(stream)))
+    return out

@@ -59,6 +59,8 @@ SIGNATURES = {
     "pa_get_device_error": (c_int, [ctypes.POINTER(ctypes.c_uint32), c_vp]),
     "pa_status_string": (ctypes.c_char_p, [c_int]),
     "pa_abi_version": (c_int, []),
+    # fused sampler (include/pa_sampler.h)
+    "pa_sample": (c_int, [c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     # host KV-cache block manager (include/pa_kv_manager.h)
     "pa_kvm_create": (c_vp, [c_i32, c_i32, c_i32]),
     "pa_kvm_destroy": (None, [c_vp]),

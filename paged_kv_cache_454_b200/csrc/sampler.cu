@@ -1,0 +1,460 @@
+// Fused next-token sampling: temperature, Top-K, Top-P and the draw in one
+// kernel, one CTA per row, without sorting the vocabulary ("vLLM 基本原理",
+// FlashInfer 采样器: the fused kernel avoids sorting the logits and is
+// statistically equivalent to the sort-based sampler).
+//
+// Each logit is mapped to a 32-bit key that orders like the float.  The K-th
+// largest key is found by a radix select (four passes over the row, 8 bits at
+// a time, a 256-bin count histogram each); the Top-P cut is a second radix
+// select over the same keys whose histograms hold probability mass instead of
+// counts.  Masses are exp((x - max) / T) in 32.32 fixed point, summed as
+// 64-bit integers, so every sum and comparison is exact and the result does not
+// depend on the order the threads add in: the same inputs always draw the
+// same token.  The draw is inverse-CDF in vocabulary order: the first kept
+// token whose running mass exceeds floor(u * total).
+//
+// Semantics (the readings of the page's sampler):
+//   T <= 0: greedy, the largest logit, lowest index among equals.
+//   0 < K < V: keep the tokens whose logit is at least the K-th largest.
+//   P < 1: over those, keep the tokens in decreasing logit order until their
+//   mass reaches P of the kept mass, with every token tied with the last one.
+//   NaN logits are never drawn (their key is the smallest).
+#include <cstdint>
+
+#include "common.cuh"
+#include "internal.h"
+#include "../../include/pa_sampler.h"
+
+namespace pa {
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+constexpr int kCand = 4096;   // candidates the small-K path keeps in shared memory
+constexpr int kFastK = 1024;  // Top-K values the small-K path takes
+
+__device__ __forceinline__ uint32_t key_of(float x) {
+  if (x != x) return 0u;  // NaN: below everything
+  const uint32_t b = __float_as_uint(x);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float float_of(uint32_t k) {
+  const uint32_t b = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+  return __uint_as_float(b);
+}
+
+// Mass of logit x in 32.32 fixed point: exp2((x - xmax) * scale) * 2^32.
+__device__ __forceinline__ uint64_t mass_of(float x, float xmax, float scale) {
+  if (x != x) return 0ull;
+  const float e = exp2f((x - xmax) * scale);  // in [0, 1]
+  return static_cast<uint64_t>(__float2ull_rn(e * 4294967296.0f));
+}
+
+// Warp 0 scans a 256-bin histogram from the highest bin down and returns the
+// first nonempty bin at which the running total reaches `need`, and the total
+// of the bins above it.  The caller has made sure the total reaches `need`.
+template <typename T>
+__device__ void pick_bin(const T* hist, T need, int* bin_out, T* above_out) {
+  const int lane = threadIdx.x & 31;
+  T part = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) part += hist[255 - 8 * lane - j];
+  T incl = part;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const T y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, incl >= need && part > 0);
+  const int L = hit ? __ffs(hit) - 1 : 31;
+  if (lane == L) {
+    T c = incl - part;
+    int b = 255 - 8 * lane - 7;
+    T above = c;
+    for (int j = 0; j < 8; ++j) {
+      const int bb = 255 - 8 * lane - j;
+      const T h = hist[bb];
+      if (h > 0 && c + h >= need) {
+        b = bb;
+        above = c;
+        break;
+      }
+      c += h;
+    }
+    *bin_out = b;
+    *above_out = above;
+  }
+}
+
+// Bitonic sort of v[0, n2) (n2 a power of two <= kCand) by all threads of the CTA;
+// descending if `desc`.  Ends with a barrier.
+__device__ void block_sort(uint64_t* v, int n2, bool desc) {
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += kThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint64_t a = v[i], b = v[ixj];
+          const bool up = ((i & k) == 0) != desc;  // this pair's order: ascending if up
+          if (up ? (a > b) : (a < b)) {
+            v[i] = b;
+            v[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Inclusive scan of one uint64 per thread over the CTA; `tot` gets the total.
+__device__ uint64_t block_scan64(uint64_t x, uint64_t* wbuf, uint64_t* tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wbuf[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint64_t w = wbuf[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    wbuf[lane] = w;
+  }
+  __syncthreads();
+  const uint64_t r = x + (warp > 0 ? wbuf[warp - 1] : 0ull);
+  *tot = wbuf[kWarps - 1];
+  __syncthreads();
+  return r;
+}
+
+struct Smem {
+  uint32_t hcnt[256];
+  uint64_t hmass[256];
+  uint64_t wsum[kWarps];
+  uint64_t cand[kCand];       // small-K path: candidates, packed for sorting
+  uint32_t tmax[kThreads];    // each thread's largest key (pass 1)
+  unsigned long long red64;
+  int count;
+  int cut;
+  int bin;
+  uint32_t above_cnt;
+  uint64_t above_mass;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __restrict__ logits,
+                                                          int64_t row_stride, int V,
+                                                          const float* __restrict__ temperature,
+                                                          const int32_t* __restrict__ top_k,
+                                                          const float* __restrict__ top_p,
+                                                          const float* __restrict__ uniform,
+                                                          int32_t* __restrict__ tokens) {
+  __shared__ Smem sm;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = blockIdx.x;
+  const float* x = logits + static_cast<int64_t>(row) * row_stride;
+  const float T = temperature[row];
+  const int K = top_k[row];
+  const float P = top_p[row];
+  float u = uniform[row];
+  u = (u >= 0.f && u < 1.f) ? u : 0.f;
+
+  // ---- pass 1: the largest key, lowest index among equals ----
+  uint32_t bk = 0;
+  int bi = 0x7fffffff;
+  for (int i = tid; i < V; i += kThreads) {
+    const uint32_t k = key_of(x[i]);
+    if (k > bk || (k == bk && i < bi)) {
+      bk = k;
+      bi = i;
+    }
+  }
+  sm.tmax[tid] = bk;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint32_t k2 = __shfl_xor_sync(0xffffffffu, bk, o);
+    const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (k2 > bk || (k2 == bk && i2 < bi)) {
+      bk = k2;
+      bi = i2;
+    }
+  }
+  // (key, -index) packed so one 64-bit maximum finds both
+  __shared__ unsigned long long best;
+  if (tid == 0) best = 0ull;
+  __syncthreads();
+  if (lane == 0)
+    atomicMax(&best, (static_cast<unsigned long long>(bk) << 32) |
+                         static_cast<unsigned long long>(0x7fffffff - bi));
+  __syncthreads();
+  const uint32_t kmax = static_cast<uint32_t>(best >> 32);
+  const int argmax = 0x7fffffff - static_cast<int>(best & 0xffffffffull);
+  if (!(T > 0.f) || kmax == 0u) {
+    if (tid == 0) tokens[row] = argmax;
+    return;
+  }
+  const float xmax = float_of(kmax);
+  const float scale = kLog2e / T;
+
+  // ---- small K: candidates in shared memory ----
+  // The K-th largest of the threads' maxima t0 is a lower bound of the K-th
+  // largest key (K distinct elements reach it), so every Top-K survivor has
+  // key >= t0.  When those elements fit in shared memory, everything else is
+  // done there: sort them, cut at the K-th, cut at Top-P, draw.
+  if (K > 0 && K <= kFastK && K < V) {
+    for (int i = tid; i < kThreads; i += kThreads) sm.cand[i] = sm.tmax[i];
+    __syncthreads();
+    block_sort(sm.cand, kThreads, true);
+    const uint32_t t0 = static_cast<uint32_t>(sm.cand[K - 1]);
+    if (tid == 0) sm.count = 0;
+    __syncthreads();
+    for (int i = tid; i < V; i += kThreads) {
+      const uint32_t k = key_of(x[i]);
+      if (k >= t0) {
+        const int pos = atomicAdd(&sm.count, 1);
+        // (key, -index): descending order is by logit, then by index
+        if (pos < kCand)
+          sm.cand[pos] = (static_cast<uint64_t>(k) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
+      }
+    }
+    __syncthreads();
+    const int n = sm.count;
+    if (n <= kCand) {
+      int n2 = 1;
+      while (n2 < n) n2 <<= 1;
+      for (int i = n + tid; i < n2; i += kThreads) sm.cand[i] = 0ull;  // below every real entry
+      __syncthreads();
+      block_sort(sm.cand, n2, true);
+      const uint32_t tk = static_cast<uint32_t>(sm.cand[K - 1] >> 32);
+      // survivors of Top-K: the leading K entries and any ties with the K-th
+      if (tid == 0) {
+        int c = K;
+        while (c < n && static_cast<uint32_t>(sm.cand[c] >> 32) >= tk) ++c;
+        sm.count = c;
+      }
+      __syncthreads();
+      const int m = sm.count;
+      // thread t owns sorted entries [4t, 4t + 4)
+      const int j0 = 4 * tid;
+      uint64_t ms[4];
+      uint64_t mine = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = j0 + q;
+        ms[q] = j < m ? mass_of(float_of(static_cast<uint32_t>(sm.cand[j] >> 32)), xmax, scale) : 0ull;
+        mine += ms[q];
+      }
+      uint64_t mk = 0;
+      const uint64_t incl = block_scan64(mine, sm.wsum, &mk);
+      int m2 = m;
+      if (P < 1.f) {
+        const double want = static_cast<double>(P > 0.f ? P : 0.f) * static_cast<double>(mk);
+        uint64_t need = static_cast<uint64_t>(ceil(want));
+        if (need < 1) need = 1;
+        // the first sorted entry at which the running mass reaches `need`
+        if (tid == 0) sm.cut = m - 1;
+        __syncthreads();
+        uint64_t run = incl - mine;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int j = j0 + q;
+          if (j < m && run < need && run + ms[q] >= need) atomicMin(&sm.cut, j);
+          run += ms[q];
+        }
+        __syncthreads();
+        if (tid == 0) {
+          const uint32_t cutkey = static_cast<uint32_t>(sm.cand[sm.cut] >> 32);
+          int c = sm.cut + 1;
+          while (c < m && static_cast<uint32_t>(sm.cand[c] >> 32) >= cutkey) ++c;  // ties
+          sm.count = c;
+        }
+        __syncthreads();
+        m2 = sm.count;
+      }
+      // the draw: kept entries re-packed as (index, key) and sorted by index
+      for (int i = tid; i < n2; i += kThreads) {
+        const uint64_t e = sm.cand[i];
+        sm.cand[i] = i < m2 ? ((static_cast<uint64_t>(0xffffffffu - static_cast<uint32_t>(e)) << 32) |
+                               (e >> 32))
+                            : ~0ull;
+      }
+      __syncthreads();
+      block_sort(sm.cand, n2, false);
+      uint64_t mine2 = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = j0 + q;
+        ms[q] = j < m2 ? mass_of(float_of(static_cast<uint32_t>(sm.cand[j])), xmax, scale) : 0ull;
+        mine2 += ms[q];
+      }
+      uint64_t total = 0;
+      const uint64_t incl2 = block_scan64(mine2, sm.wsum, &total);
+      const uint64_t tg = static_cast<uint64_t>(static_cast<double>(u) * static_cast<double>(total));
+      const uint64_t tgt = tg < total ? tg : total - 1;
+      uint64_t run = incl2 - mine2;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = j0 + q;
+        if (j < m2 && ms[q] > 0 && run <= tgt && run + ms[q] > tgt)
+          tokens[row] = static_cast<int32_t>(sm.cand[j] >> 32);
+        run += ms[q];
+      }
+      return;
+    }
+    __syncthreads();
+  }
+
+  // ---- Top-K: the K-th largest key by radix select ----
+  uint32_t tk = 0;
+  if (K > 0 && K < V) {
+    uint32_t prefix = 0, pmask = 0, need = static_cast<uint32_t>(K);
+    for (int d = 3; d >= 0; --d) {
+      for (int b = tid; b < 256; b += kThreads) sm.hcnt[b] = 0;
+      __syncthreads();
+      const int sh = 8 * d;
+      for (int i = tid; i < V; i += kThreads) {
+        const uint32_t k = key_of(x[i]);
+        if ((k & pmask) == prefix) atomicAdd(&sm.hcnt[(k >> sh) & 255u], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) pick_bin<uint32_t>(sm.hcnt, need, &sm.bin, &sm.above_cnt);
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(sm.bin) << sh;
+      pmask |= 255u << sh;
+      need -= sm.above_cnt;
+      __syncthreads();
+    }
+    tk = prefix;
+  }
+
+  // ---- Top-P: the cut key by a radix select over mass ----
+  uint32_t tcut = tk;
+  if (P < 1.f) {
+    // mass of the Top-K survivors
+    uint64_t s = 0;
+    for (int i = tid; i < V; i += kThreads) {
+      const float xi = x[i];
+      if (key_of(xi) >= tk) s += mass_of(xi, xmax, scale);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) sm.wsum[warp] = s;
+    __syncthreads();
+    if (tid == 0) {
+      uint64_t t = 0;
+      for (int w = 0; w < kWarps; ++w) t += sm.wsum[w];
+      sm.red64 = t;
+    }
+    __syncthreads();
+    const uint64_t mk = sm.red64;
+    const double want = static_cast<double>(P > 0.f ? P : 0.f) * static_cast<double>(mk);
+    uint64_t need = static_cast<uint64_t>(ceil(want));
+    if (need < 1) need = 1;
+    uint32_t prefix = 0, pmask = 0;
+    for (int d = 3; d >= 0; --d) {
+      for (int b = tid; b < 256; b += kThreads) sm.hmass[b] = 0;
+      __syncthreads();
+      const int sh = 8 * d;
+      for (int i = tid; i < V; i += kThreads) {
+        const float xi = x[i];
+        const uint32_t k = key_of(xi);
+        if (k >= tk && (k & pmask) == prefix) {
+          const uint64_t m = mass_of(xi, xmax, scale);
+          if (m) atomicAdd(reinterpret_cast<unsigned long long*>(&sm.hmass[(k >> sh) & 255u]),
+                           static_cast<unsigned long long>(m));
+        }
+      }
+      __syncthreads();
+      if (warp == 0) pick_bin<uint64_t>(sm.hmass, need, &sm.bin, &sm.above_mass);
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(sm.bin) << sh;
+      pmask |= 255u << sh;
+      need -= sm.above_mass;
+      __syncthreads();
+    }
+    tcut = prefix > tk ? prefix : tk;
+  }
+
+  // ---- the draw: inverse CDF in vocabulary order over keys >= tcut ----
+  // warp w owns the contiguous segment [w * seg, (w + 1) * seg)
+  const int seg = (V + kWarps - 1) / kWarps;
+  const int lo = min(V, warp * seg), hi = min(V, lo + seg);
+  uint64_t s = 0;
+  for (int i = lo + lane; i < hi; i += 32) {
+    const float xi = x[i];
+    if (key_of(xi) >= tcut) s += mass_of(xi, xmax, scale);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) sm.wsum[warp] = s;
+  __syncthreads();
+  if (warp == 0) {
+    const uint64_t mine = sm.wsum[lane];
+    uint64_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint64_t total = __shfl_sync(0xffffffffu, incl, 31);
+    const uint64_t target =
+        static_cast<uint64_t>(static_cast<double>(u) * static_cast<double>(total));
+    const uint64_t tgt = target < total ? target : (total ? total - 1 : 0);
+    const unsigned hit = __ballot_sync(0xffffffffu, incl > tgt && mine > 0);
+    const int W = hit ? __ffs(hit) - 1 : 0;
+    const uint64_t excl_w = __shfl_sync(0xffffffffu, incl - mine, W);
+    if (lane == 0) {
+      sm.bin = W;           // the warp whose segment holds the draw
+      sm.above_mass = excl_w;
+      sm.red64 = tgt;
+    }
+  }
+  __syncthreads();
+  if (warp == sm.bin) {
+    const uint64_t tgt = sm.red64;
+    uint64_t run = sm.above_mass;
+    int found = -1;
+    for (int base = lo; base < hi && found < 0; base += 32) {
+      const int i = base + lane;
+      uint64_t m = 0;
+      if (i < hi) {
+        const float xi = x[i];
+        if (key_of(xi) >= tcut) m = mass_of(xi, xmax, scale);
+      }
+      uint64_t incl = m;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, m > 0 && run + incl > tgt);
+      if (hit) found = base + __ffs(hit) - 1;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) tokens[row] = found >= 0 ? found : argmax;
+  }
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" int pa_sample(const float* logits, int64_t row_stride, int32_t num_rows, int32_t vocab,
+                         const float* temperature, const int32_t* top_k, const float* top_p,
+                         const float* uniform, int32_t* tokens, void* stream) {
+  if (num_rows < 0 || vocab <= 0 || row_stride < vocab) return PA_ERR_ARG;
+  if (num_rows == 0) return PA_OK;
+  if (!logits || !temperature || !top_k || !top_p || !uniform || !tokens) return PA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(logits) % alignof(float)) return PA_ERR_ARG;
+  sample_kernel<<<num_rows, kThreads, 0, as_stream(stream)>>>(logits, row_stride, vocab,
+                                                             temperature, top_k, top_p, uniform,
+                                                             tokens);
+  return launch_status();
+}
