@@ -270,6 +270,34 @@ def sampler_timing(w: Workload, stream, reps: int = 50):
                                 for k, v in res.items()}}
 
 
+def swap_timing(w: Workload, stream, blocks: int = 512, reps: int = 10):
+    """Device time of moving `blocks` whole blocks (K and V, all KV heads) of this
+    pool to page-locked host memory and back (``pa_swap_blocks``), as GB/s
+    each way; CUDA events around ``reps`` calls after warm-up."""
+    torch = w.torch
+    kp, vp = w.t["k_pool"], w.t["v_pool"]
+    blocks = min(blocks, kp.shape[0])
+    kh = torch.empty((blocks,) + tuple(kp.shape[1:]), dtype=kp.dtype).pin_memory()
+    vh = torch.empty_like(kh).pin_memory()
+    out_pairs = np.stack([np.arange(blocks), np.arange(blocks)], 1).astype(np.int64)
+    res = {}
+    for name, direction in (("out", 0), ("in", 1)):
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                w.pa.pa_swap_blocks(kp, vp, kh, vh, out_pairs, direction, stream=stream)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                w.pa.pa_swap_blocks(kp, vp, kh, vh, out_pairs, direction, stream=stream)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        res[name] = round(2 * kh.numel() * kh.element_size() / (ms * 1e-3) / 1e9, 1)
+    return {"gb_per_s": res, "blocks": blocks,
+            "bytes_each_way": 2 * kh.numel() * kh.element_size()}
+
+
 def e2e_run(w: Workload, stream, steps, warmup):
     """The same step through the public API with host buffers: per step, pinned
     host -> device copies of the step's inputs (q, new K/V, slot mapping, block
@@ -521,6 +549,7 @@ def main():
         "clocks": clk,
         "host_block_manager": host_manager_timing(w) if rank == 0 else None,
         "fused_sampler": sampler_timing(w, stream) if rank == 0 else None,
+        "block_swap": swap_timing(w, stream) if rank == 0 else None,
     }
     if rank == 0:
         print(json.dumps(res), flush=True)

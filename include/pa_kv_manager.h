@@ -60,11 +60,13 @@ extern "C" {
 typedef struct pa_kvm pa_kvm; /* opaque manager */
 
 /*
- * pa_kvm_create -- a manager of `num_blocks` blocks of `block_size` slots.
+ * pa_kvm_create -- a manager of `num_blocks` device blocks of `block_size`
+ * slots and `num_host_blocks` (>= 0) blocks of host swap space.
  * prefix_caching != 0 turns on prefix caching (token ids are then required by
  * add/append).  Returns NULL on bad sizes or when out of host memory.
  */
-PA_API pa_kvm* pa_kvm_create(int32_t num_blocks, int32_t block_size, int32_t prefix_caching);
+PA_API pa_kvm* pa_kvm_create(int32_t num_blocks, int32_t block_size, int32_t prefix_caching,
+                             int32_t num_host_blocks);
 
 /* pa_kvm_destroy -- release the manager (NULL is allowed). */
 PA_API void pa_kvm_destroy(pa_kvm* m);
@@ -155,6 +157,32 @@ PA_API int pa_kvm_batch(const pa_kvm* m, const int64_t* seq_ids, int32_t num_seq
  */
 PA_API int pa_kvm_batch_update(const pa_kvm* m, const int64_t* seq_ids, int32_t num_seqs,
                                int32_t max_blocks, int32_t* block_tables, int32_t* context_lens);
+
+/*
+ * pa_kvm_swap_out -- move a sequence that holds every one of its blocks alone
+ * ("当大模型推理遇上内存瓶颈" 5.1 CPU swap space, 7.3 cold blocks to slower
+ * storage): each block gets the lowest free host block, in table order; the
+ * device blocks are released (last first; cached ones stay in the prefix cache)
+ * and the table now lists host blocks.  pairs (int64 [capacity][2]) receives
+ * the (device, host) pairs for pa_swap_blocks(PA_SWAP_OUT), run before the
+ * device blocks are reused.  PA_ERR_ARG for a shared block or a swapped-out
+ * sequence, PA_ERR_SHAPE if capacity is too small, PA_ERR_NO_BLOCKS if the
+ * host space is short.  A swapped-out sequence can only be swapped in, freed or
+ * inspected.
+ */
+PA_API int pa_kvm_swap_out(pa_kvm* m, int64_t seq_id, int64_t* pairs, int32_t capacity,
+                           int32_t* num_pairs);
+
+/*
+ * pa_kvm_swap_in -- bring a swapped-out sequence back into fresh device blocks
+ * (nothing is registered in the prefix cache); pairs receives the (host,
+ * device) pairs for pa_swap_blocks(PA_SWAP_IN), run before the sequence is used.
+ */
+PA_API int pa_kvm_swap_in(pa_kvm* m, int64_t seq_id, int64_t* pairs, int32_t capacity,
+                          int32_t* num_pairs);
+
+/* Free blocks of host swap space. */
+PA_API int32_t pa_kvm_num_free_host_blocks(const pa_kvm* m);
 
 /* Tables referencing `block`, or -1 when it is out of range. */
 PA_API int32_t pa_kvm_ref_count(const pa_kvm* m, int32_t block);

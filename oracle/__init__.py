@@ -21,6 +21,7 @@ from .paged_attention import (  # noqa: F401
     chunked_prefill,
     reshape_and_cache,
     copy_blocks,
+    swap_blocks,
     CopyBlocksError,
 )
 from .kv_manager import KvManager, KvManagerError, NoBlocks  # noqa: F401,E402

@@ -53,6 +53,12 @@ Readings taken where the pages are silent or leave a choice:
   becomes ``src``'s block ``i``;
   the block ``dst`` held there loses a reference, and ``dst``'s tokens in that
   block's positions become ``src``'s.
+* Swapping ("当大模型推理遇上内存瓶颈" 5.1 CPU swap space, 7.3 cold blocks to
+  slower storage): a sequence that holds every one of its blocks alone can be
+  swapped out -- each block gets the lowest free host block, the device blocks
+  are released (last first; cached ones stay cached) and the table lists host
+  blocks; swapping in takes fresh device blocks (registering nothing in the
+  prefix cache).  A swapped-out sequence can only be swapped in or freed.
 * Every operation is all-or-nothing: when the pool cannot supply the blocks it
   needs, it raises ``NoBlocks`` and changes nothing.
 """
@@ -70,9 +76,11 @@ class KvManagerError(ValueError):
 
 
 class KvManager:
-    def __init__(self, num_blocks: int, block_size: int, prefix_caching: bool):
-        if num_blocks <= 0 or block_size <= 0:
+    def __init__(self, num_blocks: int, block_size: int, prefix_caching: bool,
+                 num_host_blocks: int = 0):
+        if num_blocks <= 0 or block_size <= 0 or num_host_blocks < 0:
             raise KvManagerError("bad sizes")
+        self.host_free = set(range(num_host_blocks))  # host swap-space blocks
         self.num_blocks = num_blocks
         self.bs = block_size
         self.prefix_caching = bool(prefix_caching)
@@ -139,10 +147,13 @@ class KvManager:
         if n > self.num_free_blocks():
             raise NoBlocks(f"need {n} blocks, {self.num_free_blocks()} free")
 
-    def _seq(self, sid):
+    def _seq(self, sid, resident=True):
         if sid not in self.seqs:
             raise KvManagerError(f"unknown sequence {sid}")
-        return self.seqs[sid]
+        s = self.seqs[sid]
+        if resident and s.get("swapped"):
+            raise KvManagerError(f"sequence {sid} is swapped out")
+        return s
 
     # ------------------------------------------------------------- sequences
     def add_sequence(self, sid, tokens):
@@ -269,18 +280,60 @@ class KvManager:
                 d["tokens"][t] = s["tokens"][t]
 
     def free_sequence(self, sid):
+        s = self._seq(sid, resident=False)
+        if s.get("swapped"):
+            self.host_free.update(s["table"])
+        else:
+            # the last blocks first, so a released prompt's early blocks stay cached longest
+            for b in reversed(s["table"]):
+                self._release(b)
+        del self.seqs[sid]
+
+    # ---------------------------------------------------------------- swapping
+    def swap_out(self, sid):
+        """Move a sequence's blocks to host blocks ("当大模型推理遇上内存瓶颈" 5.1,
+        7.3).  Only a sequence that holds all its blocks alone can move.
+        Returns the (device, host) pairs to copy."""
         s = self._seq(sid)
-        # the last blocks first, so a released prompt's early blocks stay cached longest
+        if any(self.ref[b] != 1 for b in s["table"]):
+            raise KvManagerError("a shared block cannot be swapped out")
+        if len(s["table"]) > len(self.host_free):
+            raise NoBlocks("host swap space exhausted")
+        host = []
+        for _ in s["table"]:
+            h = min(self.host_free)
+            self.host_free.remove(h)
+            host.append(h)
+        pairs = list(zip(s["table"], host))
         for b in reversed(s["table"]):
             self._release(b)
-        del self.seqs[sid]
+        s["table"] = host
+        s["swapped"] = True
+        return pairs
+
+    def swap_in(self, sid):
+        """Bring a swapped-out sequence back into fresh device blocks.  Returns
+        the (host, device) pairs to copy."""
+        s = self._seq(sid, resident=False)
+        if not s.get("swapped"):
+            raise KvManagerError(f"sequence {sid} is not swapped out")
+        self._need(len(s["table"]))
+        dev = [self._alloc() for _ in s["table"]]
+        pairs = list(zip(s["table"], dev))
+        self.host_free.update(s["table"])
+        s["table"] = dev
+        s["swapped"] = False
+        return pairs
+
+    def num_free_host_blocks(self) -> int:
+        return len(self.host_free)
 
     # ----------------------------------------------------------------- views
     def block_table(self, sid):
-        return list(self._seq(sid)["table"])
+        return list(self._seq(sid, resident=False)["table"])
 
     def context_len(self, sid):
-        return self._seq(sid)["len"]
+        return self._seq(sid, resident=False)["len"]
 
     def ref_count(self, b):
         return self.ref[b]

@@ -225,3 +225,22 @@ def copy_blocks(k_pool, v_pool, pairs):
         k[d] = k_pool[s]
         v[d] = v_pool[s]
     return k, v
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, pairs):
+    """Copy whole K and V blocks from the source pools to the destination pools
+    (``src -> dst`` per pair; "当大模型推理遇上内存瓶颈" 5.1 and 7.3: KV blocks moved
+    to a CPU swap space and read back).  The two sides are different pools, so
+    only the destinations must be distinct.  Returns the new destination pools."""
+    pairs = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
+    ns, nd = src_k.shape[0], dst_k.shape[0]
+    for s_, d_ in pairs:
+        if not (0 <= s_ < ns and 0 <= d_ < nd):
+            raise CopyBlocksError(f"pair ({s_}, {d_}) outside the pools ({ns}, {nd})")
+    if len(set(int(d_) for d_ in pairs[:, 1])) != len(pairs):
+        raise CopyBlocksError("repeated destination block")
+    k, v = dst_k.copy(), dst_v.copy()
+    for s_, d_ in pairs:
+        k[d_] = src_k[s_]
+        v[d_] = src_v[s_]
+    return k, v

@@ -19,7 +19,8 @@ from ._abi import (PA_DEV_ERR_BLOCK_ID, PA_DEV_ERR_CONTEXT, PA_DEV_ERR_SLOT,  # 
 __all__ = [
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
     "pa_decode_noalloc",
-    "pa_chunked_prefill", "pa_gather_kv", "pa_get_device_error", "pa_sample", "pool_desc", "lib",
+    "pa_chunked_prefill", "pa_gather_kv", "pa_get_device_error", "pa_sample", "pa_swap_blocks",
+    "pool_desc", "lib",
     "PaError", "PA_KERNEL_AUTO", "PA_KERNEL_SIMT", "PA_KERNEL_TCGEN05",
 ]
 
@@ -239,3 +240,22 @@ def pa_sample(logits, temperature, top_k, top_p, uniform, out=None, stream=None)
         _ptr(logits), logits.stride(0), rows, vocab, _ptr(temperature), _ptr(top_k),
         _ptr(top_p), _ptr(uniform), _ptr(out), _stream(stream)))
     return out
+
+
+def pa_swap_blocks(k_pool, v_pool, k_host, v_host, pairs, direction, stream=None) -> None:
+    """Copy whole blocks between the device pools and page-locked host pools of
+    the same block shape (``k_host``/``v_host``: pinned CPU tensors).
+    ``direction``: ``_abi.PA_SWAP_OUT`` (device src -> host dst) or
+    ``_abi.PA_SWAP_IN`` (host src -> device dst); ``pairs``: int64 [P, 2]."""
+    torch = _torch()
+    _check_pools(k_pool, v_pool)
+    for name, t in (("k_host", k_host), ("v_host", v_host)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_pinned():
+            raise TypeError(f"{name} must be a pinned CPU tensor")
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape[1:] != k_pool.shape[1:]:
+            raise ValueError(f"{name} must be bf16 [num_host_blocks, {tuple(k_pool.shape[1:])}]")
+    arr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+    _abi.check("pa_swap_blocks", lib().pa_swap_blocks(
+        _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(k_host), _ptr(v_host),
+        k_host.shape[0], arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], int(direction),
+        _stream(stream)))

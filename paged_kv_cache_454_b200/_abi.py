@@ -20,6 +20,9 @@ PA_ERR_WORKSPACE = 4
 PA_ERR_CUDA = 5
 PA_ERR_NO_BLOCKS = 6
 
+PA_SWAP_OUT = 0
+PA_SWAP_IN = 1
+
 PA_DEV_ERR_BLOCK_ID = 0x1
 PA_DEV_ERR_SLOT = 0x2
 PA_DEV_ERR_CONTEXT = 0x4
@@ -62,7 +65,7 @@ SIGNATURES = {
     # fused sampler (include/pa_sampler.h)
     "pa_sample": (c_int, [c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     # host KV-cache block manager (include/pa_kv_manager.h)
-    "pa_kvm_create": (c_vp, [c_i32, c_i32, c_i32]),
+    "pa_kvm_create": (c_vp, [c_i32, c_i32, c_i32, c_i32]),
     "pa_kvm_destroy": (None, [c_vp]),
     "pa_kvm_num_free_blocks": (c_i32, [c_vp]),
     "pa_kvm_add_sequence": (c_int, [c_vp, c_i64, c_vp, c_i32, c_vp, c_vp]),
@@ -77,6 +80,11 @@ SIGNATURES = {
     "pa_kvm_batch": (c_int, [c_vp, c_vp, c_i32, c_i32, c_vp, c_vp]),
     "pa_kvm_batch_update": (c_int, [c_vp, c_vp, c_i32, c_i32, c_vp, c_vp]),
     "pa_kvm_ref_count": (c_i32, [c_vp, c_i32]),
+    "pa_kvm_swap_out": (c_int, [c_vp, c_i64, c_vp, c_i32, c_vp]),
+    "pa_kvm_swap_in": (c_int, [c_vp, c_i64, c_vp, c_i32, c_vp]),
+    "pa_kvm_num_free_host_blocks": (c_i32, [c_vp]),
+    # block swapping (include/pa_swap.h)
+    "pa_swap_blocks": (c_int, [c_vp, c_vp, PoolDesc, c_vp, c_vp, c_i32, c_vp, c_i32, c_i32, c_vp]),
 }
 
 _lib = None

@@ -86,6 +86,7 @@ struct Seq {
   std::vector<int32_t> table;
   int32_t len = 0;
   uint64_t stamp = 0;           // last batch call that listed this sequence
+  bool swapped = false;         // table lists host swap-space blocks
   std::vector<int32_t> tokens;  // kept only with prefix caching
   std::vector<uint64_t> hash;   // chain hash of each full block (prefix caching)
 };
@@ -97,6 +98,7 @@ struct pa_kvm {
   bool pc;
   std::vector<int32_t> ref;
   IdSet free_set;
+  IdSet host_free;  // host swap-space blocks
   // LRU of unreferenced cached blocks
   std::vector<int32_t> prev, next;
   std::vector<uint8_t> in_lru;
@@ -109,10 +111,18 @@ struct pa_kvm {
   std::unordered_map<int64_t, Seq> seqs;
   uint64_t calls = 0;  // batch-call counter (duplicate detection)
 
-  pa_kvm(int32_t n, int32_t b, bool p)
-      : nb(n), bs(b), pc(p), ref(n, 0), free_set(n), prev(n, -1), next(n, -1), in_lru(n, 0),
-        cached(n, 0), bhash(n, 0), bparent(n, 0), btokens(p ? n : 0), children(p ? n : 0) {
+  pa_kvm(int32_t n, int32_t b, bool p, int32_t nh)
+      : nb(n), bs(b), pc(p), ref(n, 0), free_set(n), host_free(nh > 0 ? nh : 1), prev(n, -1),
+        next(n, -1), in_lru(n, 0), cached(n, 0), bhash(n, 0), bparent(n, 0),
+        btokens(p ? n : 0), children(p ? n : 0) {
     for (int32_t i = 0; i < n; ++i) free_set.insert(i);
+    for (int32_t i = 0; i < nh; ++i) host_free.insert(i);
+  }
+
+  // A sequence that is present and resident on the device, or NULL.
+  Seq* resident(int64_t id) {
+    auto it = seqs.find(id);
+    return it == seqs.end() || it->second.swapped ? nullptr : &it->second;
   }
 
   int32_t num_free() const { return free_set.size() + n_lru; }
@@ -260,9 +270,10 @@ using namespace std;
 
 extern "C" {
 
-PA_API pa_kvm* pa_kvm_create(int32_t num_blocks, int32_t block_size, int32_t prefix_caching) {
-  if (num_blocks <= 0 || block_size <= 0) return nullptr;
-  return new (std::nothrow) pa_kvm(num_blocks, block_size, prefix_caching != 0);
+PA_API pa_kvm* pa_kvm_create(int32_t num_blocks, int32_t block_size, int32_t prefix_caching,
+                             int32_t num_host_blocks) {
+  if (num_blocks <= 0 || block_size <= 0 || num_host_blocks < 0) return nullptr;
+  return new (std::nothrow) pa_kvm(num_blocks, block_size, prefix_caching != 0, num_host_blocks);
 }
 
 PA_API void pa_kvm_destroy(pa_kvm* m) { delete m; }
@@ -321,9 +332,9 @@ PA_API int pa_kvm_append_tokens(pa_kvm* m, int64_t seq_id, const int32_t* tokens
                                 int64_t* slots, int64_t* copy_pair, int32_t* num_pairs) {
   if (!m || n < 0 || (n > 0 && !slots) || (m->pc && n > 0 && !tokens) || !num_pairs)
     return PA_ERR_ARG;
-  auto it = m->seqs.find(seq_id);
-  if (it == m->seqs.end()) return PA_ERR_ARG;
-  Seq& s = it->second;
+  Seq* sp = m->resident(seq_id);
+  if (!sp) return PA_ERR_ARG;
+  Seq& s = *sp;
   *num_pairs = 0;
   if (n == 0) return PA_OK;
   bool cow = false;
@@ -347,7 +358,7 @@ PA_API int pa_kvm_decode_step(pa_kvm* m, const int64_t* seq_ids, int32_t num_seq
   int32_t need = 0;
   for (int32_t i = 0; i < num_seqs; ++i) {
     auto it = m->seqs.find(seq_ids[i]);
-    if (it == m->seqs.end() || it->second.stamp == stamp) return PA_ERR_ARG;
+    if (it == m->seqs.end() || it->second.swapped || it->second.stamp == stamp) return PA_ERR_ARG;
     Seq& s = it->second;
     s.stamp = stamp;
     ss[i] = &s;
@@ -376,9 +387,9 @@ PA_API int pa_kvm_decode_step(pa_kvm* m, const int64_t* seq_ids, int32_t num_seq
 
 PA_API int pa_kvm_fork(pa_kvm* m, int64_t parent, int64_t child) {
   if (!m) return PA_ERR_ARG;
-  auto it = m->seqs.find(parent);
-  if (it == m->seqs.end() || m->seqs.count(child)) return PA_ERR_ARG;
-  Seq c = it->second;
+  Seq* p = m->resident(parent);
+  if (!p || m->seqs.count(child)) return PA_ERR_ARG;
+  Seq c = *p;
   for (int32_t b : c.table) m->retain(b);
   m->seqs.emplace(child, std::move(c));
   return PA_OK;
@@ -386,9 +397,9 @@ PA_API int pa_kvm_fork(pa_kvm* m, int64_t parent, int64_t child) {
 
 PA_API int pa_kvm_share_prefix(pa_kvm* m, int64_t src, int64_t dst, int32_t n_blocks) {
   if (!m) return PA_ERR_ARG;
-  auto it = m->seqs.find(src);
-  if (it == m->seqs.end() || m->seqs.count(dst)) return PA_ERR_ARG;
-  const Seq& s = it->second;
+  const Seq* sp = m->resident(src);
+  if (!sp || m->seqs.count(dst)) return PA_ERR_ARG;
+  const Seq& s = *sp;
   if (n_blocks < 0 || n_blocks > static_cast<int32_t>(s.table.size())) return PA_ERR_ARG;
   Seq d;
   d.len = std::min(s.len, n_blocks * m->bs);
@@ -404,11 +415,11 @@ PA_API int pa_kvm_share_prefix(pa_kvm* m, int64_t src, int64_t dst, int32_t n_bl
 
 PA_API int pa_kvm_share_blocks(pa_kvm* m, int64_t src, int64_t dst, const int32_t* idx, int32_t n) {
   if (!m || n < 0 || (n > 0 && !idx)) return PA_ERR_ARG;
-  auto si = m->seqs.find(src);
-  auto di = m->seqs.find(dst);
-  if (si == m->seqs.end() || di == m->seqs.end()) return PA_ERR_ARG;
-  Seq& s = si->second;
-  Seq& d = di->second;
+  Seq* sp = m->resident(src);
+  Seq* dp = m->resident(dst);
+  if (!sp || !dp) return PA_ERR_ARG;
+  Seq& s = *sp;
+  Seq& d = *dp;
   const int32_t bs = m->bs;
   for (int32_t k = 0; k < n; ++k) {
     const int32_t i = idx[k];
@@ -437,7 +448,11 @@ PA_API int pa_kvm_free_sequence(pa_kvm* m, int64_t seq_id) {
   auto it = m->seqs.find(seq_id);
   if (it == m->seqs.end()) return PA_ERR_ARG;
   const vector<int32_t>& t = it->second.table;
-  for (auto b = t.rbegin(); b != t.rend(); ++b) m->release(*b);
+  if (it->second.swapped) {
+    for (int32_t h : t) m->host_free.insert(h);
+  } else {
+    for (auto b = t.rbegin(); b != t.rend(); ++b) m->release(*b);
+  }
   m->seqs.erase(it);
   return PA_OK;
 }
@@ -469,7 +484,7 @@ PA_API int pa_kvm_batch(const pa_kvm* m, const int64_t* seq_ids, int32_t num_seq
     return PA_ERR_ARG;
   for (int32_t i = 0; i < num_seqs; ++i) {
     auto it = m->seqs.find(seq_ids[i]);
-    if (it == m->seqs.end()) return PA_ERR_ARG;
+    if (it == m->seqs.end() || it->second.swapped) return PA_ERR_ARG;
     if (static_cast<int32_t>(it->second.table.size()) > max_blocks) return PA_ERR_SHAPE;
   }
   for (int32_t i = 0; i < num_seqs; ++i) {
@@ -490,7 +505,7 @@ PA_API int pa_kvm_batch_update(const pa_kvm* m, const int64_t* seq_ids, int32_t 
     return PA_ERR_ARG;
   for (int32_t i = 0; i < num_seqs; ++i) {
     auto it = m->seqs.find(seq_ids[i]);
-    if (it == m->seqs.end()) return PA_ERR_ARG;
+    if (it == m->seqs.end() || it->second.swapped) return PA_ERR_ARG;
     const Seq& s = it->second;
     const int32_t nt = static_cast<int32_t>(s.table.size());
     if (nt > max_blocks) return PA_ERR_SHAPE;
@@ -498,6 +513,58 @@ PA_API int pa_kvm_batch_update(const pa_kvm* m, const int64_t* seq_ids, int32_t 
     context_lens[i] = s.len;
   }
   return PA_OK;
+}
+
+PA_API int pa_kvm_swap_out(pa_kvm* m, int64_t seq_id, int64_t* pairs, int32_t capacity,
+                           int32_t* num_pairs) {
+  if (!m || capacity < 0 || !num_pairs || (capacity > 0 && !pairs)) return PA_ERR_ARG;
+  Seq* sp = m->resident(seq_id);
+  if (!sp) return PA_ERR_ARG;
+  Seq& s = *sp;
+  const int32_t n = static_cast<int32_t>(s.table.size());
+  for (int32_t b : s.table)
+    if (m->ref[b] != 1) return PA_ERR_ARG;  // shared with another table
+  if (n > capacity) return PA_ERR_SHAPE;
+  if (n > m->host_free.size()) return PA_ERR_NO_BLOCKS;
+  vector<int32_t> host(n);
+  for (int32_t i = 0; i < n; ++i) {
+    host[i] = m->host_free.lowest();
+    m->host_free.erase(host[i]);
+    pairs[2 * i] = s.table[i];
+    pairs[2 * i + 1] = host[i];
+  }
+  for (auto b = s.table.rbegin(); b != s.table.rend(); ++b) m->release(*b);
+  s.table = std::move(host);
+  s.swapped = true;
+  *num_pairs = n;
+  return PA_OK;
+}
+
+PA_API int pa_kvm_swap_in(pa_kvm* m, int64_t seq_id, int64_t* pairs, int32_t capacity,
+                          int32_t* num_pairs) {
+  if (!m || capacity < 0 || !num_pairs || (capacity > 0 && !pairs)) return PA_ERR_ARG;
+  auto it = m->seqs.find(seq_id);
+  if (it == m->seqs.end() || !it->second.swapped) return PA_ERR_ARG;
+  Seq& s = it->second;
+  const int32_t n = static_cast<int32_t>(s.table.size());
+  if (n > capacity) return PA_ERR_SHAPE;
+  if (n > m->num_free()) return PA_ERR_NO_BLOCKS;
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t b = m->alloc();
+    pairs[2 * i] = s.table[i];
+    pairs[2 * i + 1] = b;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    m->host_free.insert(s.table[i]);
+    s.table[i] = static_cast<int32_t>(pairs[2 * i + 1]);
+  }
+  s.swapped = false;
+  *num_pairs = n;
+  return PA_OK;
+}
+
+PA_API int32_t pa_kvm_num_free_host_blocks(const pa_kvm* m) {
+  return m ? m->host_free.size() : 0;
 }
 
 PA_API int32_t pa_kvm_ref_count(const pa_kvm* m, int32_t block) {

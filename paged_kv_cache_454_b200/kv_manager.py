@@ -32,9 +32,11 @@ def _p(a: np.ndarray):
 class KvManager:
     """One pool of ``num_blocks`` blocks of ``block_size`` token slots."""
 
-    def __init__(self, num_blocks: int, block_size: int = 16, prefix_caching: bool = False):
+    def __init__(self, num_blocks: int, block_size: int = 16, prefix_caching: bool = False,
+                 num_host_blocks: int = 0):
         self._lib = _abi.load()
-        self._h = self._lib.pa_kvm_create(num_blocks, block_size, 1 if prefix_caching else 0)
+        self._h = self._lib.pa_kvm_create(num_blocks, block_size, 1 if prefix_caching else 0,
+                                          num_host_blocks)
         if not self._h:
             raise ValueError("pa_kvm_create failed (bad sizes or out of memory)")
         self.num_blocks = num_blocks
@@ -160,6 +162,24 @@ class KvManager:
                     self._lib.pa_kvm_batch_update(self._h, _p(ids), len(ids), tables.shape[1],
                                                   _p(tables), _p(lens)))
         return tables, lens
+
+    def _swap(self, fn, seq_id):
+        _, nb = self.sequence_info(seq_id)
+        pairs = np.empty((max(nb, 1), 2), np.int64)
+        n = ctypes.c_int32(0)
+        self._check(fn, getattr(self._lib, fn)(self._h, seq_id, _p(pairs), nb, ctypes.byref(n)))
+        return [(int(a), int(b)) for a, b in pairs[:n.value]]
+
+    def swap_out(self, seq_id: int):
+        """Move the sequence to host swap space; returns the (device, host) pairs."""
+        return self._swap("pa_kvm_swap_out", seq_id)
+
+    def swap_in(self, seq_id: int):
+        """Bring it back to fresh device blocks; returns the (host, device) pairs."""
+        return self._swap("pa_kvm_swap_in", seq_id)
+
+    def num_free_host_blocks(self) -> int:
+        return self._lib.pa_kvm_num_free_host_blocks(self._h)
 
     def ref_count(self, block: int) -> int:
         return self._lib.pa_kvm_ref_count(self._h, block)

@@ -120,3 +120,69 @@ def test_manager_drives_cache_writes_copies_and_decode():
         assert np.array_equal(vb[cu[i]:cu[i + 1]], rows[s][1])
     assert pa().pa_get_device_error() == 0
     torch.cuda.synchronize()
+
+
+def test_swap_blocks_bit_exact():
+    torch = H.torch()
+    rng = np.random.default_rng(9)
+    nb, nh = 40, 12
+    kd = synth.normal_bf16(rng, (nb, HKV, BS, D))
+    vd = synth.normal_bf16(rng, (nb, HKV, BS, D))
+    kh = synth.normal_bf16(rng, (nh, HKV, BS, D))
+    vh = synth.normal_bf16(rng, (nh, HKV, BS, D))
+    k_pool, v_pool = H.dev_bf16(kd), H.dev_bf16(vd)
+    k_host = torch.from_numpy(kh.view(np.int16)).view(torch.bfloat16).pin_memory()
+    v_host = torch.from_numpy(vh.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_pairs = np.array([[3, 0], [7, 5], [39, 11], [7, 2]], np.int64)   # a source twice
+    pa().pa_swap_blocks(k_pool, v_pool, k_host, v_host, out_pairs, 0)
+    torch.cuda.synchronize()
+    rk, rv = oracle.swap_blocks(kd, vd, kh, vh, out_pairs)
+    assert np.array_equal(k_host.view(torch.int16).numpy().view(np.uint16), rk)
+    assert np.array_equal(v_host.view(torch.int16).numpy().view(np.uint16), rv)
+    in_pairs = np.array([[0, 1], [11, 2], [4, 30]], np.int64)
+    pa().pa_swap_blocks(k_pool, v_pool, k_host, v_host, in_pairs, 1)
+    rk2, rv2 = oracle.swap_blocks(rk, rv, kd, vd, in_pairs)
+    assert np.array_equal(H.host_bits(k_pool), rk2) and np.array_equal(H.host_bits(v_pool), rv2)
+    from paged_kv_cache_454_b200 import _abi
+    with pytest.raises(pa().PaError):
+        pa().pa_swap_blocks(k_pool, v_pool, k_host, v_host, np.array([[0, 12]]), 0)  # host id out
+    with pytest.raises(pa().PaError):
+        pa().pa_swap_blocks(k_pool, v_pool, k_host, v_host, np.array([[0, 1], [2, 1]]), 0)
+    assert _abi.PA_SWAP_IN == 1
+
+
+def test_manager_swaps_a_sequence_out_and_back():
+    torch = H.torch()
+    from paged_kv_cache_454_b200.kv_manager import KvManager
+    rng = np.random.default_rng(13)
+    nb, nh = 8, 8
+    m = KvManager(nb, BS, num_host_blocks=nh)
+    k_pool = H.dev_bf16(synth.normal_bf16(rng, (nb, HKV, BS, D)))
+    v_pool = H.dev_bf16(synth.normal_bf16(rng, (nb, HKV, BS, D)))
+    k_host = torch.empty((nh, HKV, BS, D), dtype=torch.bfloat16).pin_memory()
+    v_host = torch.empty((nh, HKV, BS, D), dtype=torch.bfloat16).pin_memory()
+    rows = {}
+    for s, n in ((0, 70), (1, 20)):
+        slots, _ = m.add_sequence(s, np.zeros(n, np.int32))
+        k, v = synth.normal_bf16(rng, (n, HKV, D)), synth.normal_bf16(rng, (n, HKV, D))
+        pa().pa_reshape_and_cache(H.dev_bf16(k), H.dev_bf16(v), k_pool, v_pool, H.dev_i64(slots))
+        rows[s] = [k, v]
+    # sequence 0 (5 blocks) moves out; sequence 2 takes its device blocks
+    pa().pa_swap_blocks(k_pool, v_pool, k_host, v_host, m.swap_out(0), 0)
+    slots2, _ = m.add_sequence(2, np.zeros(80, np.int32))
+    k2, v2 = synth.normal_bf16(rng, (80, HKV, D)), synth.normal_bf16(rng, (80, HKV, D))
+    pa().pa_reshape_and_cache(H.dev_bf16(k2), H.dev_bf16(v2), k_pool, v_pool, H.dev_i64(slots2))
+    rows[2] = [k2, v2]
+    m.free_sequence(2)
+    del rows[2]
+    pa().pa_swap_blocks(k_pool, v_pool, k_host, v_host, m.swap_in(0), 1)
+    seqs = [0, 1]
+    tables, lens = m.batch(seqs, 8)
+    q = synth.normal_bf16(rng, (2, HQ, D))
+    out, lse = pa().pa_decode(H.dev_bf16(q), k_pool, v_pool, H.dev_i32(tables), H.dev_i32(lens),
+                              0.125, want_lse=True)
+    ut, ul, ukp, uvp = unshared_pools([rows[s] for s in seqs])
+    ref_o, ref_l = oracle.decode(q, ukp, uvp, ut, ul, 0.125)
+    H.assert_close(H.host_f64(out), ref_o, what="after swap in")
+    H.assert_lse_close(lse.cpu().numpy(), ref_l, what="after swap in")
+    assert pa().pa_get_device_error() == 0

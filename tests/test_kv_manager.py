@@ -34,6 +34,10 @@ def run(target, op):
             target.share_prefix(op[1], op[2], op[3])
         elif kind == "share_blocks":
             target.share_blocks(op[1], op[2], op[3])
+        elif kind == "swap_out":
+            return ("ok", [tuple(map(int, p)) for p in target.swap_out(op[1])])
+        elif kind == "swap_in":
+            return ("ok", [tuple(map(int, p)) for p in target.swap_in(op[1])])
         else:
             target.free_sequence(op[1])
         return ("ok",)
@@ -48,6 +52,7 @@ def run(target, op):
 
 def compare_state(ref, lib, live):
     assert lib.num_free_blocks() == ref.num_free_blocks()
+    assert lib.num_free_host_blocks() == ref.num_free_host_blocks()
     assert [lib.ref_count(b) for b in range(ref.num_blocks)] == ref.ref
     for sid in live:
         assert lib.block_table(sid) == ref.block_table(sid), sid
@@ -58,8 +63,8 @@ def compare_state(ref, lib, live):
 @pytest.mark.parametrize("seed", range(8))
 def test_cpp_manager_matches_oracle_op_by_op(seed, prefix_caching):
     nb, bs = 24, 4
-    ref = oracle.KvManager(nb, bs, prefix_caching)
-    lib = KvManager(nb, bs, prefix_caching)
+    ref = oracle.KvManager(nb, bs, prefix_caching, 10)
+    lib = KvManager(nb, bs, prefix_caching, 10)
     for op in random_ops(seed, 500, nb, bs, prefix_caching):
         a, b = run(ref, op), run(lib, op)
         assert a == b, (op, a, b)
@@ -69,8 +74,8 @@ def test_cpp_manager_matches_oracle_op_by_op(seed, prefix_caching):
 @pytest.mark.parametrize("prefix_caching", [False, True])
 def test_cpp_manager_matches_oracle_on_a_larger_pool(prefix_caching):
     nb, bs = 300, 16
-    ref = oracle.KvManager(nb, bs, prefix_caching)
-    lib = KvManager(nb, bs, prefix_caching)
+    ref = oracle.KvManager(nb, bs, prefix_caching, 60)
+    lib = KvManager(nb, bs, prefix_caching, 60)
     for i, op in enumerate(random_ops(100 + int(prefix_caching), 1500, nb, bs, prefix_caching)):
         assert run(ref, op) == run(lib, op), op
         if i % 50 == 0:
@@ -99,9 +104,9 @@ def test_batch_builds_decode_inputs():
 
 def test_host_argument_checks():
     lib = _abi.load()
-    assert not lib.pa_kvm_create(0, 16, 0)
-    assert not lib.pa_kvm_create(4, 0, 0)
-    h = lib.pa_kvm_create(8, 4, 1)
+    assert not lib.pa_kvm_create(0, 16, 0, 0)
+    assert not lib.pa_kvm_create(4, 0, 0, 0)
+    h = lib.pa_kvm_create(8, 4, 1, 0)
     try:
         slots = (ctypes.c_int64 * 4)()
         toks = (ctypes.c_int32 * 4)(1, 2, 3, 4)
@@ -123,7 +128,7 @@ def test_host_argument_checks():
 
 def test_without_prefix_caching_tokens_may_be_omitted():
     lib = _abi.load()
-    h = lib.pa_kvm_create(8, 4, 0)
+    h = lib.pa_kvm_create(8, 4, 0, 0)
     try:
         slots = (ctypes.c_int64 * 6)()
         assert lib.pa_kvm_add_sequence(h, 1, None, 6, slots, None) == _abi.PA_OK

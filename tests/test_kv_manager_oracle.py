@@ -20,10 +20,12 @@ from oracle import KvManager, KvManagerError, NoBlocks
 class Sim:
     """A manager plus a token-id pool and the expected token list per sequence."""
 
-    def __init__(self, num_blocks, bs, prefix_caching):
-        self.m = KvManager(num_blocks, bs, prefix_caching)
+    def __init__(self, num_blocks, bs, prefix_caching, num_host_blocks=0):
+        self.m = KvManager(num_blocks, bs, prefix_caching, num_host_blocks)
         self.bs = bs
         self.pool = [[None] * bs for _ in range(num_blocks)]
+        self.host = [[None] * bs for _ in range(num_host_blocks)]
+        self.swapped = set()
         self.expect = {}
 
     def _write(self, slots, tokens):
@@ -75,6 +77,21 @@ class Sim:
     def free(self, sid):
         self.m.free_sequence(sid)
         del self.expect[sid]
+        self.swapped.discard(sid)
+
+    def swap_out(self, sid):
+        pairs = self.m.swap_out(sid)
+        for d, h in pairs:
+            self.host[h] = list(self.pool[d])
+        self.swapped.add(sid)
+        return pairs
+
+    def swap_in(self, sid):
+        pairs = self.m.swap_in(sid)
+        for h, d in pairs:
+            self.pool[d] = list(self.host[h])
+        self.swapped.discard(sid)
+        return pairs
 
     def check(self):
         m, bs = self.m, self.bs
@@ -84,10 +101,12 @@ class Sim:
             assert m.context_len(sid) == len(toks)
             # on-demand allocation: only the last block may be partly used
             assert len(table) == -(-len(toks) // bs)
-            got = [self.pool[table[t // bs]][t % bs] for t in range(len(toks))]
+            src = self.host if sid in self.swapped else self.pool
+            got = [src[table[t // bs]][t % bs] for t in range(len(toks))]
             assert got == toks, (sid, got, toks)
-            for b in table:
-                refs[b] += 1
+            if sid not in self.swapped:
+                for b in table:
+                    refs[b] += 1
         assert refs == [m.ref_count(b) for b in range(m.num_blocks)]
         unref = {b for b in range(m.num_blocks) if refs[b] == 0}
         assert m.num_free_blocks() == len(unref)
@@ -244,7 +263,7 @@ def random_ops(seed, n_ops, num_blocks, bs, prefix_caching):
     few shared templates so that prefixes repeat."""
     rng = random.Random(seed)
     templates = [[rng.randrange(4) for _ in range(rng.randrange(1, 5 * bs))] for _ in range(4)]
-    live, next_id, ops = [], 0, []
+    live, next_id, ops, outs = [], 0, [], []
     for _ in range(n_ops):
         r = rng.random()
         if r < 0.25 or not live:
@@ -274,6 +293,12 @@ def random_ops(seed, n_ops, num_blocks, bs, prefix_caching):
         elif r < 0.8 and len(live) > 1:
             a, b = rng.sample(live, 2)
             ops.append(("share_blocks", a, b, sorted(rng.sample(range(3), rng.randrange(1, 3)))))
+        elif r < 0.83:
+            sid = rng.choice(live)
+            ops.append(("swap_out", sid))
+            outs.append(sid)
+        elif r < 0.86:
+            ops.append(("swap_in", outs.pop(rng.randrange(len(outs))) if outs else rng.choice(live)))
         else:
             sid = rng.choice(live)
             live.remove(sid)
@@ -297,6 +322,10 @@ def apply_op(target, op):
             return target.share_prefix(op[1], op[2], op[3])
         if kind == "share_blocks":
             return target.share_blocks(op[1], op[2], op[3])
+        if kind == "swap_out":
+            return target.swap_out(op[1])
+        if kind == "swap_in":
+            return target.swap_in(op[1])
         return target.free(op[1])
     except (NoBlocks, KvManagerError) as e:
         return type(e)
@@ -305,7 +334,7 @@ def apply_op(target, op):
 @pytest.mark.parametrize("prefix_caching", [False, True])
 @pytest.mark.parametrize("seed", range(6))
 def test_random_streams_keep_every_sequence_readable(seed, prefix_caching):
-    sim = Sim(24, 4, prefix_caching)
+    sim = Sim(24, 4, prefix_caching, num_host_blocks=10)
     for op in random_ops(seed, 400, 24, 4, prefix_caching):
         res = apply_op(sim, op)
         if res in (NoBlocks, KvManagerError):
@@ -314,3 +343,28 @@ def test_random_streams_keep_every_sequence_readable(seed, prefix_caching):
                 new = op[1] if op[0] == "add" else op[2]
                 sim.expect.pop(new, None)
         sim.check()
+
+
+def test_swap_out_and_in_move_a_sequence_through_host_blocks():
+    # "当大模型推理遇上内存瓶颈" 5.1 / 7.3: KV blocks move to a CPU swap space and back
+    sim = Sim(8, 4, False, num_host_blocks=4)
+    sim.add(0, list(range(10)))               # 3 blocks
+    sim.add(1, list(range(20, 25)))           # 2 blocks
+    pairs = sim.swap_out(0)
+    assert [d for d, _ in pairs] == [0, 1, 2] and [h for _, h in pairs] == [0, 1, 2]
+    assert sim.m.num_free_blocks() == 6 and sim.m.num_free_host_blocks() == 1
+    sim.check()
+    with pytest.raises(KvManagerError):
+        sim.append(0, [1])                    # swapped out: nothing but swap in / free
+    sim.add(2, list(range(40, 52)))           # reuses the freed device blocks
+    back = sim.swap_in(0)
+    assert [h for h, _ in back] == [0, 1, 2] and sim.m.num_free_host_blocks() == 4
+    sim.append(0, [7, 8])
+    sim.check()
+    sim.fork(1, 3)
+    with pytest.raises(KvManagerError):
+        sim.swap_out(1)                       # shares its blocks with 3
+    sim.swap_out(2)                           # 3 of the 4 host blocks
+    with pytest.raises(NoBlocks):
+        sim.swap_out(0)                       # 3 more blocks, 1 host block left
+    sim.check()
