@@ -76,6 +76,12 @@ def lay_gqa2_h6():
                               num_kv_heads=6, head_dim=128)
 
 
+def lay_gqa8_h3():
+    # group 8 over 3 KV heads: no pairs, one KV head per tile
+    return synth.build_layout("gqa8_h3", 117, [5, 200, 1800], num_q_heads=24, num_kv_heads=3,
+                              head_dim=128)
+
+
 def lay_mha_h5():
     # one q head per KV head, 5 KV heads: one head per tile
     return synth.build_layout("mha_h5", 115, [2, 17, 300, 1300], num_q_heads=5,
@@ -122,6 +128,7 @@ DECODE_LAYOUTS = {
     "gqa2_h6": lay_gqa2_h6,
     "mha_h5": lay_mha_h5,
     "mha_h16": lay_mha_h16,
+    "gqa8_h3": lay_gqa8_h3,
     "short_gqa": lay_short_gqa,
     "short_mha": lay_short_mha,
 }
@@ -220,7 +227,7 @@ def test_decode_simt(name, partition):
 
 @pytest.mark.parametrize("name", ["gqa8", "gqa5", "g16", "shared_prefix", "shared_many", "mha128",
                                   "short_gqa", "short_mha", "gqa4", "gqa2_h6", "mha_h5",
-                                  "mha_h16"])
+                                  "mha_h16", "gqa8_h3"])
 @pytest.mark.parametrize("partition", [0, 128, 1024, 1 << 20])
 def test_decode_tcgen05(name, partition):
     st, ref = _step_and_ref(name)
