@@ -180,31 +180,6 @@ __device__ __forceinline__ PfItem pf_decode(const PfParams& p, const PfRaw& r) {
   return it;
 }
 
-// 2^x on the FMA pipe, for the share of the softmax exponentials taken off the
-// multi-function unit.  x = j + f with j = rint(x) (by the 1.5 * 2^23 rounding
-// trick) and |f| <= 1/2; 2^f = e^(f ln 2) by its Taylor series to degree 5
-// (relative error below 3.3e-6 on |f| <= 1/2); j is added to the exponent
-// field.  x is clamped below at -126; callers pass x <= 8.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = __fadd_rn(x, 12582912.f);
-  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
-  float y = 1.3333558146428441e-3f;       // (ln 2)^5 / 5!
-  y = fmaf(y, f, 9.618129107628477e-3f);  // (ln 2)^4 / 4!
-  y = fmaf(y, f, 5.5504108664821576e-2f); // (ln 2)^3 / 3!
-  y = fmaf(y, f, 2.402265069591007e-1f);  // (ln 2)^2 / 2!
-  y = fmaf(y, f, 6.931471805599453e-1f);  // ln 2
-  y = fmaf(y, f, 1.f);
-  return __int_as_float(__float_as_int(y) + (__float_as_int(t) << 23));
-}
-
-#ifndef PA_PREFILL_EXP_FMA_EVERY
-#define PA_PREFILL_EXP_FMA_EVERY 0
-#endif
-// Every kExpFmaEvery-th exponential of the softmax is computed with exp2_fma
-// (0: none), balancing the multi-function unit against the FMA pipe.
-constexpr int kExpFmaEvery = PA_PREFILL_EXP_FMA_EVERY;
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return static_cast<uint32_t>(f32_to_bf16_bits(lo)) |
          (static_cast<uint32_t>(f32_to_bf16_bits(hi)) << 16);
@@ -570,11 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           for (int k = 0; k < 16; k += 2) {
             const int kk = c * 16 + k;
             const float2 x = __ffma2_rn(make_float2(sv[kk], sv[kk + 1]), sc2, nm2);
-            float p0 = (kExpFmaEvery > 0 && kk % kExpFmaEvery == kExpFmaEvery - 1) ? exp2_fma(x.x)
-                                                                                   : exp2f(x.x);
-            float p1 = (kExpFmaEvery > 0 && (kk + 1) % kExpFmaEvery == kExpFmaEvery - 1)
-                           ? exp2_fma(x.y)
-                           : exp2f(x.y);
+            float p0 = exp2f(x.x);
+            float p1 = exp2f(x.y);
             if (!all_vis) {
               p0 = ((vis[kk >> 5] >> (kk & 31)) & 1u) ? p0 : 0.f;
               p1 = ((vis[kk >> 5] >> ((kk + 1) & 31)) & 1u) ? p1 : 0.f;
