@@ -161,10 +161,13 @@ class Workload:
         self.flops_pf = synth.prefill_flops(lay) if len(self.pf) else 0
         self.tokens = len(self.dec) + int(lay.q_lens[self.pf].sum()) if len(self.pf) else len(self.dec)
 
-    # one pass of the hot path; `ev` collects per-component events
-    def step(self, stream, ev=None):
+    # one pass of the hot path; `ev` collects per-component events; `io`
+    # optionally replaces the step's input / output tensors (same shapes)
+    def step(self, stream, ev=None, io=None):
         pa, lay, t = self.pa, self.layout, self.t
         torch = self.torch
+        io = io or {}
+        get = lambda name, default: io.get(name, default)
 
         def mark(name):
             if ev is not None:
@@ -175,17 +178,19 @@ class Workload:
         mark("start")
         if lay.copy_pairs.size:
             pa.pa_copy_blocks(t["k_pool"], t["v_pool"], lay.copy_pairs, stream=stream)
-        pa.pa_reshape_and_cache(t["key"], t["value"], t["k_pool"], t["v_pool"],
-                                self.slot_mapping, stream=stream)
+        pa.pa_reshape_and_cache(get("key", t["key"]), get("value", t["value"]), t["k_pool"],
+                                t["v_pool"], get("slot_mapping", self.slot_mapping), stream=stream)
         mark("cache")
         if len(self.pf):
-            pa.pa_chunked_prefill(self.q_pf, self.cu_pf, self.max_q_pf, t["k_pool"], t["v_pool"],
-                                  self.tab_pf, self.len_pf, lay.scale, out=self.out_pf,
-                                  stream=stream)
+            pa.pa_chunked_prefill(get("q_pf", self.q_pf), get("cu_pf", self.cu_pf), self.max_q_pf,
+                                  t["k_pool"], t["v_pool"], get("tab_pf", self.tab_pf),
+                                  get("len_pf", self.len_pf), lay.scale,
+                                  out=get("out_pf", self.out_pf), stream=stream)
         mark("prefill")
         if len(self.dec):
-            pa.pa_decode(self.q_dec, t["k_pool"], t["v_pool"], self.tab_dec, self.len_dec,
-                         lay.scale, out=self.out_dec, workspace=self.ws, kernel=self.kernel,
+            pa.pa_decode(get("q_dec", self.q_dec), t["k_pool"], t["v_pool"],
+                         get("tab_dec", self.tab_dec), get("len_dec", self.len_dec), lay.scale,
+                         out=get("out_dec", self.out_dec), workspace=self.ws, kernel=self.kernel,
                          partition_tokens=self.partition, stream=stream)
         mark("decode")
 
@@ -299,20 +304,20 @@ def swap_timing(w: Workload, stream, blocks: int = 512, reps: int = 10):
 
 
 def e2e_run(w: Workload, stream, steps, warmup):
-    """The same step through the public API with host buffers: per step, pinned
-    host -> device copies of the step's inputs (q, new K/V, slot mapping, block
-    tables, context lengths), the calls, and a device -> host read of the
-    output.  The KV pool itself is device-resident state."""
+    """The same step through the public API with host buffers: every step copies
+    its inputs (q, new K/V, slot mapping, block tables, context lengths) from
+    pinned host memory and reads its output back to pinned host memory, all
+    inside the timed region.  As a serving loop would, the copies run on their
+    own streams with double-buffered device tensors, so step i+1's inputs move
+    while step i computes and step i's output moves while step i+1 computes.
+    The KV pool itself is device-resident state."""
     torch = w.torch
-    lay = w.layout
-    host = {}
-    dev = {}
-    names = []
+    names, host, proto = [], {}, {}
 
     def add(name, tensor):
         host[name] = torch.empty(tensor.shape, dtype=tensor.dtype, pin_memory=True)
         host[name].copy_(tensor.cpu())
-        dev[name] = tensor
+        proto[name] = tensor
         names.append(name)
 
     add("key", w.t["key"])
@@ -327,27 +332,65 @@ def e2e_run(w: Workload, stream, steps, warmup):
         add("cu_pf", w.cu_pf)
         add("tab_pf", w.tab_pf)
         add("len_pf", w.len_pf)
-    outs = [o for o in (w.out_dec, w.out_pf) if o is not None]
-    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    out_names = [n for n, o in (("out_dec", w.out_dec), ("out_pf", w.out_pf)) if o is not None]
+    out_proto = {"out_dec": w.out_dec, "out_pf": w.out_pf}
+    bufs = [{n: torch.empty_like(proto[n]) for n in names} for _ in range(2)]
+    for b in bufs:
+        for n in out_names:
+            b[n] = torch.empty_like(out_proto[n])
+    host_out = [{n: torch.empty(out_proto[n].shape, dtype=out_proto[n].dtype, pin_memory=True)
+                 for n in out_names} for _ in range(2)]
     h2d = sum(host[n].numel() * host[n].element_size() for n in names)
-    d2h = sum(o.numel() * o.element_size() for o in outs)
+    d2h = sum(out_proto[n].numel() * out_proto[n].element_size() for n in out_names)
+    s_in = torch.cuda.Stream(device=w.dev)
+    s_out = torch.cuda.Stream(device=w.dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for b in range(2):   # every event recorded once, so the first waits are no-ops
+        ev_comp[b].record(stream)
+        ev_out[b].record(stream)
 
-    def one():
-        with torch.cuda.stream(stream):
+    def copy_in(i):
+        b = i % 2
+        s_in.wait_event(ev_comp[b])          # step i-2 is done reading buffer b
+        with torch.cuda.stream(s_in):
             for n in names:
-                dev[n].copy_(host[n], non_blocking=True)
-            w.step(stream)
-            for o, ho in zip(outs, host_out):
-                ho.copy_(o, non_blocking=True)
+                bufs[b][n].copy_(host[n], non_blocking=True)
+        ev_in[b].record(s_in)
 
-    for _ in range(warmup):
-        one()
+    def compute(i):
+        b = i % 2
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])         # step i-2's output has left buffer b
+        with torch.cuda.stream(stream):
+            w.step(stream, io=bufs[b])
+        ev_comp[b].record(stream)
+
+    def copy_out(i):
+        b = i % 2
+        s_out.wait_event(ev_comp[b])
+        with torch.cuda.stream(s_out):
+            for n in out_names:
+                host_out[b][n].copy_(bufs[b][n], non_blocking=True)
+        ev_out[b].record(s_out)
+
+    def run(n):
+        copy_in(0)
+        for i in range(n):
+            if i + 1 < n:
+                copy_in(i + 1)
+            compute(i)
+            copy_out(i)
+
+    run(warmup)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(steps):
-        one()
+    s_in.wait_event(e0)
+    run(steps)
+    stream.wait_event(ev_out[(steps - 1) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
