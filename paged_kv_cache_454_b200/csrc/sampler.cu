@@ -168,13 +168,23 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
   // ---- pass 1: the largest key, lowest index among equals ----
   uint32_t bk = 0;
   int bi = 0x7fffffff;
-  for (int i = tid; i < V; i += kThreads) {
-    const uint32_t k = key_of(x[i]);
+  auto take = [&](float v, int i) {
+    const uint32_t k = key_of(v);
     if (k > bk || (k == bk && i < bi)) {
       bk = k;
       bi = i;
     }
+  };
+  int i0 = tid;
+  // four independent loads in flight per thread, then the compares in index order
+  for (; i0 + 3 * kThreads < V; i0 += 4 * kThreads) {
+    float a[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) a[q] = x[i0 + q * kThreads];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) take(a[q], i0 + q * kThreads);
   }
+  for (; i0 < V; i0 += kThreads) take(x[i0], i0);
   sm.tmax[tid] = bk;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -208,21 +218,46 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
   // key >= t0.  When those elements fit in shared memory, everything else is
   // done there: sort them, cut at the K-th, cut at Top-P, draw.
   if (K > 0 && K <= kFastK && K < V) {
-    for (int i = tid; i < kThreads; i += kThreads) sm.cand[i] = sm.tmax[i];
-    __syncthreads();
-    block_sort(sm.cand, kThreads, true);
-    const uint32_t t0 = static_cast<uint32_t>(sm.cand[K - 1]);
+    // t0: the K-th largest of the 1024 thread maxima, by radix select
+    uint32_t t0 = 0;
+    {
+      uint32_t prefix = 0, pmask = 0, need = static_cast<uint32_t>(K);
+      for (int dgt = 3; dgt >= 0; --dgt) {
+        if (tid < 256) sm.hcnt[tid] = 0;
+        __syncthreads();
+        const int sh = 8 * dgt;
+        const uint32_t k = sm.tmax[tid];
+        if ((k & pmask) == prefix) atomicAdd(&sm.hcnt[(k >> sh) & 255u], 1u);
+        __syncthreads();
+        if (warp == 0) pick_bin<uint32_t>(sm.hcnt, need, &sm.bin, &sm.above_cnt);
+        __syncthreads();
+        prefix |= static_cast<uint32_t>(sm.bin) << sh;
+        pmask |= 255u << sh;
+        need -= sm.above_cnt;
+        __syncthreads();
+      }
+      t0 = prefix;
+    }
     if (tid == 0) sm.count = 0;
     __syncthreads();
-    for (int i = tid; i < V; i += kThreads) {
-      const uint32_t k = key_of(x[i]);
+    auto collect = [&](float v, int i) {
+      const uint32_t k = key_of(v);
       if (k >= t0) {
         const int pos = atomicAdd(&sm.count, 1);
         // (key, -index): descending order is by logit, then by index
         if (pos < kCand)
           sm.cand[pos] = (static_cast<uint64_t>(k) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
       }
+    };
+    int i1 = tid;
+    for (; i1 + 3 * kThreads < V; i1 += 4 * kThreads) {
+      float a[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) a[q] = x[i1 + q * kThreads];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) collect(a[q], i1 + q * kThreads);
     }
+    for (; i1 < V; i1 += kThreads) collect(x[i1], i1);
     __syncthreads();
     const int n = sm.count;
     if (n <= kCand) {
