@@ -1,5 +1,7 @@
 // The decode work plan: one CTA turns context lengths into the list of
-// (sequence, KV head, partition) work items both decode kernels consume.
+// (sequence, KV-head group, partition) work items both decode kernels consume
+// (a group is one KV head for the CUDA-core kernel, one to eight for the
+// tensor-core kernel).
 //
 //  * Partition length: `min_part` tokens, or -- when the caller leaves the
 //    choice to the library -- the largest power-of-two multiple of it (up to
@@ -31,11 +33,11 @@ __device__ __forceinline__ int clamp_len(int L, int max_blocks, unsigned int* er
   return L;
 }
 
-// Items are bucketed by their tile count n (128 tokens per tile): bucket 0
+// Items are bucketed by their length n in units (a page or a few): bucket 0
 // holds n >= 64, bucket 64 - n holds 1 <= n < 64, bucket 64 the empty items.
 constexpr int kMaxBuckets = 65;
-__device__ __forceinline__ int bucket_of(int ntiles) {
-  return ntiles == 0 ? 64 : (ntiles >= 64 ? 0 : 64 - ntiles);
+__device__ __forceinline__ int bucket_of(int nunits) {
+  return nunits == 0 ? 64 : (nunits >= 64 ? 0 : 64 - nunits);
 }
 
 constexpr int kSortMax = 1024;  // sequences the locality order sorts (one per thread)
@@ -127,7 +129,10 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
       part = min_part << k;
       break;
     }
-  const int full_bucket = bucket_of(part / 128);
+  // items are bucketed by length in units of `unit` tokens: a page for short
+  // partitions, coarser for long ones, so a partition is at most 64 units
+  const int unit = part / 64 > 16 ? part / 64 : 16;
+  const int full_bucket = bucket_of(part / unit);
 
   // ---- partitions per sequence and their exclusive prefix ----
   if (tid == 0) carry = 0;
@@ -143,7 +148,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
       // bucket counts: full partitions, the tail, or an empty context
       const int full = L / part, rem = L - full * part;
       if (full) atomicAdd(&bucket[full_bucket], full * hkv);
-      if (rem) atomicAdd(&bucket[bucket_of((rem + 127) / 128)], hkv);
+      if (rem) atomicAdd(&bucket[bucket_of((rem + unit - 1) / unit)], hkv);
       if (L == 0) atomicAdd(&bucket[bucket_of(0)], hkv);
     }
     int x = np;
@@ -274,7 +279,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
         for (int q = 0; q < full; ++q) items[at++] = make_int2(s, (g << 16) | q);
     }
     if (rem) {
-      const int at = atomicAdd(&cursor[bucket_of((rem + 127) / 128)], hkv);
+      const int at = atomicAdd(&cursor[bucket_of((rem + unit - 1) / unit)], hkv);
       for (int g = 0; g < hkv; ++g) items[at + g] = make_int2(s, (g << 16) | full);
     }
     if (L == 0) {
