@@ -178,6 +178,7 @@ class Workload:
         mark("start")
         if lay.copy_pairs.size:
             pa.pa_copy_blocks(t["k_pool"], t["v_pool"], lay.copy_pairs, stream=stream)
+        mark("copy")
         pa.pa_reshape_and_cache(get("key", t["key"]), get("value", t["value"]), t["k_pool"],
                                 t["v_pool"], get("slot_mapping", self.slot_mapping), stream=stream)
         mark("cache")
@@ -301,6 +302,48 @@ def swap_timing(w: Workload, stream, blocks: int = 512, reps: int = 10):
         res[name] = round(2 * kh.numel() * kh.element_size() / (ms * 1e-3) / 1e9, 1)
     return {"gb_per_s": res, "blocks": blocks,
             "bytes_each_way": 2 * kh.numel() * kh.element_size()}
+
+
+def probe_timing(w: Workload, stream, decode_ms, reps: int = 20):
+    """Device time of ``pa_read_probe`` over this batch's decode tables: it reads
+    the very K/V pages the decode call reads (whole pages) and computes nothing,
+    one CTA per SM.  ``decode_over_probe`` = probe time / decode time, the share
+    of the paged layout's attainable read rate the decode call reaches.  CUDA
+    events around ``reps`` calls after warm-up; the pages (GBs) exceed L2."""
+    torch = w.torch
+    if not len(w.dec):
+        return None
+    lay = w.layout
+    kp, vp = w.t["k_pool"], w.t["v_pool"]
+    lens = lay.context_lens[w.dec].astype(np.int64)
+    pages = int(sum(-(-int(x) // lay.block_size) for x in lens)) * lay.num_kv_heads
+    page_bytes = lay.block_size * lay.head_dim * kp.element_size()
+    nbytes = 2 * pages * page_bytes
+    ctas = torch.cuda.get_device_properties(kp.device).multi_processor_count
+    out = torch.empty(ctas, dtype=torch.int64, device=kp.device)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            w.pa.pa_read_probe(kp, vp, w.tab_dec, w.len_dec, num_ctas=ctas, out=out, stream=stream)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            w.pa.pa_read_probe(kp, vp, w.tab_dec, w.len_dec, num_ctas=ctas, out=out, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    return {"gb_per_s": round(nbytes / (ms * 1e-3) / 1e9, 1), "us_per_call": round(ms * 1e3, 2),
+            "page_bytes_read": nbytes, "pages": 2 * pages, "ctas": ctas,
+            "decode_over_probe": round(ms / decode_ms, 4) if decode_ms else None}
+
+
+def step_stats(ev, first, last):
+    """min / median / p90 over the timed steps of the span between two marks (ms)."""
+    v = sorted(b.elapsed_time(c) for b, c in zip(ev[first], ev[last]))
+    if not v:
+        return None
+    return {"min": round(v[0], 4), "median": round(statistics.median(v), 4),
+            "p90": round(v[min(len(v) - 1, int(0.9 * len(v)))], 4)}
 
 
 def e2e_run(w: Workload, stream, steps, warmup):
@@ -532,7 +575,7 @@ def main():
         pg.barrier()
     ms = t0.elapsed_time(t1) / a.steps
     comp = {}
-    names = ["start", "cache", "prefill", "decode"]
+    names = ["start", "copy", "cache", "prefill", "decode"]
     for i in range(1, len(names)):
         comp[names[i]] = sum(b.elapsed_time(c) for b, c in zip(ev[names[i - 1]], ev[names[i]])) / a.steps
     e2e = None
@@ -584,6 +627,9 @@ def main():
                          % ((w.bytes_dec["kv"] if w.bytes_dec else 0) / 1e9),
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
         "components_ms": {k: round(v, 4) for k, v in comp.items()},
+        "step_ms_stats": step_stats(ev, "start", "decode"),
+        "decode_ms_stats": step_stats(ev, "prefill", "decode") if len(w.dec) else None,
+        "prefill_ms_stats": step_stats(ev, "cache", "prefill") if len(w.pf) else None,
         "kv_gbs": round(w.bytes_dec["unique"] / (comp["decode"] * 1e-3) / 1e9, 1) if len(w.dec) else None,
         "roofline": roof,
         "cpu_baseline": cpu,
@@ -593,6 +639,7 @@ def main():
         "host_block_manager": host_manager_timing(w) if rank == 0 else None,
         "fused_sampler": sampler_timing(w, stream) if rank == 0 else None,
         "block_swap": swap_timing(w, stream) if rank == 0 else None,
+        "read_probe": probe_timing(w, stream, comp["decode"]) if rank == 0 else None,
     }
     if rank == 0:
         print(json.dumps(res), flush=True)
@@ -604,15 +651,15 @@ def main():
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # decode kernel from an ncu capture, keyed by workload and the kernel sources
 # it was taken with (reported as null once those sources change).  The
-# gqa70b_long figure is the 48-sequence capture (1,764,388,096 bytes for
+# gqa70b_long figure is the 48-sequence capture (1,765,374,464 bytes for
 # 1,755,018,024 algorithmic bytes) scaled by algorithmic bytes to the full
 # 128-sequence batch; the captures are summarised in profiles/.
 TRAFFIC = {
-    # 48-sequence capture of the same shape (1.00534 x its algorithmic bytes), scaled
-    "gqa70b_long": {"bytes": 4785960097, "sources": "42a4d2966519"},
+    # 48-sequence capture of the same shape (1.00590 x its algorithmic bytes), scaled
+    "gqa70b_long": {"bytes": 4788635652, "sources": "6dc4103053c2"},
     # full-size captures
-    "llama13b_sampling": {"bytes": 2205319680, "sources": "42a4d2966519"},
-    "llama7b_decode": {"bytes": 1125474816, "sources": "42a4d2966519"},
+    "llama13b_sampling": {"bytes": 2198025472, "sources": "6dc4103053c2"},
+    "llama7b_decode": {"bytes": 1125487616, "sources": "6dc4103053c2"},
 }
 
 

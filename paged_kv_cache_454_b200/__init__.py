@@ -20,6 +20,7 @@ __all__ = [
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
     "pa_decode_noalloc",
     "pa_chunked_prefill", "pa_gather_kv", "pa_get_device_error", "pa_sample", "pa_swap_blocks",
+    "pa_read_probe",
     "pool_desc", "lib",
     "PaError", "PA_KERNEL_AUTO", "PA_KERNEL_SIMT", "PA_KERNEL_TCGEN05",
 ]
@@ -259,3 +260,28 @@ def pa_swap_blocks(k_pool, v_pool, k_host, v_host, pairs, direction, stream=None
         _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(k_host), _ptr(v_host),
         k_host.shape[0], arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], int(direction),
         _stream(stream)))
+
+
+def pa_read_probe(k_pool, v_pool, block_tables, context_lens, num_ctas=None, out=None,
+                  stream=None):
+    """Read every K/V page a decode over ``block_tables`` / ``context_lens``
+    reads, and nothing else (a read-bandwidth measurement).  Returns the
+    per-CTA sums (int64 [num_ctas], the bits of uint64 sums modulo 2^64) of the
+    pages' 32-bit words; ``num_ctas`` defaults to the SM count."""
+    torch = _torch()
+    _check_pools(k_pool, v_pool)
+    _need_cuda("block_tables", block_tables, torch.int32)
+    _need_cuda("context_lens", context_lens, torch.int32)
+    if block_tables.dim() != 2 or block_tables.shape[0] != context_lens.shape[0]:
+        raise ValueError("block_tables must be [S, max_blocks] with S = len(context_lens)")
+    if num_ctas is None:
+        num_ctas = torch.cuda.get_device_properties(k_pool.device).multi_processor_count
+    if out is None:
+        out = torch.empty(num_ctas, dtype=torch.int64, device=k_pool.device)
+    _need_cuda("out", out, torch.int64)
+    if out.numel() < num_ctas:
+        raise ValueError("out holds fewer than num_ctas sums")
+    _abi.check("pa_read_probe", lib().pa_read_probe(
+        _ptr(k_pool), _ptr(v_pool), pool_desc(k_pool), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), context_lens.shape[0], _ptr(out), int(num_ctas), _stream(stream)))
+    return out

@@ -85,6 +85,8 @@ SIGNATURES = {
     "pa_kvm_num_free_host_blocks": (c_i32, [c_vp]),
     # block swapping (include/pa_swap.h)
     "pa_swap_blocks": (c_int, [c_vp, c_vp, PoolDesc, c_vp, c_vp, c_i32, c_vp, c_i32, c_i32, c_vp]),
+    # paged read-bandwidth probe (include/pa_probe.h)
+    "pa_read_probe": (c_int, [c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp, c_i32, c_vp, c_i32, c_vp]),
 }
 
 _lib = None

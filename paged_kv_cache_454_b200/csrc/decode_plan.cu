@@ -15,7 +15,8 @@
 //    next to one SM's share of the work, the list is instead ordered by that
 //    block, then KV head, then sequence: the samples of a group read the shared
 //    pages of one KV head at the same time, so DRAM serves them once and L2
-//    the rest.  (Up to kSortMax sequences.)
+//    the rest.  (Up to kSortMax sequences.)  A hash set of first blocks finds
+//    whether any repeats; the sort runs only then.
 //  * It also clears the dynamic item counter and the per-(sequence, KV head)
 //    counters the tensor-core kernel uses to find the last partition to finish.
 #include "common.cuh"
@@ -42,6 +43,8 @@ __device__ __forceinline__ int bucket_of(int nunits) {
 
 constexpr int kSortMax = 1024;  // sequences the locality order sorts (one per thread)
 constexpr int kLensCache = 2048;  // sequences whose lengths the plan keeps in shared memory
+constexpr int kFirstSet = 2 * kSortMax;  // slots of the set that detects shared first blocks
+static_assert(kFirstSet == 2048, "the set's hash keeps 11 bits");
 
 // Inclusive block-wide scan (sum or max) of one value per thread, 1024 threads.
 template <bool kMax>
@@ -86,11 +89,19 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   __shared__ int run_tab[2 * kSortMax];           // per run start: partition prefix, run total
   __shared__ int sflag[4];                        // [0] any sharing, [1] max item tiles, [2] total tiles x KV heads
   __shared__ int slens[kLensCache];               // context lengths as given (S <= kLensCache)
+  __shared__ unsigned first_set[kFirstSet];       // open-addressing set of first blocks
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   // The decode kernel that follows may start its prologue now; it waits for
   // this grid's results before reading them.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // Thread i's sequence's first table entry, loaded now so its latency overlaps
+  // the passes below (used only when S fits the locality sort).
+  const bool sortable = S > 1 && S <= kSortMax && max_blocks > 0;
+  unsigned my_first = 0xffffffffu;
+  if (sortable && tid < S) my_first = static_cast<unsigned>(block_tables[static_cast<int64_t>(tid) * max_blocks]);
+  for (int i = tid; i < kFirstSet; i += 1024) first_set[i] = 0xffffffffu;
 
   // Context lengths are read once into shared memory when they fit; every pass
   // below reads them through `lens`.
@@ -175,33 +186,69 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     if (tid == 1023) carry += incl;
     __syncthreads();
   }
-  if (tid == 0) {
-    part_base[S] = carry;
-    int acc = 0;
-    for (int b = 0; b < kMaxBuckets; ++b) {
-      cursor[b] = acc;
-      acc += bucket[b];
+  if (warp == 0) {
+    // bucket start offsets: lane l owns buckets 3l .. 3l + 2
+    int c[3], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int b = 3 * lane + j;
+      c[j] = b < kMaxBuckets ? bucket[b] : 0;
+      sum += c[j];
     }
-    header[0] = carry * hkv;  // items
-    header[1] = carry;        // partitions
-    header[2] = 0;            // dynamic item counter
-    header[3] = part;         // partition length
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int acc = incl - sum;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int b = 3 * lane + j;
+      if (b < kMaxBuckets) cursor[b] = acc;
+      acc += c[j];
+    }
+    if (lane == 0) {
+      part_base[S] = carry;
+      header[0] = carry * hkv;  // items
+      header[1] = carry;        // partitions
+      header[2] = 0;            // dynamic item counter
+      header[3] = part;         // partition length
+    }
   }
   __syncthreads();
 
-  // ---- shared prefixes: sort sequences by their first physical block ----
+  // ---- shared prefixes: does any first physical block repeat?  (a set in
+  // shared memory; the sort below runs only if one does) ----
   bool locality = false;
-  if (S > 1 && S <= kSortMax) {
+  if (sortable) {
+    if (tid < 4) sflag[tid] = 0;
+    __syncthreads();
+    if (tid < S && clamp_len(lens[tid], max_blocks, nullptr) > 0) {
+      unsigned h = (my_first * 2654435761u) >> 21;  // 11 bits: kFirstSet slots
+      for (int probe = 0; probe < kFirstSet; ++probe, h = (h + 1) & (kFirstSet - 1)) {
+        const unsigned old = atomicCAS(&first_set[h], 0xffffffffu, my_first);
+        if (old == 0xffffffffu) break;
+        if (old == my_first) {
+          atomicOr(&sflag[0], 1);
+          break;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // ---- sort sequences by their first physical block ----
+  if (sortable && sflag[0]) {
     int n2 = 1;
     while (n2 < S) n2 <<= 1;
-    if (tid < 4) sflag[tid] = 0;
     for (int i = tid; i < n2; i += 1024) {
       unsigned long long k = ~0ull;
       if (i < S) {
         const int L = clamp_len(lens[i], max_blocks, nullptr);
-        const unsigned first =
-            L > 0 ? static_cast<unsigned>(block_tables[static_cast<int64_t>(i) * max_blocks])
-                  : 0xffffffffu;
+        const unsigned first = L > 0 ? (i == tid ? my_first
+                                                : static_cast<unsigned>(
+                                                      block_tables[static_cast<int64_t>(i) * max_blocks]))
+                                     : 0xffffffffu;
         k = (static_cast<unsigned long long>(first) << 32) | static_cast<unsigned>(i);
       }
       skey[i] = k;
@@ -223,11 +270,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
       }
     }
     if (tid < S) {
-      const unsigned first = static_cast<unsigned>(skey[tid] >> 32);
-      const bool shared = tid > 0 && first != 0xffffffffu &&
-                          first == static_cast<unsigned>(skey[tid - 1] >> 32);
       const int L = clamp_len(lens[tid], max_blocks, nullptr);
-      if (shared) atomicOr(&sflag[0], 1);
       atomicMax(&sflag[1], (min(L, part) + 127) / 128);
       atomicAdd(&sflag[2], ((L + 127) / 128) * hkv);
     }

@@ -2,11 +2,15 @@
 //
 // All G = Hq/Hkv query heads of one KV head read the same K/V pages.  A tile
 // is 128 rows of the pool: HT KV heads x 16 tokens of each of 8/HT pages (the
-// HT heads of one page are adjacent in the pool, so a page of the tile moves
-// as one HT*2 KiB tensor copy per 64-dim half).  HT = 1 for large groups; for
-// small groups (MHA above all) several KV heads share a tile, which keeps the
-// copies large -- the copy engine moves 2 KiB boxes at well under the HBM
-// rate -- and fills the product's N dimension with useful columns.
+// HT heads of one page are adjacent in the pool, so a page of K moves as one
+// HT*2 KiB tensor copy per 64-dim half).  HT = 1 for large groups; for small
+// groups (MHA above all) several KV heads share a tile, which keeps the copies
+// large -- the copy engine moves 2 KiB boxes at well under the HBM rate -- and
+// fills the product's N dimension with useful columns.  A page of V (HT < 8)
+// moves as one 3-D copy of both halves, which land next to each other: the
+// second product takes its K = 16 slices page by page, so per-page halves
+// suit it, while the first product's M = 128 rows span all pages of the tile
+// and need each half's rows evenly spaced, so K keeps one copy per half.
 // With NH q columns per tile (the group's q heads of the tile's KV heads,
 // padded) the work is two small dense products:
 //     S^T [128 rows x 16] = K_tile [128 x D] . Q^T [D x 16]
@@ -113,7 +117,8 @@ static_assert(sizeof(TileDesc) == 64, "descriptor slot size");
 
 struct __align__(64) TcParams {
   CUtensorMap tm_k;
-  CUtensorMap tm_v;
+  CUtensorMap tm_v;   // V as rows of 64 dims (two copies per page, one per half)
+  CUtensorMap tm_v3;  // V as (64 dims, row, half): one copy per page
   CUtensorMap tm_q;
   const int32_t* block_tables;
   const int32_t* context_lens;
@@ -229,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     *abort_flag = 0;
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
+    prefetch_tmap(&p.tm_v3);
     prefetch_tmap(&p.tm_q);
   }
   if (warp == 1) tmem_alloc(tmem_slot, L::kTmemCols);
@@ -364,11 +370,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           if (pb >= 0) {
             const int prow = (pb * p.hkv + (g << hts)) * 16;
             const uint32_t kdst = stage + lane * (ht * 2048);
-            const uint32_t vdst = kdst + kKBytes;
+            const uint32_t vdst = stage + kKBytes + lane * (ht * 4096);
             tma_load_2d_hint(kdst, &p.tm_k, 0, prow, &full[st], pol);
             tma_load_2d_hint(kdst + kRegion, &p.tm_k, 64, prow, &full[st], pol);
-            tma_load_2d_hint(vdst, &p.tm_v, 0, prow, &full[st], pol);
-            tma_load_2d_hint(vdst + kRegion, &p.tm_v, 64, prow, &full[st], pol);
+            if (ht < 8) {
+              tma_load_3d_hint(vdst, &p.tm_v3, 0, prow, 0, &full[st], pol);  // both halves
+            } else {
+              // a 128-row page: two 16 KiB copies ran faster than one of 32 KiB
+              tma_load_2d_hint(vdst, &p.tm_v, 0, prow, &full[st], pol);
+              tma_load_2d_hint(vdst + kRegion, &p.tm_v, 64, prow, &full[st], pol);
+            }
           }
         }
         ++t;
@@ -398,7 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       // a product then costs only constant adds (the single issuing thread is
       // otherwise bound by its own address arithmetic).
       const uint64_t desc_k0 = smem_desc_sw128(sbase, 16, 1024);
-      const uint64_t desc_v0 = smem_desc_sw128(sbase + kKBytes, kRegion, 1024);
+      const uint64_t desc_v0 = smem_desc_sw128(sbase + kKBytes, ht * 2048, 1024);
+      // rows 16k.. of the V tile: page k >> hts, its (k & (ht-1))-th 16 rows
+      uint32_t voff[kRows / 16];
+#pragma unroll
+      for (int k = 0; k < kRows / 16; ++k) voff[k] = 2048u * (k + ((k >> hts) << hts));
       const uint64_t desc_q0 = smem_desc_sw128(sbase + L::kOffQ, 16, 1024);
       const uint64_t desc_p0 = smem_desc_sw128(sbase + L::kOffP, 16, 1024);
       uint32_t d = 0, ts = 0, tpv = 0, mq = 0;  // ts: next S tile; tpv: next O tile
@@ -418,9 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             const uint32_t dt = tmem + 2 * kN + b * kNpv;
 #pragma unroll
             for (int k = 0; k < kRows / 16; ++k) {
-              // A = V^T (MN-major): 16 rows = 2 groups of 8; D halves kRegion apart
+              // A = V^T (MN-major): 16 rows = 2 groups of 8; D halves ht*2 KiB apart
               // B = P (K-major, kNpv rows = q columns): row half k/4, 32 bytes per 16 rows
-              umma_ss(dt, desc_add(a0, k * 2048), desc_add(b0, (k >> 2) * (kNpv * 128) + (k & 3) * 32),
+              umma_ss(dt, desc_add(a0, voff[k]), desc_add(b0, (k >> 2) * (kNpv * 128) + (k & 3) * 32),
                       kIdescO, k > 0 ? 1u : 0u);
             }
             umma_commit(&o_full[b]);
@@ -591,6 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     const int wi = warp - 2;
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
     const int pj = r >> (4 + hts);
+    // row r of the V tile: page pj holds its rows for dims 0-63, then 64-127
+    const uint32_t v_row_off = pj * (ht * 4096) + (r & ((16 << hts) - 1)) * 128;
     const int col = (r >> 4) & (ht - 1);          // this row's q column
     const int col0 = (2 * q4) & (ht - 1);         // column of lanes 0-15 (S load base)
     const bool upper = ht > 1 && lane >= 16;      // lanes 16-31 hold column col0 + 1
@@ -680,11 +697,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         sts16(pbuf + swz(col, c >> 3) + (c & 7) * 2, hi);
         sts16(pbuf + swz(NH + col, c >> 3) + (c & 7) * 2, f32_to_bf16_bits(rem));
         if (!valid) {
-          const uint32_t vrow = sbase + st * kStageBytes + kKBytes + r * 128;
+          const uint32_t vrow = sbase + st * kStageBytes + kKBytes + v_row_off;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             sts128_zero(vrow + k * 16);
-            sts128_zero(vrow + kRegion + k * 16);
+            sts128_zero(vrow + ht * 2048 + k * 16);
           }
         }
         fence_proxy_async_smem();
@@ -741,6 +758,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
     // tile row r: page j, KV head hh of the tile, token j * 16 + r % 16
     const int pj = r >> (4 + hts);
+    // row r of the V tile: page pj holds its rows for dims 0-63, then 64-127
+    const uint32_t v_row_off = pj * (ht * 4096) + (r & ((16 << hts) - 1)) * 128;
     const int c_lo = ((r >> 4) & (ht - 1)) * p.group;  // this row's q columns [c_lo, c_lo + G)
     const int c_hi = c_lo + p.group;
     const int rtok = (pj << 4) | (r & 15);
@@ -847,11 +866,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         if (!valid) {
           // zero this row of V (both 64-dim halves) so padding never reaches O
-          const uint32_t vrow = sbase + st * kStageBytes + kKBytes + r * 128;
+          const uint32_t vrow = sbase + st * kStageBytes + kKBytes + v_row_off;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             sts128_zero(vrow + k * 16);
-            sts128_zero(vrow + kRegion + k * 16);
+            sts128_zero(vrow + ht * 2048 + k * 16);
           }
         }
         fence_proxy_async_smem();
@@ -973,13 +992,21 @@ int launch_decode_tcgen05(const DecodeArgs& a) {
   if ((1 << sh.ht_shift) != a.item_heads) return PA_ERR_ARG;  // the plan's items differ
   const int64_t rows = static_cast<int64_t>(a.pool.num_blocks) * a.pool.num_kv_heads * 16;
   if (rows >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
-  TcParams p;
+  TcParams p{};
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(rows)};
     const uint64_t strides[1] = {kD * 2};
     const uint32_t box[2] = {64, static_cast<uint32_t>(16 << sh.ht_shift)};
     if (!encode_bf16_map(&p.tm_k, a.k_pool, 2, dims, strides, box)) return PA_ERR_CUDA;
     if (!encode_bf16_map(&p.tm_v, a.v_pool, 2, dims, strides, box)) return PA_ERR_CUDA;
+  }
+  {
+    // V: (dim within a 64-dim half, pool row, half) -- one copy moves a page's
+    // rows for both halves, half 0 first, as the second product reads them
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), 2};
+    const uint64_t strides[2] = {kD * 2, 128};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(16 << sh.ht_shift), 2};
+    if (!encode_bf16_map(&p.tm_v3, a.v_pool, 3, dims, strides, box)) return PA_ERR_CUDA;
   }
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(a.num_q_heads),
