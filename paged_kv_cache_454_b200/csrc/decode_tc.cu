@@ -431,12 +431,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             const uint64_t a0 = desc_add(desc_v0, st * kStageBytes);
             const uint64_t b0 = desc_add(desc_p0, b * L::kPBytes);
             const uint32_t dt = tmem + 2 * kN + b * kNpv;
+            // A = V^T (MN-major): 16 rows = 2 groups of 8; D halves ht*2 KiB apart
+            // B = P (K-major, kNpv rows = q columns): row half k/4, 32 bytes per 16 rows
+            if (ht == 8) {  // one page: slices 2 KiB apart (constant offsets)
 #pragma unroll
-            for (int k = 0; k < kRows / 16; ++k) {
-              // A = V^T (MN-major): 16 rows = 2 groups of 8; D halves ht*2 KiB apart
-              // B = P (K-major, kNpv rows = q columns): row half k/4, 32 bytes per 16 rows
-              umma_ss(dt, desc_add(a0, voff[k]), desc_add(b0, (k >> 2) * (kNpv * 128) + (k & 3) * 32),
-                      kIdescO, k > 0 ? 1u : 0u);
+              for (int k = 0; k < kRows / 16; ++k)
+                umma_ss(dt, desc_add(a0, k * 2048),
+                        desc_add(b0, (k >> 2) * (kNpv * 128) + (k & 3) * 32), kIdescO,
+                        k > 0 ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int k = 0; k < kRows / 16; ++k)
+                umma_ss(dt, desc_add(a0, voff[k]),
+                        desc_add(b0, (k >> 2) * (kNpv * 128) + (k & 3) * 32), kIdescO,
+                        k > 0 ? 1u : 0u);
             }
             umma_commit(&o_full[b]);
             umma_commit(&empty[st]);
