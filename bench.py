@@ -651,15 +651,15 @@ def main():
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # decode kernel from an ncu capture, keyed by workload and the kernel sources
 # it was taken with (reported as null once those sources change).  The
-# gqa70b_long figure is the 48-sequence capture (1,764,360,448 bytes for
+# gqa70b_long figure is the 48-sequence capture (1,760,201,728 bytes for
 # 1,755,018,024 algorithmic bytes) scaled by algorithmic bytes to the full
 # 128-sequence batch; the captures are summarised in profiles/.
 TRAFFIC = {
-    # 48-sequence capture of the same shape (1.00532 x its algorithmic bytes), scaled
-    "gqa70b_long": {"bytes": 4785885101, "sources": "58958c602ef2"},
+    # 48-sequence capture of the same shape (1.00295 x its algorithmic bytes), scaled
+    "gqa70b_long": {"bytes": 4774604438, "sources": "b0cf58fc4d2b"},
     # full-size captures
-    "llama13b_sampling": {"bytes": 2210495744, "sources": "58958c602ef2"},
-    "llama7b_decode": {"bytes": 1125037824, "sources": "58958c602ef2"},
+    "llama13b_sampling": {"bytes": 2156926208, "sources": "b0cf58fc4d2b"},
+    "llama7b_decode": {"bytes": 1121657600, "sources": "b0cf58fc4d2b"},
 }
 
 

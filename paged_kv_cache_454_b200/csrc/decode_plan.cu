@@ -4,9 +4,11 @@
 // tensor-core kernel).
 //
 //  * Partition length: `min_part` tokens, or -- when the caller leaves the
-//    choice to the library -- the largest power-of-two multiple of it (up to
-//    `max_part`) that still leaves at least `target_items` items, so long
-//    contexts are split only as far as load balance needs.
+//    choice to the library -- a power-of-two multiple of it up to `max_part`:
+//    the longest that still leaves at least `target_items` items (every item
+//    has a fixed cost, and longest-first order keeps the tail short), or, for
+//    shared prefixes, the longest whose items stay small next to one SM's
+//    share of the work (see below).
 //  * Order: longest items first (all full partitions, then the tails by
 //    decreasing length, then empty contexts), so a kernel that hands items out
 //    dynamically schedules them longest-processing-time first.
@@ -16,7 +18,8 @@
 //    block, then KV head, then sequence: the samples of a group read the shared
 //    pages of one KV head at the same time, so DRAM serves them once and L2
 //    the rest.  (Up to kSortMax sequences.)  A hash set of first blocks finds
-//    whether any repeats; the sort runs only then.
+//    whether any repeats; the sort runs only then, and only if some candidate
+//    length keeps every item at most 1/kLocalityShare of one SM's share.
 //  * It also clears the dynamic item counter and the per-(sequence, KV head)
 //    counters the tensor-core kernel uses to find the last partition to finish.
 #include "common.cuh"
@@ -44,6 +47,10 @@ __device__ __forceinline__ int bucket_of(int nunits) {
 constexpr int kSortMax = 1024;  // sequences the locality order sorts (one per thread)
 constexpr int kLensCache = 2048;  // sequences whose lengths the plan keeps in shared memory
 constexpr int kFirstSet = 2 * kSortMax;  // slots of the set that detects shared first blocks
+// In prefix order the longest item is at most 1/kLocalityShare of one SM's
+// share of the work (measured: 13B-shaped sampling batches are fastest with
+// 256-token items at this bound; longer items leave a long tail).
+constexpr int kLocalityShare = 16;
 static_assert(kFirstSet == 2048, "the set's hash keeps 11 bits");
 
 // Inclusive block-wide scan (sum or max) of one value per thread, 1024 threads.
@@ -82,12 +89,14 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
                                                            unsigned int* err) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
-  __shared__ int cand[4];
+  __shared__ int cand[4];      // items per KV-head group at each candidate length
+  __shared__ int cand_mx[4];   // longest item at each candidate length, in 128-token units
+  __shared__ int tiles_tot;    // context of all items in 128-token units (any length)
   __shared__ int bucket[kMaxBuckets];
   __shared__ int cursor[kMaxBuckets];
   __shared__ unsigned long long skey[kSortMax];  // (first block << 32 | sequence), sorted
   __shared__ int run_tab[2 * kSortMax];           // per run start: partition prefix, run total
-  __shared__ int sflag[4];                        // [0] any sharing, [1] max item tiles, [2] total tiles x KV heads
+  __shared__ int sflag[4];                        // [0] some first block repeats
   __shared__ int slens[kLensCache];               // context lengths as given (S <= kLensCache)
   __shared__ unsigned first_set[kFirstSet];       // open-addressing set of first blocks
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -112,34 +121,86 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     lens = slens;
   }
 
+  // ---- shared prefixes: does any first physical block repeat?  (a set in
+  // shared memory; the sort below runs only if one does and the items end up
+  // small enough) ----
+  if (tid < 4) sflag[tid] = 0;
+  __syncthreads();  // the set's initialisation and sflag
+  if (sortable && tid < S && clamp_len(lens[tid], max_blocks, nullptr) > 0) {
+    unsigned h = (my_first * 2654435761u) >> 21;  // 11 bits: kFirstSet slots
+    for (int probe = 0; probe < kFirstSet; ++probe, h = (h + 1) & (kFirstSet - 1)) {
+      const unsigned old = atomicCAS(&first_set[h], 0xffffffffu, my_first);
+      if (old == 0xffffffffu) break;
+      if (old == my_first) {
+        atomicOr(&sflag[0], 1);
+        break;
+      }
+    }
+  }
+
   // ---- partition length ----
+  // Without shared prefixes items run longest first, so the tail is short
+  // whatever their lengths, and every item costs a fixed start and finish:
+  // the longest candidate that still gives `target_items` items wins (the
+  // shortest when none does -- a small batch needs the parallelism).  With
+  // shared prefixes items run in prefix order instead, so the longest item
+  // must stay small next to one SM's share of the work: the longest candidate
+  // whose longest item is at most 1/kLocalityShare of that share, in which
+  // case the list takes the locality order.
   int ncand = 1;
   while (ncand < 4 && (min_part << ncand) <= max_part) ++ncand;
-  if (tid < 4) cand[tid] = 0;
+  if (tid < 4) {
+    cand[tid] = 0;
+    cand_mx[tid] = 0;
+  }
+  if (tid == 0) tiles_tot = 0;
   __syncthreads();
-  if (ncand > 1) {
-    int cnt[4] = {0, 0, 0, 0};
+  {
+    int cnt[4] = {0, 0, 0, 0}, mx[4] = {0, 0, 0, 0}, tt = 0;
     for (int s = tid; s < S; s += 1024) {
       const int L = clamp_len(lens[s], max_blocks, nullptr);
+      tt += (L + 127) / 128;
       for (int k = 0; k < ncand; ++k) {
         const int pk = min_part << k;
         const int n = (L + pk - 1) / pk;
         cnt[k] += n < 1 ? 1 : n;
+        mx[k] = max(mx[k], (min(L, pk) + 127) / 128);
       }
     }
+    for (int o = 16; o > 0; o >>= 1) tt += __shfl_xor_sync(0xffffffffu, tt, o);
+    if (lane == 0) atomicAdd(&tiles_tot, tt);
     for (int k = 0; k < ncand; ++k) {
-      int v = cnt[k];
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) atomicAdd(&cand[k], v);
+      int v = cnt[k], m = mx[k];
+      for (int o = 16; o > 0; o >>= 1) {
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      }
+      if (lane == 0) {
+        atomicAdd(&cand[k], v);
+        atomicMax(&cand_mx[k], m);
+      }
     }
   }
   __syncthreads();
-  int part = min_part;
-  for (int k = ncand - 1; k > 0; --k)
-    if (static_cast<long long>(cand[k]) * hkv >= target_items) {
-      part = min_part << k;
-      break;
-    }
+  int part = -1;
+  bool locality = false;
+  if (sortable && sflag[0]) {
+    const long long share = static_cast<long long>(tiles_tot) * hkv;
+    for (int k = ncand - 1; k >= 0; --k)
+      if (static_cast<long long>(cand_mx[k]) * kLocalityShare * num_sms <= share) {
+        part = min_part << k;
+        locality = true;
+        break;
+      }
+  }
+  if (part < 0) {
+    part = min_part;
+    for (int k = ncand - 1; k > 0; --k)
+      if (static_cast<long long>(cand[k]) * hkv >= target_items) {
+        part = min_part << k;
+        break;
+      }
+  }
   // items are bucketed by length in units of `unit` tokens: a page for short
   // partitions, coarser for long ones, so a partition is at most 64 units
   const int unit = part / 64 > 16 ? part / 64 : 16;
@@ -218,27 +279,8 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   }
   __syncthreads();
 
-  // ---- shared prefixes: does any first physical block repeat?  (a set in
-  // shared memory; the sort below runs only if one does) ----
-  bool locality = false;
-  if (sortable) {
-    if (tid < 4) sflag[tid] = 0;
-    __syncthreads();
-    if (tid < S && clamp_len(lens[tid], max_blocks, nullptr) > 0) {
-      unsigned h = (my_first * 2654435761u) >> 21;  // 11 bits: kFirstSet slots
-      for (int probe = 0; probe < kFirstSet; ++probe, h = (h + 1) & (kFirstSet - 1)) {
-        const unsigned old = atomicCAS(&first_set[h], 0xffffffffu, my_first);
-        if (old == 0xffffffffu) break;
-        if (old == my_first) {
-          atomicOr(&sflag[0], 1);
-          break;
-        }
-      }
-    }
-    __syncthreads();
-  }
   // ---- sort sequences by their first physical block ----
-  if (sortable && sflag[0]) {
+  if (locality) {
     int n2 = 1;
     while (n2 < S) n2 <<= 1;
     for (int i = tid; i < n2; i += 1024) {
@@ -269,15 +311,6 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
         __syncthreads();
       }
     }
-    if (tid < S) {
-      const int L = clamp_len(lens[tid], max_blocks, nullptr);
-      atomicMax(&sflag[1], (min(L, part) + 127) / 128);
-      atomicAdd(&sflag[2], ((L + 127) / 128) * hkv);
-    }
-    __syncthreads();
-    // order for locality only when no single item is large next to one SM's work
-    locality = sflag[0] &&
-               static_cast<long long>(sflag[1]) * 16 * num_sms <= static_cast<long long>(sflag[2]);
   }
   if (locality) {
     // thread i handles sorted position i (S <= 1024).  A run of equal first

@@ -94,13 +94,15 @@ int launch_decode_tcgen05(const DecodeArgs& a);  // merges split partitions itse
 int launch_decode_merge(const DecodeArgs& a);
 
 // Partition lengths (tokens) of the two decode kernels: the CUDA-core kernel
-// uses a fixed length; the tensor-core kernel starts from kTcPartition and
-// lengthens partitions up to kTcMaxPartition while each SM keeps at least
-// kTcItemsPerSm items.
+// uses a fixed length; the tensor-core kernel starts from kTcPartition (of one
+// KV head) and lengthens partitions up to kTcMaxPartition while each SM keeps
+// at least kTcItemsPerSm items (longest-first order keeps the tail short, and
+// every item has a fixed cost: a sweep of fixed lengths on B200 found the
+// longest such length fastest on the 7B-, 70B- and mixed-shaped batches).
 constexpr int kSimtPartition = 512;
 constexpr int kTcPartition = 1024;
 constexpr int kTcMaxPartition = 8192;
-constexpr int kTcItemsPerSm = 16;
+constexpr int kTcItemsPerSm = 2;
 
 struct PrefillArgs {
   const uint16_t* q;
