@@ -125,3 +125,25 @@ def test_python_binding_refuses_cpu_tensors():
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="missing"):
         _abi.load(str(tmp_path / "libpa.so"))
+
+
+def test_read_probe_host_argument_checks(lib):
+    fake = ctypes.c_void_p(0x10000)  # aligned, never dereferenced: calls fail first
+    odd = ctypes.c_void_p(0x10004)
+    call = lambda **kw: lib.pa_read_probe(
+        kw.get("k", fake), kw.get("v", fake), kw.get("pool", pool()), kw.get("tables", fake),
+        kw.get("max_blocks", 4), kw.get("lens", fake), kw.get("seqs", 3), kw.get("out", fake),
+        kw.get("ctas", 8), None)
+    assert call(pool=pool(bs=32)) == _abi.PA_ERR_UNSUPPORTED
+    assert call(pool=pool(d=96)) == _abi.PA_ERR_UNSUPPORTED
+    assert call(ctas=0) == _abi.PA_ERR_ARG
+    assert call(ctas=65536) == _abi.PA_ERR_ARG
+    assert call(seqs=-1) == _abi.PA_ERR_ARG
+    assert call(seqs=4097) == _abi.PA_ERR_ARG
+    assert call(max_blocks=-1) == _abi.PA_ERR_ARG
+    assert call(k=None) == _abi.PA_ERR_ARG
+    assert call(out=None) == _abi.PA_ERR_ARG
+    assert call(tables=None) == _abi.PA_ERR_ARG
+    assert call(lens=None) == _abi.PA_ERR_ARG
+    assert call(v=odd) == _abi.PA_ERR_ARG
+    assert call(out=odd) == _abi.PA_ERR_ARG
