@@ -7,9 +7,12 @@ of ``bench.py`` may import it.  It shares no code with the CUDA path and imports
 nothing from it; the only thing both sides share is the seeded input generator
 in ``workloads``.
 
-Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
-invariants the pages state, a brute-force scalar implementation and the pages'
-own worked numbers; see each docstring for the passage it follows.
+The attention functions are pinned by ``tests/test_oracle_pins.py`` against
+closed forms, invariants the pages state, a brute-force scalar implementation
+and the pages' own worked numbers; the block manager by
+``tests/test_kv_manager_oracle.py``, the sampler by ``tests/test_sampler_oracle.py``
+and the block swap by ``tests/test_swap_oracle.py``.  Each docstring names the
+passage it follows.
 """
 from .paged_attention import (  # noqa: F401
     bf16_bits_to_f64,
