@@ -25,8 +25,10 @@ def _i32(a) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
 
 
-def _p(a: np.ndarray):
-    return a.ctypes.data_as(ctypes.c_void_p)
+def _p(a: np.ndarray) -> int:
+    # the address as a plain int (the argument types are c_void_p): half the
+    # cost of building a c_void_p object per argument
+    return a.ctypes.data
 
 
 class KvManager:
@@ -42,6 +44,11 @@ class KvManager:
         self.num_blocks = num_blocks
         self.block_size = block_size
         self.prefix_caching = prefix_caching
+        # scratch the per-step call reuses: copy pairs and their count
+        self._pairs = np.empty((0, 2), np.int64)
+        self._pairs_addr = self._pairs.ctypes.data
+        self._npairs = ctypes.c_int32(0)
+        self._npairs_ref = ctypes.byref(self._npairs)
 
     def close(self):
         if self._h:
@@ -92,12 +99,14 @@ class KvManager:
             slots = np.empty(len(ids), np.int64)
         elif slots.shape != (len(ids),) or slots.dtype != np.int64:
             raise ValueError("slots does not match the batch")
-        pairs = np.empty((max(len(ids), 1), 2), np.int64)
-        npairs = ctypes.c_int32(0)
+        if self._pairs.shape[0] < max(len(ids), 1):
+            self._pairs = np.empty((max(len(ids), 1), 2), np.int64)
+            self._pairs_addr = self._pairs.ctypes.data
         self._check("pa_kvm_decode_step",
                     self._lib.pa_kvm_decode_step(self._h, _p(ids), len(ids), _p(t), _p(slots),
-                                                 _p(pairs), ctypes.byref(npairs)))
-        return slots, [(int(a), int(b)) for a, b in pairs[:npairs.value]]
+                                                 self._pairs_addr, self._npairs_ref))
+        n = self._npairs.value
+        return slots, [(int(a), int(b)) for a, b in self._pairs[:n]] if n else []
 
     def fork(self, parent: int, child: int):
         self._check("pa_kvm_fork", self._lib.pa_kvm_fork(self._h, parent, child))
