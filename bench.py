@@ -342,8 +342,9 @@ def step_stats(ev, first, last):
     v = sorted(b.elapsed_time(c) for b, c in zip(ev[first], ev[last]))
     if not v:
         return None
+    p90 = v[max(0, math.ceil(0.9 * len(v)) - 1)]  # nearest rank
     return {"min": round(v[0], 4), "median": round(statistics.median(v), 4),
-            "p90": round(v[min(len(v) - 1, int(0.9 * len(v)))], 4)}
+            "p90": round(p90, 4)}
 
 
 def e2e_run(w: Workload, stream, steps, warmup):

@@ -67,3 +67,22 @@ def test_max_over_ranks_without_group():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks([1, 2.5]) == [1.0, 2.5]
+
+
+def test_step_stats_min_median_p90():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Ev:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    # spans 1..10 ms in scrambled order
+    spans = [7, 3, 10, 1, 5, 9, 2, 8, 4, 6]
+    ev = {"a": [Ev(0.0) for _ in spans], "b": [Ev(float(s)) for s in spans]}
+    st = bench.step_stats(ev, "a", "b")
+    assert st == {"min": 1.0, "median": 5.5, "p90": 9.0}  # nearest rank: 9th of 10
+    assert bench.step_stats({"a": [], "b": []}, "a", "b") is None
