@@ -12,8 +12,11 @@ import gpu_helpers as H
 pytestmark = pytest.mark.gpu
 
 
-def _samples(lay, rows, k_random=2, seed=0):
-    """First, last, longest, shortest and a few random rows of `rows`."""
+def _samples(lay, rows, k_random=6, seed=0):
+    """First, last, longest, shortest and a few random rows of `rows`; where
+    rows share their first physical block (samples of one prompt, which the
+    plan may lay out side by side), every row sharing it with the first and
+    the last row too."""
     rows = list(rows)
     if not rows:
         return []
@@ -21,6 +24,8 @@ def _samples(lay, rows, k_random=2, seed=0):
     pick = {rows[0], rows[-1], rows[int(np.argmax(lens))], rows[int(np.argmin(lens))]}
     rng = np.random.default_rng(seed)
     pick.update(int(x) for x in rng.choice(rows, size=min(k_random, len(rows)), replace=False))
+    first = {int(lay.block_tables[r, 0]) for r in (rows[0], rows[-1]) if lay.context_lens[r] > 0}
+    pick.update(r for r in rows if lay.context_lens[r] > 0 and int(lay.block_tables[r, 0]) in first)
     return sorted(pick)
 
 

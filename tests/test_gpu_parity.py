@@ -57,8 +57,11 @@ def lay_shared():
 
 
 def lay_shared_many():
-    # enough small items (160 sequences x 32 KV heads, one tile each) that the
-    # work plan orders them by shared first block instead of by length
+    # 160 short sequences x 32 KV heads sharing first blocks: the plan finds the
+    # sharing, but the batch is too small for prefix order (an item would be
+    # more than 1/16 of an SM's share), so it runs longest first.  Prefix order
+    # needs about a GB of context at 148 SMs; the full-size sampling batch
+    # (tests/test_gpu_fullsize.py) runs it.
     lay = synth.llama13b_sampling(seed=112, groups=40, samples=4, prefix=64, max_suffix=60)
     lay.num_q_heads = lay.num_kv_heads = 32
     return lay
