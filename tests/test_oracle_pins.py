@@ -538,6 +538,46 @@ def test_poison_is_never_read():
     check_poison_is_never_read()
 
 
+# ----------------------------------------------------------------------------
+# Library softmax on contiguous tensors
+# ----------------------------------------------------------------------------
+def check_matches_library_softmax():
+    """Decode and causal prefill through an identity table equal
+    ``scipy.special.softmax(scale * Q K^T) V`` on the contiguous tensors, and the
+    log-sum-exp equals ``scipy.special.logsumexp`` of the scaled scores."""
+    from scipy.special import logsumexp, softmax
+    rng = np.random.default_rng(31)
+    hq, hkv, d, L, n = 4, 2, 32, 45, 7
+    K = bits(rng.normal(size=(hkv, L, d)))
+    V = bits(rng.normal(size=(hkv, L, d)))
+    kp, vp, table = contiguous_to_pool(K, V)
+    Kf, Vf = f64(K), f64(V)
+    scale = 0.37
+    # decode: one query per head over all L keys
+    q = bits(rng.normal(size=(1, hq, d)))
+    out, lse = oracle.decode(q, kp, vp, table[None, :], np.array([L]), scale)
+    for h in range(hq):
+        g = h // (hq // hkv)
+        s = scale * (Kf[g] @ f64(q[0, h]))
+        assert np.allclose(out[0, h], softmax(s) @ Vf[g], rtol=0, atol=1e-12)
+        assert abs(lse[0, h] - logsumexp(s)) < 1e-12
+    # prefill: the last n positions as the chunk, causal mask as -inf
+    qp = bits(rng.normal(size=(n, hq, d)))
+    outp, lsep = oracle.chunked_prefill(qp, np.array([0, n]), kp, vp, table[None, :],
+                                        np.array([L]), scale)
+    for i in range(n):
+        for h in range(hq):
+            g = h // (hq // hkv)
+            s = scale * (Kf[g] @ f64(qp[i, h]))
+            s[L - n + i + 1:] = -np.inf
+            assert np.allclose(outp[i, h], softmax(s) @ Vf[g], rtol=0, atol=1e-12)
+            assert abs(lsep[i, h] - logsumexp(s)) < 1e-12
+
+
+def test_matches_library_softmax():
+    check_matches_library_softmax()
+
+
 ALL_CHECKS = [
     check_bf16_widening, check_addressing_golden, check_identity_table,
     check_permutation_invariance, check_hand_example, check_single_token_is_v0,
@@ -546,4 +586,6 @@ ALL_CHECKS = [
     check_brute_force_decode, check_brute_force_prefill, check_prefill_one_token_is_decode,
     check_chunk_split_equivalence, check_prefill_causal_boundary, check_reshape_and_cache,
     check_copy_blocks, check_shared_prefix_equals_unshared, check_poison_is_never_read,
+    check_matches_library_softmax,
 ]
+
