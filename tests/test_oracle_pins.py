@@ -561,17 +561,19 @@ def check_matches_library_softmax():
         s = scale * (Kf[g] @ f64(q[0, h]))
         assert np.allclose(out[0, h], softmax(s) @ Vf[g], rtol=0, atol=1e-12)
         assert abs(lse[0, h] - logsumexp(s)) < 1e-12
-    # prefill: the last n positions as the chunk, causal mask as -inf
-    qp = bits(rng.normal(size=(n, hq, d)))
-    outp, lsep = oracle.chunked_prefill(qp, np.array([0, n]), kp, vp, table[None, :],
-                                        np.array([L]), scale)
-    for i in range(n):
-        for h in range(hq):
-            g = h // (hq // hkv)
-            s = scale * (Kf[g] @ f64(qp[i, h]))
-            s[L - n + i + 1:] = -np.inf
-            assert np.allclose(outp[i, h], softmax(s) @ Vf[g], rtol=0, atol=1e-12)
-            assert abs(lsep[i, h] - logsumexp(s)) < 1e-12
+    # prefill: the last n positions as the chunk (and, with n = L, no cached
+    # context: plain causal self-attention), causal mask as -inf
+    for nn in (n, L):
+        qp = bits(rng.normal(size=(nn, hq, d)))
+        outp, lsep = oracle.chunked_prefill(qp, np.array([0, nn]), kp, vp, table[None, :],
+                                            np.array([L]), scale)
+        for i in range(nn):
+            for h in range(hq):
+                g = h // (hq // hkv)
+                s = scale * (Kf[g] @ f64(qp[i, h]))
+                s[L - nn + i + 1:] = -np.inf
+                assert np.allclose(outp[i, h], softmax(s) @ Vf[g], rtol=0, atol=1e-12)
+                assert abs(lsep[i, h] - logsumexp(s)) < 1e-12
 
 
 def test_matches_library_softmax():
