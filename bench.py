@@ -447,10 +447,8 @@ def e2e_run(w: Workload, stream, steps, warmup):
 def oracle_sample_runner(w: Workload):
     """Returns (prepare(rows), run(prepared, groups)).  ``prepare`` takes host
     copies of exactly the device inputs of some decode rows (before any library
-    call wrote to the pools); ``run`` times the oracle's copy / cache write /
-    decode over the first ``groups`` KV heads of them (KV-head groups are
-    independent, so this is an exact slice of the step's work)."""
-    import oracle
+    call wrote to the pools); ``run`` (``oracle_step``) times the oracle's copy /
+    cache write / decode over the first ``groups`` KV heads of them."""
     torch = w.torch
     lay = w.layout
 
@@ -466,20 +464,41 @@ def oracle_sample_runner(w: Workload):
         val = bits(w.t["value"].index_select(0, tok))
         return sub, kp, vp, q, key, val
 
-    def run(prepared, groups=None):
-        sub, kp, vp, q, key, val = prepared
-        ng = sub.num_kv_heads if groups is None else groups
-        G = sub.group_size
-        kp, vp = kp[:, :ng], vp[:, :ng]
-        key, val, q = key[:, :ng], val[:, :ng], q[:, : ng * G]
-        t0 = time.perf_counter()
-        if sub.copy_pairs.size:
-            kp, vp = oracle.copy_blocks(kp, vp, sub.copy_pairs)
-        kp, vp = oracle.reshape_and_cache(kp, vp, key, val, sub.slot_mapping())
-        oracle.decode(q, kp, vp, sub.block_tables, sub.context_lens, sub.scale)
-        return time.perf_counter() - t0
+    return prepare, oracle_step
 
-    return prepare, run
+
+def oracle_step(prepared, groups=None):
+    """Seconds the oracle takes for the copy-on-write copies, the cache write and
+    the decode of one prepared slice ``(sub_layout, k_pool, v_pool, q, key,
+    value)``, restricted to its first ``groups`` KV heads (KV-head groups are
+    independent, so this is an exact slice of the work)."""
+    import oracle
+    sub, kp, vp, q, key, val = prepared
+    ng = sub.num_kv_heads if groups is None else groups
+    G = sub.group_size
+    kp, vp = kp[:, :ng], vp[:, :ng]
+    key, val, q = key[:, :ng], val[:, :ng], q[:, : ng * G]
+    t0 = time.perf_counter()
+    if sub.copy_pairs.size:
+        kp, vp = oracle.copy_blocks(kp, vp, sub.copy_pairs)
+    kp, vp = oracle.reshape_and_cache(kp, vp, key, val, sub.slot_mapping())
+    oracle.decode(q, kp, vp, sub.block_tables, sub.context_lens, sub.scale)
+    return time.perf_counter() - t0
+
+
+def host_oracle_slices(workload: str, rows: int = 4):
+    """Host-only inputs for the reference arm: the workload's first ``rows``
+    decode sequences, each over a compact pool of exactly its blocks, drawn on
+    the host (``synth.fill_host``: the same shapes, value distribution and
+    poisons as the device batch, from NumPy's generator).  Neither torch nor the
+    CUDA library is touched."""
+    lay = synth.CONFIGS[workload]()
+    out = []
+    for r in list(lay.decode_rows())[:rows]:
+        sub, _ = synth.subset(lay, [int(r)])
+        h = synth.fill_host(sub)
+        out.append((sub, h["k_pool"], h["v_pool"], h["q"], h["key"], h["value"]))
+    return lay, out
 
 
 def blas_threads():
@@ -554,13 +573,22 @@ def main():
         cpu = cpu_baseline(w, a.cpu_budget)
 
     stream = torch.cuda.Stream(device=dev)
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(a.warmup):
         w.step(stream)
     torch.cuda.synchronize()
+    # Clock soak: more untimed steps until the GPU has run this load for at
+    # least 1 s, so the clock record (100 ms samples from here to the end of
+    # the e2e leg) holds the steady state the timed region runs in.
+    soak_steps, soak_t0 = 0, time.perf_counter()
+    while time.perf_counter() - soak_t0 < 1.0:
+        for _ in range(10):
+            w.step(stream)
+        soak_steps += 10
+        torch.cuda.synchronize()
     if pg:
         pg.barrier()
-    clocks = ClockSampler(local)
-    clocks.start()
     ev = {}
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -583,6 +611,9 @@ def main():
     if not a.skip_e2e:
         e2e_ms, h2d, d2h = e2e_run(w, stream, max(10, a.steps // 4), a.warmup)
     clk = clocks.stop()
+    if clk:
+        clk["window"] = (f"{soak_steps} untimed steps (>= 1 s) right before the timed region, "
+                         "the timed region and the e2e leg")
     if pg:
         ms, e2e_ms = max_over_ranks([ms, e2e_ms if not a.skip_e2e else 0.0], pg, dev)
     if not a.skip_e2e:
@@ -687,31 +718,26 @@ def traffic_for(workload, w):
 def reference_arm(a, rank, world):
     """The CPU oracle as the reference: each step runs the oracle over a bounded
     slice (some KV-head groups of one decode sequence) of the same workload,
-    sized so the whole run stays within about two minutes."""
+    sized so the whole run stays within about two minutes.  Its inputs are drawn
+    on the host; this arm imports neither torch nor the CUDA library."""
     if rank != 0:
         return
-    import torch
-    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
-    if dev.type == "cuda":
-        torch.cuda.set_device(0)
-    w = Workload(a.workload, None, dev)
-    prepare, run = oracle_sample_runner(w)
-    rows = list(w.dec)
-    prepared = [prepare([r]) for r in rows[: min(len(rows), 4)]]
-    hkv = w.layout.num_kv_heads
-    probe = max(run(p, 1) for p in prepared)  # one KV group of the longest sample
+    lay, prepared = host_oracle_slices(a.workload)
+    hkv = lay.num_kv_heads
+    probe = max(oracle_step(p, 1) for p in prepared)  # one KV group of the longest sample
     budget = 120.0 / (a.steps + a.warmup)
     groups = int(max(1, min(hkv, budget // max(probe, 1e-6))))
     for i in range(a.warmup):
-        run(prepared[i % len(prepared)], groups)
+        oracle_step(prepared[i % len(prepared)], groups)
     secs, toks = 0.0, 0.0
     for i in range(a.steps):
-        secs += run(prepared[i % len(prepared)], groups)
+        secs += oracle_step(prepared[i % len(prepared)], groups)
         toks += groups / hkv
     value = toks / secs
     sample = (f"each step: oracle copy/cache-write/decode of {groups} of {hkv} KV-head groups "
-              f"(all their q heads) of one decode sequence of {w.name} (cycling over the first "
-              f"{len(prepared)}), NumPy fp64; counted as {groups}/{hkv} of a token")
+              f"(all their q heads) of one decode sequence of {a.workload} (cycling over the "
+              f"first {len(prepared)}; inputs drawn on the host with the workload's shapes), "
+              f"NumPy fp64; counted as {groups}/{hkv} of a token")
     res = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
            "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
            "ms_per_step": secs / max(1, a.steps) * 1e3, "higher_is_better": True,

@@ -25,6 +25,11 @@
  *     pa_get_device_error() returns and clears.
  *   - Every pointer argument must be 16-byte aligned; strides are in elements
  *     and must be multiples of 8 (16 bytes).
+ *   - The library caches, per device and for the life of the process, the
+ *     device address of its error word (and of the scratch array of
+ *     pa_decode_noalloc).  Do not keep using it after cudaDeviceReset().
+ *   - Each entry point opens an NVTX range named after itself (visible in
+ *     Nsight Systems timelines); a build with -DPA_NO_NVTX has none.
  *
  * Pool layout (both pools):  bf16 [num_blocks][num_kv_heads][block_size][head_dim],
  * densely packed.  One (block, kv head) page is block_size*head_dim contiguous
@@ -129,14 +134,18 @@ PA_API int pa_copy_blocks(void* k_pool, void* v_pool, pa_pool_desc pool, const i
  *     lse[s][h] = log(sum_t exp(x_t))          (natural log)
  * where K_s[g][t] = k_pool[block_tables[s][t / bs]][g][t % bs].  Long contexts
  * are split into partitions whose partial results are merged by their
- * log-sum-exp (a second kernel on the same stream).  L == 0 gives out = 0 and
- * lse = -inf.
+ * log-sum-exp (inside the tensor-core decode kernel, by the CTA that finishes
+ * a sequence's last partition; by a second kernel on the same stream on the
+ * CUDA-core path).  L == 0 gives out = 0 and lse = -inf.
  *
  *   q              bf16 [num_seqs][num_q_heads][head_dim], token stride q_stride
  *                  elements (>= num_q_heads*head_dim); heads packed.
  *   block_tables   int32 [num_seqs][max_blocks_per_seq]; entries past
  *                  ceil(L/bs) are never read.
  *   context_lens   int32 [num_seqs]; 0 <= L <= max_blocks_per_seq*block_size.
+ *                  A table able to describe more than 65535 partitions of
+ *                  the shortest partition length (about 8.4M tokens at 128)
+ *                  returns PA_ERR_UNSUPPORTED, as do more than 32767 KV heads.
  *   out            bf16 [num_seqs][num_q_heads][head_dim], packed.
  *   lse            float [num_seqs][num_q_heads], or NULL.
  *   workspace      device scratch of at least pa_decode_workspace_size() bytes
@@ -192,9 +201,17 @@ PA_API int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, con
  *   - All calls on a device share the array and it keeps the last call's
  *     contents; nothing in it needs to start at zero.  Calls whose kernels
  *     overlap on the GPU (e.g. on two streams) race on it: do not issue them.
- *   - A batch whose workspace (pa_decode_workspace_size for the same sizes)
- *     exceeds PA_NOALLOC_SCRATCH_BYTES returns PA_ERR_WORKSPACE and launches
+ *   - The call needs the workspace of the kernel pa_decode would choose for
+ *     the same sizes.  pa_decode_workspace_size() is an upper bound of that
+ *     need (it sizes for either kernel): a batch whose
+ *     pa_decode_workspace_size() is at most PA_NOALLOC_SCRATCH_BYTES always
+ *     fits.  A larger batch still runs when the chosen kernel's own need fits
+ *     (typically GQA batches on the tensor-core kernel, whose partitions are
+ *     longer); otherwise the call returns PA_ERR_WORKSPACE and launches
  *     nothing.  Other errors as for pa_decode.
+ *   - The array's device address is cached per device for the life of the
+ *     process: do not use the library across a cudaDeviceReset() (the same
+ *     holds for the device error word every call uses).
  */
 #define PA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 

@@ -1,6 +1,7 @@
 """Build ``libpa.so`` (the C-ABI PagedAttention library) in-tree with nvcc for sm_100a.
 
-Usage: ``python -m paged_kv_cache_454_b200.build [--verbose] [--ptxas-info]``.
+Usage: ``python -m paged_kv_cache_454_b200.build [--verbose] [--ptxas-info]``
+(``PA_NO_NVTX=1`` in the environment compiles the NVTX ranges out).
 Object files go to ``_build/`` at the repository root; the shared library lands
 next to this file, where the Python binding loads it from.
 """
@@ -23,6 +24,9 @@ LIB = os.path.join(HERE, "libpa.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--use_fast_math", "-Xcompiler", "-fPIC",
               "-Xcompiler", "-fvisibility=hidden", "-I" + os.path.join(ROOT, "include")]
+# PA_NO_NVTX=1 in the environment builds the library without its NVTX ranges
+if os.environ.get("PA_NO_NVTX", "") not in ("", "0"):
+    NVCC_FLAGS.append("-DPA_NO_NVTX")
 
 
 def nvcc() -> str:

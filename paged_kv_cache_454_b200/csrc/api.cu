@@ -171,6 +171,7 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
                  const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads, float scale,
                  void* out, float* lse, void* workspace, size_t workspace_bytes,
                  int32_t partition_tokens, int32_t kernel, void* stream) {
+  PA_NVTX_RANGE("pa_decode_ex");
   int st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0) return PA_ERR_ARG;
@@ -199,6 +200,8 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
     if (part > cap) part = static_cast<int>(cap < 128 ? 128 : cap);
   }
   const int max_parts = max_parts_for(max_blocks_per_seq, pool.block_size, part);
+  // work items carry (KV-head group << 16 | partition) in one int32
+  if (max_parts > 0xffff || pool.num_kv_heads > 0x7fff) return PA_ERR_UNSUPPORTED;
   const size_t need = decode_workspace_bytes(num_seqs, num_q_heads, pool.num_kv_heads,
                                              pool.head_dim, max_parts);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
@@ -249,6 +252,7 @@ int pa_decode(const void* q, int64_t q_stride, const void* k_pool, const void* v
               pa_pool_desc pool, const int32_t* block_tables, int32_t max_blocks_per_seq,
               const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads, float scale,
               void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  PA_NVTX_RANGE("pa_decode");
   return pa_decode_ex(q, q_stride, k_pool, v_pool, pool, block_tables, max_blocks_per_seq,
                       context_lens, num_seqs, num_q_heads, scale, out, lse, workspace,
                       workspace_bytes, 0, PA_KERNEL_AUTO, stream);
@@ -260,6 +264,7 @@ int pa_chunked_prefill(const void* q, int64_t q_stride, const int32_t* cu_q_lens
                        int32_t max_blocks_per_seq, const int32_t* context_lens,
                        int32_t num_seqs, int32_t num_q_heads, float scale, void* out, float* lse,
                        void* stream) {
+  PA_NVTX_RANGE("pa_chunked_prefill");
   int st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || num_q_heads <= 0 ||
@@ -299,6 +304,7 @@ int pa_chunked_prefill(const void* q, int64_t q_stride, const int32_t* cu_q_lens
 }
 
 int pa_get_device_error(uint32_t* flags_host, void* stream) {
+  PA_NVTX_RANGE("pa_get_device_error");
   if (!flags_host) return PA_ERR_ARG;
   unsigned int* w = device_error_word();
   if (!w) return PA_ERR_CUDA;

@@ -127,6 +127,7 @@ extern "C" {
 int pa_reshape_and_cache(const void* key, const void* value, int64_t token_stride, void* k_pool,
                          void* v_pool, pa_pool_desc pool, const int64_t* slot_mapping,
                          int32_t num_tokens, void* stream) {
+  PA_NVTX_RANGE("pa_reshape_and_cache");
   int st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_tokens < 0) return PA_ERR_ARG;
@@ -152,6 +153,7 @@ int pa_reshape_and_cache(const void* key, const void* value, int64_t token_strid
 
 int pa_copy_blocks(void* k_pool, void* v_pool, pa_pool_desc pool, const int64_t* pairs_host,
                    int32_t num_pairs, void* stream) {
+  PA_NVTX_RANGE("pa_copy_blocks");
   int st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_pairs < 0) return PA_ERR_ARG;
@@ -192,6 +194,7 @@ int pa_gather_kv(const void* k_pool, const void* v_pool, pa_pool_desc pool,
                  const int32_t* block_tables, int32_t max_blocks_per_seq,
                  const int32_t* context_lens, const int32_t* cu_kv_lens, int32_t num_seqs,
                  int32_t max_context, void* k_out, void* v_out, void* stream) {
+  PA_NVTX_RANGE("pa_gather_kv");
   int st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || max_context < 0 || max_blocks_per_seq <= 0) return PA_ERR_ARG;

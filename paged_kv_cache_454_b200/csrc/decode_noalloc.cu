@@ -52,6 +52,7 @@ extern "C" int pa_decode_noalloc(const void* q, int64_t q_stride, const void* k_
                                  const int32_t* context_lens, int32_t num_seqs,
                                  int32_t num_q_heads, float scale, void* out, float* lse,
                                  void* stream) {
+  PA_NVTX_RANGE("pa_decode_noalloc");
   void* scratch = scratch_address();
   if (!scratch) return PA_ERR_CUDA;
   // pa_decode_ex checks every argument and returns PA_ERR_WORKSPACE, launching

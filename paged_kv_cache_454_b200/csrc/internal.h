@@ -7,6 +7,10 @@
 
 #include "../../include/pa.h"
 
+#ifndef PA_NO_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 namespace pa {
 
 // Device address of the sticky error word of the current device (looked up
@@ -17,6 +21,22 @@ unsigned int* device_error_word();
 int num_sms();
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// An NVTX range around one C-ABI call (named after the entry point), so a
+// profiler timeline shows which library call each kernel belongs to.  NVTX is
+// header-only: without a profiler attached a push/pop costs a few nanoseconds
+// and loads nothing.  -DPA_NO_NVTX compiles the ranges out.
+#ifndef PA_NO_NVTX
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define PA_NVTX_RANGE(name) ::pa::NvtxRange pa_nvtx_range_(name)
+#else
+#define PA_NVTX_RANGE(name) ((void)0)
+#endif
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

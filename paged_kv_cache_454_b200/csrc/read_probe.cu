@@ -219,6 +219,7 @@ extern "C" int pa_read_probe(const void* k_pool, const void* v_pool, pa_pool_des
                              const int32_t* block_tables, int32_t max_blocks_per_seq,
                              const int32_t* context_lens, int32_t num_seqs,
                              uint64_t* partial_sums, int32_t num_ctas, void* stream) {
+  PA_NVTX_RANGE("pa_read_probe");
   int st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || num_seqs > PA_PROBE_MAX_SEQS || max_blocks_per_seq < 0) return PA_ERR_ARG;

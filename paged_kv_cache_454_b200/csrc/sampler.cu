@@ -484,6 +484,7 @@ using namespace pa;
 extern "C" int pa_sample(const float* logits, int64_t row_stride, int32_t num_rows, int32_t vocab,
                          const float* temperature, const int32_t* top_k, const float* top_p,
                          const float* uniform, int32_t* tokens, void* stream) {
+  PA_NVTX_RANGE("pa_sample");
   if (num_rows < 0 || vocab <= 0 || row_stride < vocab) return PA_ERR_ARG;
   if (num_rows == 0) return PA_OK;
   if (!logits || !temperature || !top_k || !top_p || !uniform || !tokens) return PA_ERR_ARG;

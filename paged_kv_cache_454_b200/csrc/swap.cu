@@ -65,6 +65,7 @@ using namespace pa;
 extern "C" int pa_swap_blocks(void* k_pool, void* v_pool, pa_pool_desc pool, void* k_host,
                               void* v_host, int32_t num_host_blocks, const int64_t* pairs_host,
                               int32_t num_pairs, int32_t direction, void* stream) {
+  PA_NVTX_RANGE("pa_swap_blocks");
   int st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_pairs < 0 || num_host_blocks < 0) return PA_ERR_ARG;

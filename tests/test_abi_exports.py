@@ -147,3 +147,23 @@ def test_read_probe_host_argument_checks(lib):
     assert call(lens=None) == _abi.PA_ERR_ARG
     assert call(v=odd) == _abi.PA_ERR_ARG
     assert call(out=odd) == _abi.PA_ERR_ARG
+
+
+@pytest.mark.parametrize("flags", [[], ["-DPA_NO_NVTX"]], ids=["nvtx", "no_nvtx"])
+def test_nvtx_range_compiles_in_and_out(tmp_path, flags):
+    # the range guard every entry point opens, built with and without NVTX
+    import shutil
+    import subprocess
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / "r.cpp"
+    src.write_text('#include "internal.h"\n'
+                   'int f() { PA_NVTX_RANGE("pa_test"); return 7; }\n'
+                   'int main() { return f() == 7 ? 0 : 1; }\n')
+    csrc = os.path.join(ROOT, "paged_kv_cache_454_b200", "csrc")
+    exe = tmp_path / "r"
+    r = subprocess.run([gxx, "-std=c++17", "-I", csrc, "-I", "/usr/local/cuda/include", *flags,
+                        str(src), "-o", str(exe), "-ldl"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0

@@ -80,15 +80,24 @@ def test_noalloc_rejects_batches_beyond_its_scratch():
     lib = _abi.load()
     lay = _layouts()[0]
     st = _prepared(lay)
-    # a table width of 2^20 blocks per sequence asks for far more scratch than
-    # the array holds: rejected on the host, nothing launched
-    S, hq = 64, lay.num_q_heads
-    need = lib.pa_decode_workspace_size(S, hq, _abi.PoolDesc(*st.k_pool.shape), 1 << 20)
+    # 64 sequences with tables of 16384 blocks (4 MiB of int32) need about
+    # 135 MB of split-context scratch, twice what the array holds: rejected on
+    # the host, nothing launched.  Every buffer is sized for the declared
+    # shapes (q rows, lengths, table width), so a launch, were the check ever
+    # to regress, would read nothing out of bounds and the assert below fails
+    # cleanly instead.
+    S, hq, mb = 64, lay.num_q_heads, 16384
+    pool = _abi.PoolDesc(*st.k_pool.shape)
+    need = lib.pa_decode_workspace_size(S, hq, pool, mb)
     assert need > _abi.PA_NOALLOC_SCRATCH_BYTES
+    q = torch.zeros((S, hq, lay.head_dim), dtype=torch.bfloat16, device="cuda")
+    lens = torch.zeros(S, dtype=torch.int32, device="cuda")
+    tables = torch.zeros((S, mb), dtype=torch.int32, device="cuda")
     out = torch.zeros((S, hq, lay.head_dim), dtype=torch.bfloat16, device="cuda")
     status = lib.pa_decode_noalloc(
-        st.q.data_ptr(), hq * lay.head_dim, st.k_pool.data_ptr(), st.v_pool.data_ptr(),
-        _abi.PoolDesc(*st.k_pool.shape), st.tables.data_ptr(), 1 << 20, st.lens.data_ptr(), S,
-        hq, ctypes.c_float(lay.scale), out.data_ptr(), None,
-        torch.cuda.current_stream().cuda_stream)
+        q.data_ptr(), q.stride(0), st.k_pool.data_ptr(), st.v_pool.data_ptr(), pool,
+        tables.data_ptr(), mb, lens.data_ptr(), S, hq, ctypes.c_float(lay.scale),
+        out.data_ptr(), None, torch.cuda.current_stream().cuda_stream)
     assert status == _abi.PA_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out).item() == 0  # nothing ran
