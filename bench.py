@@ -68,26 +68,96 @@ def max_over_ranks(values, dist=None, device="cpu"):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock, power and throttle-reason samples while the benchmark runs.
 
+    Reads NVML (read-only queries) every ``interval_s`` from a background
+    thread, with host timestamps, so even a timed region of a few milliseconds
+    gets samples; ``mark_timed(start, end)`` brackets the timed region and the
+    record reports its samples (and those of the whole window for context).
+    Falls back to ``nvidia-smi -lms 100`` when NVML cannot be used."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, interval_s: float = 0.002):
         self.idx = device_index
+        self.interval = interval_s
+        self.samples = []  # (host time, sm MHz, max sm MHz, reasons bitmask, watts)
+        self.window = None
+        self.thread = None
         self.proc = None
+        self.stop_flag = False
+        self.source = None
 
     def start(self):
+        import threading
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            return self._start_smi()
+        self.source = "nvml"
+
+        def run():
+            while not self.stop_flag:
+                try:
+                    self.samples.append((time.perf_counter(),
+                                         pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                         smax,
+                                         pynvml.nvmlDeviceGetCurrentClocksEventReasons(h),
+                                         pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0))
+                except Exception:
+                    pass
+                time.sleep(self.interval)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def _start_smi(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi"
         except (OSError, FileNotFoundError):
             self.proc = None
 
+    def mark_timed(self, t_start, t_end):
+        self.window = (t_start, t_end)
+
+    def _summary(self, rows):
+        if not rows:
+            return None
+        mhz = [r[1] for r in rows]
+        reasons = sorted({n for r in rows for n, bit in self.REASONS if r[3] & bit})
+        return {"sm_mhz": statistics.median(mhz), "sm_min_mhz": min(mhz),
+                "sm_max_mhz": max(r[2] for r in rows), "samples": len(rows),
+                "reasons": reasons,
+                "power_w_median": round(statistics.median(r[4] for r in rows), 1)}
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            rows = list(self.samples)
+            timed = rows
+            if self.window:
+                timed = [r for r in rows if self.window[0] <= r[0] <= self.window[1]]
+            res = self._summary(timed) or self._summary(rows)
+            if res is None:
+                return None
+            res.update({"source": "nvml", "interval_ms": self.interval * 1e3,
+                        "window": "timed region" if timed else "whole run (no sample fell "
+                                                                 "inside the timed region)",
+                        "whole_run": self._summary(rows)})
+            return res
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -113,7 +183,8 @@ class ClockSampler:
         if not mhz:
             return None
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxes),
-                "samples": len(mhz), "reasons": sorted(reasons)}
+                "samples": len(mhz), "reasons": sorted(reasons), "source": "nvidia-smi",
+                "window": "warm-up, timed region and e2e leg (100 ms samples)"}
 
 
 # ----------------------------------------------------------------------------
@@ -578,15 +649,6 @@ def main():
     for _ in range(a.warmup):
         w.step(stream)
     torch.cuda.synchronize()
-    # Clock soak: more untimed steps until the GPU has run this load for at
-    # least 1 s, so the clock record (100 ms samples from here to the end of
-    # the e2e leg) holds the steady state the timed region runs in.
-    soak_steps, soak_t0 = 0, time.perf_counter()
-    while time.perf_counter() - soak_t0 < 1.0:
-        for _ in range(10):
-            w.step(stream)
-        soak_steps += 10
-        torch.cuda.synchronize()
     if pg:
         pg.barrier()
     ev = {}
@@ -595,11 +657,13 @@ def main():
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
+    h0 = time.perf_counter()
     t0.record(stream)
     for _ in range(a.steps):
         w.step(stream, ev)
     t1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_timed(h0, time.perf_counter())
     if pg:
         pg.barrier()
     ms = t0.elapsed_time(t1) / a.steps
@@ -611,9 +675,6 @@ def main():
     if not a.skip_e2e:
         e2e_ms, h2d, d2h = e2e_run(w, stream, max(10, a.steps // 4), a.warmup)
     clk = clocks.stop()
-    if clk:
-        clk["window"] = (f"{soak_steps} untimed steps (>= 1 s) right before the timed region, "
-                         "the timed region and the e2e leg")
     if pg:
         ms, e2e_ms = max_over_ranks([ms, e2e_ms if not a.skip_e2e else 0.0], pg, dev)
     if not a.skip_e2e:

@@ -1,4 +1,4 @@
-// Paged decode on CUDA cores (any group size up to 8, and 16), the work plan
+// Paged decode on CUDA cores (any group size up to 16), the work plan
 // shared by both decode kernels, and the log-sum-exp merge of split contexts.
 //
 // Design (B200):
@@ -458,6 +458,13 @@ int launch_simt_d(const SimtParams& prm, int group, int64_t item_bound, cudaStre
     case 6: return launch_simt_impl<D, 6>(prm, item_bound, stream);
     case 7: return launch_simt_impl<D, 7>(prm, item_bound, stream);
     case 8: return launch_simt_impl<D, 8>(prm, item_bound, stream);
+    case 9: return launch_simt_impl<D, 9>(prm, item_bound, stream);
+    case 10: return launch_simt_impl<D, 10>(prm, item_bound, stream);
+    case 11: return launch_simt_impl<D, 11>(prm, item_bound, stream);
+    case 12: return launch_simt_impl<D, 12>(prm, item_bound, stream);
+    case 13: return launch_simt_impl<D, 13>(prm, item_bound, stream);
+    case 14: return launch_simt_impl<D, 14>(prm, item_bound, stream);
+    case 15: return launch_simt_impl<D, 15>(prm, item_bound, stream);
     case 16: return launch_simt_impl<D, 16>(prm, item_bound, stream);
     default: return PA_ERR_UNSUPPORTED;
   }

@@ -86,3 +86,21 @@ def test_step_stats_min_median_p90():
     st = bench.step_stats(ev, "a", "b")
     assert st == {"min": 1.0, "median": 5.5, "p90": 9.0}  # nearest rank: 9th of 10
     assert bench.step_stats({"a": [], "b": []}, "a", "b") is None
+
+
+def test_clock_record_keeps_the_timed_window_and_every_reason():
+    import bench
+    cs = bench.ClockSampler(0)
+    cs.thread = object.__new__(type("T", (), {"join": lambda self, timeout=None: None}))
+    # (host time, SM MHz, max MHz, reasons bitmask, watts): two samples before,
+    # three inside and one after the timed region
+    cs.samples = [(0.0, 1965, 1965, 0, 300.0), (1.0, 1965, 1965, 0, 310.0),
+                  (2.0, 1900, 1965, 0x4, 900.0), (2.5, 1800, 1965, 0x4 | 0x40, 950.0),
+                  (3.0, 1850, 1965, 0, 920.0), (5.0, 1500, 1965, 0x20, 400.0)]
+    cs.mark_timed(1.5, 3.2)
+    rec = cs.stop()
+    assert rec["samples"] == 3 and rec["sm_mhz"] == 1850 and rec["sm_min_mhz"] == 1800
+    assert rec["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert rec["window"] == "timed region"
+    assert rec["whole_run"]["samples"] == 6
+    assert "sw_thermal_slowdown" in rec["whole_run"]["reasons"]
