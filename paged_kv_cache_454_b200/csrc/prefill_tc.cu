@@ -14,25 +14,35 @@
 // memory its scores came from (for each 16-key group: 8 columns of P_hi, then 8
 // of P_lo) and the second product reads it from there.
 //
-// Softmax with a lazily raised maximum: each row keeps the maximum m it last
-// used; a tile whose maximum exceeds m by more than 8 (log2 units) raises m,
-// and only then is the row of O in tensor memory (and the row sum) rescaled.
-// Otherwise exp2(s - m) <= 256 is used as is; the final division by the row
-// sum accumulated with the same m makes the result exact either way.
+// Softmax: thread r of the softmax warpgroup owns row r of the tile whole
+// (every key column, every output dim), so no warp exchanges anything with
+// another.  A row is taken in four chunks of 32 keys, the next chunk's scores
+// loading from tensor memory while this one is processed.  The maximum is
+// raised lazily: each row keeps the maximum m it last used, and a chunk whose
+// scaled scores exceed m by more than 8 (log2 units) raises it -- by a whole
+// power of two, or to the chunk's maximum when the row had none -- rescaling
+// the row of O in tensor memory, the row sum and the weights already written
+// for the tile, all exactly (the factor is a power of two).  Otherwise
+// exp2(s - m) <= 256 is used as is; the final division by the row sum
+// accumulated with the same m makes the result exact either way.
 //
-// Tensor memory (512 columns): S/P of three tiles (128 each) and O (128).
-// Shared memory: q of one row tile, two K slots, three V slots (128B swizzle).
+// Tensor memory (512 columns): S/P of three key tiles (128 each) and O (128),
+// so the scores of the next two tiles are computed while the softmax works on
+// this one and the P.V of the previous one runs: the tensor core's work hides
+// behind the softmax.
+// Shared memory: q of two row tiles (the next item's loads early), two K
+// slots, three V slots (128-byte swizzle).
 //
 // Roles (one CTA per SM, persistent over (sequence, KV head, row tile) items,
 // longest causal ranges first):
-//   warp 0      producer of q and K: the row tile of q with one 3-D tensor copy
-//               (tokens x heads x 64 dims, twice), then each key tile's 8 pages.
-//   warp 10     producer of V: each key tile's 8 pages.
-//   warp 1      allocates tensor memory; one lane issues S of tile t, then the
-//               P.V of tile t-1.
-//   warps 2-9   softmax, two warpgroups: thread (r, half) owns row r and key
-//               columns (and output dims) 64*half .. +63; row maxima and sums
-//               are exchanged with the partner warp through shared memory.
+//   warp 0      producer of q and K: each item's row tile of q (one 3-D tensor
+//               copy per 64-dim half: tokens x heads x dims), then each key
+//               tile's 8 pages.
+//   warp 1      allocates tensor memory; one lane issues S of the next key
+//               tile and P.V of an earlier one, each as soon as its inputs are
+//               ready.
+//   warp 2      producer of V: each key tile's 8 pages.
+//   warps 4-7   softmax (thread = row).
 // Keys past a row's causal limit get p = 0; key rows past the context or in
 // pages with a bad block id are zeroed in V before the second product.  Every
 // wait is bounded; no unbounded barrier is used inside the role loops.
@@ -49,24 +59,25 @@ using namespace tc;
 constexpr int kD = 128;
 constexpr int kRegion = 128 * 128;            // 128 rows x 128 bytes
 constexpr int kTileBytes = 2 * kRegion;       // one 128 x 128 bf16 operand tile
-constexpr int kQSlots = 1, kKSlots = 2, kVSlots = 3, kSP = 3;
+constexpr int kQSlots = 2, kKSlots = 2, kVSlots = 3, kSP = 3;
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQSlots * kTileBytes;
 constexpr int kOffV = kOffK + kKSlots * kTileBytes;
 constexpr int kOffBar = kOffV + kVSlots * kTileBytes;
 // q_full/empty, k_full/empty, v_full/empty (per slot); s_full, p_full, pv_done
-// (per S/P buffer); o_free; drain; row-quadrant exchange (x4)
-constexpr int kNumBars = 2 * (kQSlots + kKSlots + kVSlots) + 3 * kSP + 1 + 1 + 4;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem slot, abort flag, kmask[8]
-constexpr int kOffX = kOffMisc + 64;                // exchange buffer [2][2][128] floats
-constexpr int kSmemUsed = kOffX + 2 * 2 * 128 * 4;
+// (per S/P buffer); o_free; drain
+constexpr int kNumBars = 2 * (kQSlots + kKSlots + kVSlots) + 3 * kSP + 1 + 1;
+constexpr int kMaskRing = 16;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem slot, abort flag, kmask ring
+constexpr int kSmemUsed = kOffMisc + 16 + 4 * kMaskRing;
 constexpr int kSmemBytes = kSmemUsed + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-constexpr int kThreads = 352;   // q/K producer, MMA, 8 softmax warps, V producer
+constexpr int kThreads = 256;   // q/K producer, MMA, V producer, (idle), 4 softmax warps
 constexpr int kTmemCols = 512;  // S/P x3 (128 each), O (128)
 constexpr int kOcol = kSP * 128;
 constexpr uint32_t kPageHalf = 16 * 128;  // one 64-dim half of one page: 2 KiB
-constexpr float kRescaleLog2 = 8.f;       // raise the row maximum only past 2^8
+constexpr float kRescaleLog2 = 32.f;      // raise the row maximum only past 2^32
+constexpr float kRaiseSum = 4294967296.f;  // 2^32: weights summing to less need no raise
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);
@@ -98,49 +109,20 @@ struct PfItem {
   int s, g, q0, i0, ntok, c, ctx, kv_end, ntiles;
 };
 
-// Virtual item v -> (row tile, sequence, KV head); later row tiles (longer
-// causal ranges) first.
-__device__ __forceinline__ PfItem pf_item(const PfParams& p, int v, bool flag_errors) {
-  PfItem it;
-  it.g = v % p.hkv;
-  const int rest = v / p.hkv;
-  it.s = rest % p.num_seqs;
-  const int mt = p.mt_max - 1 - rest / p.num_seqs;
-  it.q0 = p.cu_q[it.s];
-  const int n = p.cu_q[it.s + 1] - it.q0;
-  it.i0 = mt * p.tpt;
-  it.valid = it.i0 < n;
-  if (!it.valid) return it;
-  it.ntok = min(p.tpt, n - it.i0);
-  int L = p.context_lens[it.s];
-  const int cap = p.max_blocks * 16;
-  if (L < n || L > cap) {
-    if (flag_errors) raise_error(p.err, PA_DEV_ERR_CONTEXT);
-    L = L > cap ? cap : L;
-    if (L < n) {  // a chunk longer than its context: nothing consistent to compute
-      it.valid = false;
-      return it;
-    }
-  }
-  it.ctx = L;
-  it.c = L - n;
-  it.kv_end = min(L, it.c + it.i0 + it.ntok);
-  it.ntiles = (it.kv_end + 127) / 128;
-  return it;
-}
-
-// The same in two steps for a thread that must not stall on the loads: the
-// three loads of item v are issued early (volatile, so they stay where they
-// are written) and the item is decoded when it is needed.
-struct PfRaw {
-  int v, q0, q1, L;
-};
-
 __device__ __forceinline__ int ld_early(const int32_t* ptr) {
   int x;
   asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(x) : "l"(ptr));
   return x;
 }
+
+// Virtual item v -> (row tile, sequence, KV head).  Row tiles are counted from
+// the end of each sequence's chunk (k = 0: its last row tile, the longest
+// causal range), and lower k come first, so the work list runs longest first.
+// The three loads are issued early (pf_fetch) and decoded later (pf_decode), so
+// a thread that must not stall can overlap them with other work.
+struct PfRaw {
+  int v, q0, q1, L;
+};
 
 __device__ __forceinline__ PfRaw pf_fetch(const PfParams& p, int v) {
   PfRaw r;
@@ -152,32 +134,40 @@ __device__ __forceinline__ PfRaw pf_fetch(const PfParams& p, int v) {
   return r;
 }
 
-__device__ __forceinline__ PfItem pf_decode(const PfParams& p, const PfRaw& r) {
+__device__ __forceinline__ PfItem pf_decode(const PfParams& p, const PfRaw& r, bool flag_errors) {
   PfItem it;
   it.g = r.v % p.hkv;
   const int rest = r.v / p.hkv;
   it.s = rest % p.num_seqs;
-  const int mt = p.mt_max - 1 - rest / p.num_seqs;
+  const int k = rest / p.num_seqs;
   it.q0 = r.q0;
   const int n = r.q1 - r.q0;
-  it.i0 = mt * p.tpt;
-  it.valid = it.i0 < n;
+  const int mt = (n + p.tpt - 1) / p.tpt;  // row tiles of this chunk
+  const int ti = mt - 1 - k;
+  it.valid = n > 0 && ti >= 0;
+  it.ntiles = 0;
   if (!it.valid) return it;
-  it.ntok = min(p.tpt, n - it.i0);
   int L = r.L;
   const int cap = p.max_blocks * 16;
   if (L < n || L > cap) {
+    if (flag_errors) raise_error(p.err, PA_DEV_ERR_CONTEXT);
     L = L > cap ? cap : L;
-    if (L < n) {
+    if (L < n) {  // a chunk longer than its context: nothing consistent to compute
       it.valid = false;
       return it;
     }
   }
+  it.i0 = ti * p.tpt;
+  it.ntok = min(p.tpt, n - it.i0);
   it.ctx = L;
   it.c = L - n;
   it.kv_end = min(L, it.c + it.i0 + it.ntok);
   it.ntiles = (it.kv_end + 127) / 128;
   return it;
+}
+
+__device__ __forceinline__ PfItem pf_item(const PfParams& p, int v, bool flag_errors) {
+  return pf_decode(p, pf_fetch(p, v), flag_errors);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -217,13 +207,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   uint64_t* pv_done = p_full + kSP;       // P.V of tile t complete
   uint64_t* o_free = pv_done + kSP;       // O of an item read out
   uint64_t* drain = o_free + 1;
-  uint64_t* xq = drain + 1;               // [4]: the two softmax warps sharing a row quadrant
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sptr + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + kOffMisc + 4);
-  // loaded pages of key tile t, in slot t % 8 (written by the K producer; the
-  // slot is rewritten only after the scores of tile t + 6 are done)
+  // loaded pages of key tile t, in slot t % kMaskRing (written by the K
+  // producer before the tile's copies; the softmax reads it after the tile's
+  // scores, long before the producer can come round to the slot again)
   uint32_t* kmask = reinterpret_cast<uint32_t*>(sptr + kOffMisc + 16);
-  float* xbuf = reinterpret_cast<float*>(sptr + kOffX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -241,12 +230,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     }
     for (int i = 0; i < kSP; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 256);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
       mbar_init(&pv_done[i], 1);
     }
-    mbar_init(o_free, 256);
+    mbar_init(o_free, 4);
     mbar_init(drain, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&xq[i], 2);
     *abort_flag = 0;
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
@@ -282,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         mbar_wait(&k_empty[ks], ((t / kKSlots) & 1) ^ 1, abort_flag, p.err);
         if (*abort_flag) continue;
         if (lane == 0) {
-          kmask[t & 7] = vm;
+          kmask[t % kMaskRing] = vm;
           mbar_arrive_expect_tx(&k_full[ks], __popc(vm) * 2 * kPageHalf);
         }
         __syncwarp();
@@ -300,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       for (uint32_t u = it > kQSlots ? it - kQSlots : 0; u < it; ++u)
         mbar_wait(&q_full[u % kQSlots], (u / kQSlots) & 1, nullptr, p.err);
     }
-  } else if (warp == 10) {
+  } else if (warp == 2) {
     // =========================== V producer ===========================
     uint32_t t = 0;
     for (int v = blockIdx.x; v < p.total; v += gridDim.x) {
@@ -329,9 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     // ============================= MMA ==============================
     // One lane issues S of the next key tile and P.V of an earlier one, each as
     // soon as its inputs are ready (non-blocking polls, one shared limit on time
-    // without progress).  Operand descriptors are computed once; an issue is
-    // then a constant add.  The next item's indices are loaded while the
-    // current one runs.
+    // without progress).  S of tile t may run ahead of the softmax by up to two
+    // tiles (three S/P buffers).  Operand descriptors are computed once; an
+    // issue is then a constant add.  The next item's indices are loaded while
+    // the current one runs.
     if (lane == 0) {
       const uint64_t dq0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(sbase + kOffK, 16, 1024);
@@ -371,14 +360,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (!have && !s_end) {
           // the next valid item: the prefetched one, else load in place
           while (nxt_ok) {
-            I = pf_decode(p, nxt);
+            I = pf_decode(p, nxt, false);
             const int vn = nxt.v + gridDim.x;
             nxt_ok = vn < p.total;
-            if (I.valid) {
-              if (nxt_ok) nxt = pf_fetch(p, vn);
-              break;
-            }
             if (nxt_ok) nxt = pf_fetch(p, vn);
+            if (I.valid) break;
           }
           if (I.valid) {
             have = true;
@@ -429,22 +415,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       mbar_wait(drain, 0, nullptr, p.err);
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 4) {
     // ============================ softmax ============================
     const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;        // row of the tile, TMEM lane
-    const int half = (warp - 2) >> 2;    // key columns / output dims 64*half .. +63
-    const int cofs = half * 64;
+    const int r = q4 * 32 + lane;  // row of the tile, TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t ocol = tmem + lane_addr + kOcol + cofs;
-    uint32_t t = 0, xk = 0;
-    // the two warps that share this row quadrant have both passed this point
-    auto exchange = [&]() {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&xq[q4]);
-      mbar_wait(&xq[q4], xk & 1, abort_flag, p.err);
-      ++xk;
-    };
+    const uint32_t ocol = tmem + lane_addr + kOcol;
+    const float sc = p.scale_log2;
+    const float2 sc2 = make_float2(sc, sc);
+    const float2 neg1 = make_float2(-1.f, -1.f);
+    uint32_t t = 0;
     for (int v = blockIdx.x; v < p.total; v += gridDim.x) {
       const PfItem I = pf_item(p, v, false);
       if (!I.valid) continue;
@@ -455,165 +435,195 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       for (int j = 0; j < I.ntiles; ++j, ++t) {
         const int sb = t % kSP;
         const int kv0 = j * 128;
+        const uint32_t scol = tmem + lane_addr + sb * 128;
         mbar_wait(&s_full[sb], (t / kSP) & 1, abort_flag, p.err);
         tc_fence_after();
-        const uint32_t vm = kmask[t & 7];
-        float sv[64];
-        tmem_ld64(tmem + lane_addr + sb * 128 + cofs, sv);
-        // visibility of this half row's 64 keys as two 32-bit masks: keys below
-        // the row's causal limit, in pages that were loaded
-        uint32_t vis[2];
+        const uint32_t vm = kmask[t % kMaskRing];
+        // Visibility of the row's keys: below the row's causal limit, in pages
+        // that were loaded.  A row outside the tile's tokens sees everything:
+        // its weights are never read out, and treating it as fully visible
+        // keeps its warp on the unmasked path.
+        const int nvis = min(max(limit - kv0, 0), 128);  // leading visible keys
+        const bool all_vis = __all_sync(0xffffffffu, !row_ok || (nvis == 128 && vm == 0xffu));
+        // the whole row of scores in registers (one wait), scaled
+        float xv[128];
         {
-          const int nvis = min(max(limit - kv0 - cofs, 0), 64);  // leading visible keys
-          const uint32_t pages = (vm >> (cofs >> 4)) & 0xfu;     // this half's 4 pages
+          uint32_t sr[128];
+          tmem_ld128u(scol, sr);
+          const float negm = m == -CUDART_INF_F ? 0.f : -m;
+          const float2 nm2 = make_float2(negm, negm);
 #pragma unroll
-          for (int w = 0; w < 2; ++w) {
+          for (int k = 0; k < 128; k += 2) {
+            const float2 xx = __ffma2_rn(
+                make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), sc2, nm2);
+            xv[k] = xx.x;
+            xv[k + 1] = xx.y;
+          }
+        }
+        if (!all_vis) {
+          // keys that are not visible become -inf (p = 0), whatever their score
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
             const int nw = min(max(nvis - 32 * w, 0), 32);
             const uint32_t lead = nw >= 32 ? 0xffffffffu : ((1u << nw) - 1u);
-            const uint32_t pg = (((pages >> (2 * w)) & 1u) ? 0x0000ffffu : 0u) |
-                                (((pages >> (2 * w + 1)) & 1u) ? 0xffff0000u : 0u);
-            vis[w] = lead & pg;
+            const uint32_t pg = (((vm >> (2 * w)) & 1u) ? 0x0000ffffu : 0u) |
+                                (((vm >> (2 * w + 1)) & 1u) ? 0xffff0000u : 0u);
+            const uint32_t vw = row_ok ? (lead & pg) : 0xffffffffu;
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              xv[32 * w + k] = ((vw >> k) & 1u) ? xv[32 * w + k] : -CUDART_INF_F;
           }
         }
-        // Row maximum of the scaled scores.  Scaling is folded into the
-        // exponent's FMA below, so the maximum is taken on the raw scores (the
-        // largest for a positive scale, the smallest for a negative one).  A
-        // warp whose rows see all 64 keys skips the per-key visibility test.
-        const bool all_vis = __all_sync(0xffffffffu, (vis[0] & vis[1]) == 0xffffffffu);
-        const float sc = p.scale_log2;
-        float mx;
-        if (sc >= 0.f) {
-          float mx4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-          if (all_vis) {
-#pragma unroll
-            for (int k = 0; k < 64; ++k) mx4[k & 3] = fmaxf(mx4[k & 3], sv[k]);
-          } else {
-#pragma unroll
-            for (int k = 0; k < 64; ++k) {
-              const bool on = (vis[k >> 5] >> (k & 31)) & 1u;
-              mx4[k & 3] = fmaxf(mx4[k & 3], on ? sv[k] : -CUDART_INF_F);
-            }
-          }
-          mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        } else {  // a negative scale turns the smallest raw score into the largest
-          float mn4[4] = {CUDART_INF_F, CUDART_INF_F, CUDART_INF_F, CUDART_INF_F};
-#pragma unroll
-          for (int k = 0; k < 64; ++k) {
-            const bool on = (vis[k >> 5] >> (k & 31)) & 1u;
-            mn4[k & 3] = fminf(mn4[k & 3], on ? sv[k] : CUDART_INF_F);
-          }
-          mx = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
-          mx = mx == CUDART_INF_F ? -CUDART_INF_F : mx;
-        }
-        mx = mx == -CUDART_INF_F ? mx : mx * sc;  // scaled maximum
-        float* px = xbuf + (xk & 1) * 256;
-        px[half * 128 + r] = mx;
-        exchange();
-        mx = fmaxf(mx, px[(half ^ 1) * 128 + r]);
-        // raise the row maximum only when it grows past 2^8; then rescale O and l
-        const bool raise = mx > m + kRescaleLog2;
-        if (j > 0 && __any_sync(0xffffffffu, raise)) {
-          const float f = raise ? exp2f(m - mx) : 1.f;
-          mbar_wait(&pv_done[(t - 1) % kSP], ((t - 1) / kSP) & 1, abort_flag, p.err);
-          tc_fence_after();
+        // Weights of the whole row with the maximum in use, written back over
+        // the scores as P_hi / P_lo (P_hi is p with its mantissa cut to bf16,
+        // P_lo the same cut of the remainder: p = P_hi + P_lo to within 2^-15
+        // of p), formed with integer masks and byte permutes, leaving the
+        // multi-function unit to ex2; returns the row's sum of the weights.
+        auto weights = [&]() -> float {
+          float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            float ov[16];
-            tmem_ld16(ocol + c * 16, ov);
-            uint32_t ow[16];
+            uint32_t pw[32];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) ow[k] = __float_as_uint(ov[k] * f);
-            tmem_st16_nowait(ocol + c * 16, ow);
-          }
-          tmem_wait_st();
-          l *= f;
-        }
-        if (raise) m = mx;
-        // Exponentials written back over the scores as P_hi / P_lo.  P_hi is
-        // p with its mantissa cut to bf16, P_lo the same cut of the remainder
-        // (p = P_hi + P_lo to within 2^-15 of p); both are formed with integer
-        // masks and byte permutes, leaving the multi-function unit to ex2.
-        const float negm = m == -CUDART_INF_F ? 0.f : -m;
-        // pairs of keys go through the packed fp32x2 FMA/add instructions
-        const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(negm, negm);
-        const float2 neg1 = make_float2(-1.f, -1.f);
-        float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pw[16];
-#pragma unroll
-          for (int k = 0; k < 16; k += 2) {
-            const int kk = c * 16 + k;
-            const float2 x = __ffma2_rn(make_float2(sv[kk], sv[kk + 1]), sc2, nm2);
-            float p0 = exp2f(x.x);
-            float p1 = exp2f(x.y);
-            if (!all_vis) {
-              p0 = ((vis[kk >> 5] >> (kk & 31)) & 1u) ? p0 : 0.f;
-              p1 = ((vis[kk >> 5] >> ((kk + 1) & 31)) & 1u) ? p1 : 0.f;
+            for (int k = 0; k < 32; k += 2) {
+              const int kk = 32 * c + k;
+              const float p0 = exp2f(xv[kk]);
+              const float p1 = exp2f(xv[kk + 1]);
+              const float2 pp = make_float2(p0, p1);
+              rs2[(k >> 1) & 1] = __fadd2_rn(rs2[(k >> 1) & 1], pp);
+              const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+              const float2 hi = make_float2(__uint_as_float(b0 & 0xffff0000u),
+                                            __uint_as_float(b1 & 0xffff0000u));
+              const float2 lo = __ffma2_rn(hi, neg1, pp);  // p - P_hi, exact
+              const int g = k >> 4, kg = k & 15;  // 16-key group within the chunk
+              pw[16 * g + (kg >> 1)] = __byte_perm(b0, b1, 0x7632);
+              pw[16 * g + 8 + (kg >> 1)] =
+                  __byte_perm(__float_as_uint(lo.x), __float_as_uint(lo.y), 0x7632);
             }
-            const float2 pp = make_float2(p0, p1);
-            rs2[(k >> 1) & 1] = __fadd2_rn(rs2[(k >> 1) & 1], pp);
-            const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-            const float2 hi =
-                make_float2(__uint_as_float(b0 & 0xffff0000u), __uint_as_float(b1 & 0xffff0000u));
-            const float2 lo = __ffma2_rn(hi, neg1, pp);  // p - P_hi, exact
-            pw[k >> 1] = __byte_perm(b0, b1, 0x7632);
-            pw[8 + (k >> 1)] = __byte_perm(__float_as_uint(lo.x), __float_as_uint(lo.y), 0x7632);
+            tmem_st32_nowait(scol + 32 * c, pw);
           }
-          tmem_st16_nowait(tmem + lane_addr + sb * 128 + cofs + c * 16, pw);
+          return (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
+        };
+        // Raise the maximum in use to the tile's maximum xm (scaled, relative
+        // to the old one); then the row of O (earlier key tiles of this item)
+        // and l are rescaled.  The P.V of the previous tile may still be
+        // running, so that waits for it first.
+        auto raise_to = [&](bool raise, float xm) {
+          float f = 1.f;
+          if (raise) {
+            f = m == -CUDART_INF_F ? 0.f : exp2f(-xm);
+            m = m == -CUDART_INF_F ? xm : m + xm;
+            const float2 d2 = make_float2(-xm, -xm);
+#pragma unroll
+            for (int k = 0; k < 128; k += 2) {
+              const float2 xx = __fadd2_rn(make_float2(xv[k], xv[k + 1]), d2);
+              xv[k] = xx.x;
+              xv[k + 1] = xx.y;
+            }
+          }
+          l *= f;
+          if (j > 0) {
+            mbar_wait(&pv_done[(t - 1) % kSP], ((t - 1) / kSP) & 1, abort_flag, p.err);
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+              float ov[16];
+              tmem_ld16(ocol + cc * 16, ov);
+              uint32_t ow[16];
+#pragma unroll
+              for (int k = 0; k < 16; ++k) ow[k] = __float_as_uint(ov[k] * f);
+              tmem_st16(ocol + cc * 16, ow);
+            }
+          }
+        };
+        auto row_max = [&]() -> float {
+          float m8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = xv[k];
+#pragma unroll
+          for (int k = 8; k < 128; ++k) m8[k & 7] = fmaxf(m8[k & 7], xv[k]);
+          return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        };
+        // A row without a maximum yet (its first visible keys) takes the
+        // tile's maximum first.  Every other row goes straight to the weights:
+        // a sum of at most 2^32 means no weight exceeds 2^32, so the maximum
+        // in use stands (no maximum is computed in the common case); a larger
+        // (or non-finite) sum raises it to the tile's maximum and the weights
+        // are computed again.
+        if (__any_sync(0xffffffffu, m == -CUDART_INF_F)) {
+          const float xm = row_max();
+          const bool raise = m == -CUDART_INF_F ? xm != -CUDART_INF_F : xm > kRescaleLog2;
+          if (__any_sync(0xffffffffu, raise)) raise_to(raise, xm);
         }
-        const float rs = (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
+        float rs = weights();
+        {
+          const bool check = row_ok && !(rs <= kRaiseSum);
+          if (__any_sync(0xffffffffu, check)) {
+            tmem_wait_st();
+            const float xm = row_max();
+            const bool raise = check && xm > kRescaleLog2;
+            if (__any_sync(0xffffffffu, raise)) {
+              raise_to(raise, xm);
+              rs = weights();
+            }
+          }
+        }
         tmem_wait_st();
         l += rs;
-        // key rows past the context or in an unloaded page: zero this half of them in V
+        // key rows past the context or in an unloaded page: zero them in V
         if (kv0 + 128 > I.ctx || vm != 0xffu) {
           const int key = kv0 + r;
           if (key >= I.ctx || !((vm >> (r >> 4)) & 1u)) {
             const int vs = t % kVSlots;
             mbar_wait(&v_full[vs], (t / kVSlots) & 1, abort_flag, p.err);
-            const uint32_t vrow = sbase + kOffV + vs * kTileBytes + half * kRegion + r * 128;
+            const uint32_t vrow = sbase + kOffV + vs * kTileBytes + r * 128;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) sts128_zero(vrow + k * 16);
+            for (int k = 0; k < 8; ++k) {
+              sts128_zero(vrow + k * 16);
+              sts128_zero(vrow + kRegion + k * 16);
+            }
             fence_proxy_async_smem();
           }
         }
+        // every lane's stores are done (waited and fenced) before its warp's arrival
         tc_fence_before();
-        mbar_arrive(&p_full[sb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sb]);
       }
-      // end of the item: O is final once the last P.V is done
-      float ov[64];
+      // end of the item: O is final once the last P.V is done; it is read out
+      // 32 dims at a time
       if (I.ntiles > 0) {
         mbar_wait(&pv_done[(t - 1) % kSP], ((t - 1) / kSP) & 1, abort_flag, p.err);
         tc_fence_after();
-        tmem_ld64(ocol, ov);
-      } else {
-#pragma unroll
-        for (int k = 0; k < 64; ++k) ov[k] = 0.f;
       }
-      tc_fence_before();
-      mbar_arrive(o_free);
-      // row sum over both halves
-      float* px = xbuf + (xk & 1) * 256;
-      px[half * 128 + r] = l;
-      exchange();
-      l += px[(half ^ 1) * 128 + r];
-      if (row_ok) {
-        const int h = r - ti * p.group;
-        const int64_t orow = static_cast<int64_t>(I.q0 + I.i0 + ti) * p.hq + I.g * p.group + h;
-        const bool live = l > 0.f;
-        const float inv = live ? 1.f / l : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kD + cofs);
+      const int h = r - ti * p.group;
+      const int64_t orow = static_cast<int64_t>(I.q0 + I.i0 + ti) * p.hq + I.g * p.group + h;
+      const bool live = l > 0.f;
+      const float inv = live ? 1.f / l : 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kD);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint4 w;
-          w.x = pack_bf16x2(ov[8 * q] * inv, ov[8 * q + 1] * inv);
-          w.y = pack_bf16x2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv);
-          w.z = pack_bf16x2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv);
-          w.w = pack_bf16x2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv);
-          dst[q] = w;
+      for (int c = 0; c < 4; ++c) {
+        float ov[32];
+        tmem_ld32(ocol + 32 * c, ov);
+        if (c == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
         }
-        if (half == 0 && p.lse) p.lse[orow] = live ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+        if (row_ok) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = pack_bf16x2(ov[8 * q] * inv, ov[8 * q + 1] * inv);
+            w.y = pack_bf16x2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv);
+            w.z = pack_bf16x2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv);
+            w.w = pack_bf16x2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv);
+            dst[4 * c + q] = w;
+          }
+        }
       }
+      if (row_ok && p.lse) p.lse[orow] = live ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
     }
   }
 
