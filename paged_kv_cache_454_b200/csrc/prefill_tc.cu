@@ -30,11 +30,13 @@
 // so the scores of the next two tiles are computed while the softmax works on
 // this one and the P.V of the previous one runs: the tensor core's work hides
 // behind the softmax.
-// Shared memory: q of two row tiles (the next item's loads early), two K
-// slots, three V slots (128-byte swizzle).
+// Shared memory: q of one row tile, two K slots, three V slots (128-byte
+// swizzle).  K is laid out half by half (each 64-dim half of the 128 key rows
+// evenly spaced, as the first product needs), moved as two 2 KiB copies per
+// page; V page by page, one 4 KiB copy per page (the second product takes a
+// page per 16-key step).
 //
-// Roles (one CTA per SM, persistent over (sequence, KV head, row tile) items,
-// longest causal ranges first):
+// Roles (one CTA per SM, persistent over (sequence, KV head, row tile) items):
 //   warp 0      producer of q and K: each item's row tile of q (one 3-D tensor
 //               copy per 64-dim half: tokens x heads x dims), then each key
 //               tile's 8 pages.
@@ -59,22 +61,23 @@ using namespace tc;
 constexpr int kD = 128;
 constexpr int kRegion = 128 * 128;            // 128 rows x 128 bytes
 constexpr int kTileBytes = 2 * kRegion;       // one 128 x 128 bf16 operand tile
-constexpr int kQSlots = 2, kKSlots = 2, kVSlots = 3, kSP = 3;
+constexpr int kQSlots = 1, kKSlots = 2, kVSlots = 3, kSP = 2;
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQSlots * kTileBytes;
 constexpr int kOffV = kOffK + kKSlots * kTileBytes;
 constexpr int kOffBar = kOffV + kVSlots * kTileBytes;
 // q_full/empty, k_full/empty, v_full/empty (per slot); s_full, p_full, pv_done
-// (per S/P buffer); o_free; drain
-constexpr int kNumBars = 2 * (kQSlots + kKSlots + kVSlots) + 3 * kSP + 1 + 1;
+// (per S/P buffer); o_free; drain; the halves' exchange at the end of an item
+constexpr int kNumBars = 2 * (kQSlots + kKSlots + kVSlots) + 3 * kSP + 1 + 1 + 1;
 constexpr int kMaskRing = 16;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem slot, abort flag, kmask ring
-constexpr int kSmemUsed = kOffMisc + 16 + 4 * kMaskRing;
+constexpr int kOffX = kOffMisc + 16 + 4 * kMaskRing;  // [2 items][2 halves][128 rows] (m, l)
+constexpr int kSmemUsed = kOffX + 2 * 2 * 128 * 8;
 constexpr int kSmemBytes = kSmemUsed + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-constexpr int kThreads = 256;   // q/K producer, MMA, V producer, (idle), 4 softmax warps
-constexpr int kTmemCols = 512;  // S/P x3 (128 each), O (128)
-constexpr int kOcol = kSP * 128;
+constexpr int kThreads = 384;   // q/K producer, MMA, V producer, (idle), 2 softmax warpgroups
+constexpr int kTmemCols = 512;  // S/P x2 (128 each), O of each key half (128 each)
+constexpr int kOcol = kSP * 128;  // O_0 at kOcol, O_1 at kOcol + 128
 constexpr uint32_t kPageHalf = 16 * 128;  // one 64-dim half of one page: 2 KiB
 constexpr float kRescaleLog2 = 32.f;      // raise the row maximum only past 2^32
 constexpr float kRaiseSum = 4294967296.f;  // 2^32: weights summing to less need no raise
@@ -115,11 +118,15 @@ __device__ __forceinline__ int ld_early(const int32_t* ptr) {
   return x;
 }
 
-// Virtual item v -> (row tile, sequence, KV head).  Row tiles are counted from
-// the end of each sequence's chunk (k = 0: its last row tile, the longest
-// causal range), and lower k come first, so the work list runs longest first.
-// The three loads are issued early (pf_fetch) and decoded later (pf_decode), so
-// a thread that must not stall can overlap them with other work.
+// Virtual item v -> (sequence, KV head, row tile), row tile fastest: the row
+// tiles of one (sequence, KV head) are consecutive items, so the persistent
+// CTAs work on them at the same time and stream the same K/V pages -- read
+// from HBM once, from L2 for the rest (in another order each row tile's pass
+// over the pages comes long after the previous one, and a batch's pages
+// outgrow L2).  Row tiles are counted from the end of the sequence's chunk
+// (k = 0: its last row tile, the longest causal range).  The three loads are
+// issued early (pf_fetch) and decoded later (pf_decode), so a thread that must
+// not stall can overlap them with other work.
 struct PfRaw {
   int v, q0, q1, L;
 };
@@ -127,7 +134,7 @@ struct PfRaw {
 __device__ __forceinline__ PfRaw pf_fetch(const PfParams& p, int v) {
   PfRaw r;
   r.v = v;
-  const int s = (v / p.hkv) % p.num_seqs;
+  const int s = v / (p.mt_max * p.hkv);
   r.q0 = ld_early(p.cu_q + s);
   r.q1 = ld_early(p.cu_q + s + 1);
   r.L = ld_early(p.context_lens + s);
@@ -136,10 +143,10 @@ __device__ __forceinline__ PfRaw pf_fetch(const PfParams& p, int v) {
 
 __device__ __forceinline__ PfItem pf_decode(const PfParams& p, const PfRaw& r, bool flag_errors) {
   PfItem it;
-  it.g = r.v % p.hkv;
-  const int rest = r.v / p.hkv;
-  it.s = rest % p.num_seqs;
-  const int k = rest / p.num_seqs;
+  const int k = r.v % p.mt_max;
+  const int q = r.v / p.mt_max;
+  it.g = q % p.hkv;
+  it.s = q / p.hkv;
   it.q0 = r.q0;
   const int n = r.q1 - r.q0;
   const int mt = (n + p.tpt - 1) / p.tpt;  // row tiles of this chunk
@@ -207,12 +214,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   uint64_t* pv_done = p_full + kSP;       // P.V of tile t complete
   uint64_t* o_free = pv_done + kSP;       // O of an item read out
   uint64_t* drain = o_free + 1;
+  uint64_t* xchg = drain + 1;             // both key halves' (m, l) of an item written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sptr + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + kOffMisc + 4);
   // loaded pages of key tile t, in slot t % kMaskRing (written by the K
   // producer before the tile's copies; the softmax reads it after the tile's
   // scores, long before the producer can come round to the slot again)
   uint32_t* kmask = reinterpret_cast<uint32_t*>(sptr + kOffMisc + 16);
+  float2* xbuf = reinterpret_cast<float2*>(sptr + kOffX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -230,11 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     }
     for (int i = 0; i < kSP; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
+      mbar_init(&p_full[i], 8);  // one arrival per softmax warp
       mbar_init(&pv_done[i], 1);
     }
-    mbar_init(o_free, 4);
+    mbar_init(o_free, 8);
     mbar_init(drain, 1);
+    mbar_init(xchg, 8);
     *abort_flag = 0;
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
@@ -304,9 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         __syncwarp();
         if (pb >= 0) {
           const int row = (pb * p.hkv + I.g) * 16;
-          const uint32_t vd = sbase + kOffV + vs * kTileBytes + lane * kPageHalf;
-          tma_load_2d(vd, &p.tm_v, 0, row, &v_full[vs]);
-          tma_load_2d(vd + kRegion, &p.tm_v, 64, row, &v_full[vs]);
+          // one 3-D copy of the page: both 64-dim halves, next to each other
+          const uint32_t vd = sbase + kOffV + vs * kTileBytes + lane * (2 * kPageHalf);
+          tma_load_3d(vd, &p.tm_v, 0, row, 0, &v_full[vs]);
         }
       }
     }
@@ -317,14 +327,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     // ============================= MMA ==============================
     // One lane issues S of the next key tile and P.V of an earlier one, each as
     // soon as its inputs are ready (non-blocking polls, one shared limit on time
-    // without progress).  S of tile t may run ahead of the softmax by up to two
-    // tiles (three S/P buffers).  Operand descriptors are computed once; an
+    // without progress).  S of tile t may run ahead of the softmax by a tile
+    // (two S/P buffers).  Operand descriptors are computed once; an
     // issue is then a constant add.  The next item's indices are loaded while
     // the current one runs.
     if (lane == 0) {
       const uint64_t dq0 = smem_desc_sw128(sbase + kOffQ, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(sbase + kOffK, 16, 1024);
-      const uint64_t dv0 = smem_desc_sw128(sbase + kOffV, kRegion, 1024);
+      // V page by page: [page][64-dim half][16 rows][128 B]; the second
+      // product's 16-key step is one page, its two halves 2 KiB apart
+      const uint64_t dv0 = smem_desc_sw128(sbase + kOffV, 2 * 1024, 1024);
       uint32_t ts = 0, tpv = 0, it = 0, items_pv = 0;
       uint32_t first_bits = 0;  // bit t % 8: tile t is the first of its item
       PfItem I{};
@@ -345,11 +357,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tc_fence_after();
             const uint64_t vb = desc_add(dv0, vs * kTileBytes);
             const uint32_t sp = tmem + sb * 128;
+            // keys 0-63 of the tile into O_0, keys 64-127 into O_1
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              const uint64_t bd = desc_add(vb, k * 2048);
-              umma_ts(tmem + kOcol, sp + 16 * k, bd, kIdescO, (first && k == 0) ? 0u : 1u);
-              umma_ts(tmem + kOcol, sp + 16 * k + 8, bd, kIdescO, 1u);
+              const uint64_t bd = desc_add(vb, k * 4096);
+              const uint32_t oc = tmem + kOcol + (k >> 2) * 128;
+              umma_ts(oc, sp + 16 * k, bd, kIdescO, (first && (k & 3) == 0) ? 0u : 1u);
+              umma_ts(oc, sp + 16 * k + 8, bd, kIdescO, 1u);
             }
             umma_commit(&pv_done[sb]);
             umma_commit(&v_empty[vs]);
@@ -377,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         if (have) {
           const int sb = ts % kSP, ks = ts % kKSlots, qs = it % kQSlots;
-          // S/P buffer sb is free once the P.V of tile ts - 3 is done
+          // S/P buffer sb is free once the P.V of tile ts - 2 is done
           if ((j > 0 || mbar_test_wait(&q_full[qs], (it / kQSlots) & 1)) &&
               mbar_test_wait(&k_full[ks], (ts / kKSlots) & 1) &&
               mbar_test_wait(&pv_done[sb], ((ts / kSP) & 1) ^ 1)) {
@@ -417,14 +431,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     __syncwarp();
   } else if (warp >= 4) {
     // ============================ softmax ============================
+    // Warpgroup h (0: warps 4-7, 1: warps 8-11) owns key columns 64h .. 64h+63
+    // of every tile; thread r of it owns row r of those.  Each half keeps its
+    // own maximum, row sum and accumulator O_h, so the halves never wait for
+    // each other inside an item; at its end they merge by log-sum-exp.
+    const int hf = (warp - 4) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;  // row of the tile, TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t ocol = tmem + lane_addr + kOcol;
+    const uint32_t ocol = tmem + lane_addr + kOcol + hf * 128;  // this half's O_h row
     const float sc = p.scale_log2;
     const float2 sc2 = make_float2(sc, sc);
     const float2 neg1 = make_float2(-1.f, -1.f);
-    uint32_t t = 0;
+    uint32_t t = 0, nit = 0;
     for (int v = blockIdx.x; v < p.total; v += gridDim.x) {
       const PfItem I = pf_item(p, v, false);
       if (!I.valid) continue;
@@ -434,36 +453,43 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       float m = -CUDART_INF_F, l = 0.f;
       for (int j = 0; j < I.ntiles; ++j, ++t) {
         const int sb = t % kSP;
-        const int kv0 = j * 128;
-        const uint32_t scol = tmem + lane_addr + sb * 128;
+        const int kv0 = j * 128 + 64 * hf;  // first key of this half
+        const uint32_t scol = tmem + lane_addr + sb * 128 + 64 * hf;
         mbar_wait(&s_full[sb], (t / kSP) & 1, abort_flag, p.err);
         tc_fence_after();
-        const uint32_t vm = kmask[t % kMaskRing];
-        // Visibility of the row's keys: below the row's causal limit, in pages
-        // that were loaded.  A row outside the tile's tokens sees everything:
-        // its weights are never read out, and treating it as fully visible
-        // keeps its warp on the unmasked path.
-        const int nvis = min(max(limit - kv0, 0), 128);  // leading visible keys
-        const bool all_vis = __all_sync(0xffffffffu, !row_ok || (nvis == 128 && vm == 0xffu));
-        // the whole row of scores in registers (one wait), scaled
-        float xv[128];
+        const uint32_t vm = (kmask[t % kMaskRing] >> (4 * hf)) & 0xfu;  // this half's pages
+        // Visibility of the half row's keys: below the row's causal limit, in
+        // pages that were loaded.  A row outside the tile's tokens sees
+        // everything: its weights are never read out, and treating it as fully
+        // visible keeps its warp on the unmasked path.
+        const int nvis = min(max(limit - kv0, 0), 64);  // leading visible keys
+        const bool all_vis = __all_sync(0xffffffffu, !row_ok || (nvis == 64 && vm == 0xfu));
+        // the half row of scores in registers (one wait), scaled
+        float xv[64];
         {
-          uint32_t sr[128];
-          tmem_ld128u(scol, sr);
+          uint32_t sa[32], sb2[32];
+          tmem_ld32_nowait(scol, sa);
+          tmem_ld32_nowait(scol + 32, sb2);
+          tmem_wait_ld_regs(sa);
+          tmem_wait_ld_regs(sb2);
           const float negm = m == -CUDART_INF_F ? 0.f : -m;
           const float2 nm2 = make_float2(negm, negm);
 #pragma unroll
-          for (int k = 0; k < 128; k += 2) {
-            const float2 xx = __ffma2_rn(
-                make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), sc2, nm2);
-            xv[k] = xx.x;
-            xv[k + 1] = xx.y;
+          for (int k = 0; k < 32; k += 2) {
+            const float2 xa = __ffma2_rn(
+                make_float2(__uint_as_float(sa[k]), __uint_as_float(sa[k + 1])), sc2, nm2);
+            const float2 xb = __ffma2_rn(
+                make_float2(__uint_as_float(sb2[k]), __uint_as_float(sb2[k + 1])), sc2, nm2);
+            xv[k] = xa.x;
+            xv[k + 1] = xa.y;
+            xv[32 + k] = xb.x;
+            xv[32 + k + 1] = xb.y;
           }
         }
         if (!all_vis) {
           // keys that are not visible become -inf (p = 0), whatever their score
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
+          for (int w = 0; w < 2; ++w) {
             const int nw = min(max(nvis - 32 * w, 0), 32);
             const uint32_t lead = nw >= 32 ? 0xffffffffu : ((1u << nw) - 1u);
             const uint32_t pg = (((vm >> (2 * w)) & 1u) ? 0x0000ffffu : 0u) |
@@ -474,15 +500,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
               xv[32 * w + k] = ((vw >> k) & 1u) ? xv[32 * w + k] : -CUDART_INF_F;
           }
         }
-        // Weights of the whole row with the maximum in use, written back over
+        // Weights of the half row with the maximum in use, written back over
         // the scores as P_hi / P_lo (P_hi is p with its mantissa cut to bf16,
         // P_lo the same cut of the remainder: p = P_hi + P_lo to within 2^-15
         // of p), formed with integer masks and byte permutes, leaving the
-        // multi-function unit to ex2; returns the row's sum of the weights.
+        // multi-function unit to ex2; returns the sum of the weights.
         auto weights = [&]() -> float {
           float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 2; ++c) {
             uint32_t pw[32];
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
@@ -505,9 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           return (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
         };
         // Raise the maximum in use to the tile's maximum xm (scaled, relative
-        // to the old one); then the row of O (earlier key tiles of this item)
-        // and l are rescaled.  The P.V of the previous tile may still be
-        // running, so that waits for it first.
+        // to the old one); then this half's row of O_h (earlier key tiles of
+        // this item) and l are rescaled.  The P.V of the previous tile may
+        // still be running, so that waits for it first.
         auto raise_to = [&](bool raise, float xm) {
           float f = 1.f;
           if (raise) {
@@ -515,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             m = m == -CUDART_INF_F ? xm : m + xm;
             const float2 d2 = make_float2(-xm, -xm);
 #pragma unroll
-            for (int k = 0; k < 128; k += 2) {
+            for (int k = 0; k < 64; k += 2) {
               const float2 xx = __fadd2_rn(make_float2(xv[k], xv[k + 1]), d2);
               xv[k] = xx.x;
               xv[k + 1] = xx.y;
@@ -541,12 +567,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
           for (int k = 0; k < 8; ++k) m8[k] = xv[k];
 #pragma unroll
-          for (int k = 8; k < 128; ++k) m8[k & 7] = fmaxf(m8[k & 7], xv[k]);
+          for (int k = 8; k < 64; ++k) m8[k & 7] = fmaxf(m8[k & 7], xv[k]);
           return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                        fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         };
-        // A row without a maximum yet (its first visible keys) takes the
-        // tile's maximum first.  Every other row goes straight to the weights:
+        // A half row without a maximum yet (its first visible keys) takes the
+        // tile's maximum first.  Every other one goes straight to the weights:
         // a sum of at most 2^32 means no weight exceeds 2^32, so the maximum
         // in use stands (no maximum is computed in the common case); a larger
         // (or non-finite) sum raises it to the tile's maximum and the weights
@@ -571,17 +597,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         tmem_wait_st();
         l += rs;
-        // key rows past the context or in an unloaded page: zero them in V
-        if (kv0 + 128 > I.ctx || vm != 0xffu) {
+        // key rows of this half past the context or in an unloaded page: zero
+        // them in V (threads 0-63 of the warpgroup, one key row each)
+        if (j * 128 + 128 > I.ctx || vm != 0xfu) {
           const int key = kv0 + r;
-          if (key >= I.ctx || !((vm >> (r >> 4)) & 1u)) {
+          if (r < 64 && (key >= I.ctx || !((vm >> (r >> 4)) & 1u))) {
             const int vs = t % kVSlots;
             mbar_wait(&v_full[vs], (t / kVSlots) & 1, abort_flag, p.err);
-            const uint32_t vrow = sbase + kOffV + vs * kTileBytes + r * 128;
+            const int kr = 64 * hf + r;  // key row of the tile: page kr / 16, row kr % 16
+            const uint32_t vrow =
+                sbase + kOffV + vs * kTileBytes + (kr >> 4) * 4096 + (kr & 15) * 128;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               sts128_zero(vrow + k * 16);
-              sts128_zero(vrow + kRegion + k * 16);
+              sts128_zero(vrow + 2048 + k * 16);
             }
             fence_proxy_async_smem();
           }
@@ -591,22 +620,40 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[sb]);
       }
-      // end of the item: O is final once the last P.V is done; it is read out
-      // 32 dims at a time
+      // End of the item: the halves' (m, l) meet in shared memory; O = s_0 O_0 +
+      // s_1 O_1 with s_h = 2^(m_h - M) / L, M = max(m_0, m_1) and
+      // L = l_0 2^(m_0 - M) + l_1 2^(m_1 - M).  Half h writes output dims
+      // 64h .. 64h+63 from both accumulators, once the last P.V is done.
+      float2* xb = xbuf + (nit & 1) * 256;
+      xb[hf * 128 + r] = make_float2(m, l);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xchg);
+      mbar_wait(xchg, nit & 1, abort_flag, p.err);
+      const float2 other = xb[(hf ^ 1) * 128 + r];
+      ++nit;
+      const float m0 = hf == 0 ? m : other.x, l0 = hf == 0 ? l : other.y;
+      const float m1 = hf == 0 ? other.x : m, l1 = hf == 0 ? other.y : l;
+      const float M = fmaxf(m0, m1);
+      const float e0 = M == -CUDART_INF_F ? 0.f : exp2f(m0 - M);
+      const float e1 = M == -CUDART_INF_F ? 0.f : exp2f(m1 - M);
+      const float L = l0 * e0 + l1 * e1;
+      const bool live = L > 0.f;
+      const float inv = live ? 1.f / L : 0.f;
+      const float s0 = e0 * inv, s1 = e1 * inv;
       if (I.ntiles > 0) {
         mbar_wait(&pv_done[(t - 1) % kSP], ((t - 1) / kSP) & 1, abort_flag, p.err);
         tc_fence_after();
       }
       const int h = r - ti * p.group;
       const int64_t orow = static_cast<int64_t>(I.q0 + I.i0 + ti) * p.hq + I.g * p.group + h;
-      const bool live = l > 0.f;
-      const float inv = live ? 1.f / l : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kD);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kD + 64 * hf);
+      const uint32_t o0 = tmem + lane_addr + kOcol + 64 * hf;  // dims 64h.. of O_0
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float ov[32];
-        tmem_ld32(ocol + 32 * c, ov);
-        if (c == 3) {
+      for (int c = 0; c < 2; ++c) {
+        float a0[32], a1[32];
+        tmem_ld32(o0 + 32 * c, a0);
+        tmem_ld32(o0 + 128 + 32 * c, a1);
+        if (c == 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(o_free);
@@ -614,16 +661,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (row_ok) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
+            float o[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o[k] = a0[8 * q + k] * s0 + a1[8 * q + k] * s1;
             uint4 w;
-            w.x = pack_bf16x2(ov[8 * q] * inv, ov[8 * q + 1] * inv);
-            w.y = pack_bf16x2(ov[8 * q + 2] * inv, ov[8 * q + 3] * inv);
-            w.z = pack_bf16x2(ov[8 * q + 4] * inv, ov[8 * q + 5] * inv);
-            w.w = pack_bf16x2(ov[8 * q + 6] * inv, ov[8 * q + 7] * inv);
+            w.x = pack_bf16x2(o[0], o[1]);
+            w.y = pack_bf16x2(o[2], o[3]);
+            w.z = pack_bf16x2(o[4], o[5]);
+            w.w = pack_bf16x2(o[6], o[7]);
             dst[4 * c + q] = w;
           }
         }
       }
-      if (row_ok && p.lse) p.lse[orow] = live ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+      if (hf == 0 && row_ok && p.lse) p.lse[orow] = live ? (M + log2f(L)) * kLn2 : -CUDART_INF_F;
     }
   }
 
@@ -654,7 +704,14 @@ int launch_prefill_tcgen05(const PrefillArgs& a) {
     const uint64_t strides[1] = {kD * 2};
     const uint32_t box[2] = {64, 16};
     if (!encode_bf16_map(&p.tm_k, a.k_pool, 2, dims, strides, box)) return PA_ERR_CUDA;
-    if (!encode_bf16_map(&p.tm_v, a.v_pool, 2, dims, strides, box)) return PA_ERR_CUDA;
+  }
+  {
+    // V: (dim within a 64-dim half, pool row, half) -- one copy moves a page's
+    // 16 rows for both halves, half 0 first
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), 2};
+    const uint64_t strides[2] = {kD * 2, 128};
+    const uint32_t box[3] = {64, 16, 2};
+    if (!encode_bf16_map(&p.tm_v, a.v_pool, 3, dims, strides, box)) return PA_ERR_CUDA;
   }
   p.tpt = 128 / group;
   {
