@@ -44,6 +44,51 @@ __device__ __forceinline__ float float_of(uint32_t k) {
   return __uint_as_float(b);
 }
 
+// Calls f(value, index) for every element of row x[0, V), each thread keeping
+// four loads in flight: 16-byte vectors when the row is 16-byte aligned (64 KiB
+// in flight per CTA, what one SM needs to stream at its share of HBM), single
+// floats otherwise.  Elements reach f in no particular order.
+template <typename F>
+__device__ __forceinline__ void for_each_logit(const float* __restrict__ x, int V, F f) {
+  const int tid = threadIdx.x;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const int V4 = V >> 2;
+    int i = tid;
+    for (; i + 3 * kThreads < V4; i += 4 * kThreads) {
+      float4 a[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) a[q] = __ldg(x4 + i + q * kThreads);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int b = 4 * (i + q * kThreads);
+        f(a[q].x, b);
+        f(a[q].y, b + 1);
+        f(a[q].z, b + 2);
+        f(a[q].w, b + 3);
+      }
+    }
+    for (; i < V4; i += kThreads) {
+      const float4 a = __ldg(x4 + i);
+      f(a.x, 4 * i);
+      f(a.y, 4 * i + 1);
+      f(a.z, 4 * i + 2);
+      f(a.w, 4 * i + 3);
+    }
+    for (int j = 4 * V4 + tid; j < V; j += kThreads) f(x[j], j);
+    return;
+  }
+  int i = tid;
+  for (; i + 3 * kThreads < V; i += 4 * kThreads) {
+    float a[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) a[q] = x[i + q * kThreads];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) f(a[q], i + q * kThreads);
+  }
+  for (; i < V; i += kThreads) f(x[i], i);
+}
+
 // Mass of logit x in 32.32 fixed point: exp2((x - xmax) * scale) * 2^32.
 __device__ __forceinline__ uint64_t mass_of(float x, float xmax, float scale) {
   if (x != x) return 0ull;
@@ -175,16 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
       bi = i;
     }
   };
-  int i0 = tid;
-  // four independent loads in flight per thread, then the compares in index order
-  for (; i0 + 3 * kThreads < V; i0 += 4 * kThreads) {
-    float a[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) a[q] = x[i0 + q * kThreads];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) take(a[q], i0 + q * kThreads);
-  }
-  for (; i0 < V; i0 += kThreads) take(x[i0], i0);
+  for_each_logit(x, V, take);
   sm.tmax[tid] = bk;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -249,15 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
           sm.cand[pos] = (static_cast<uint64_t>(k) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
       }
     };
-    int i1 = tid;
-    for (; i1 + 3 * kThreads < V; i1 += 4 * kThreads) {
-      float a[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) a[q] = x[i1 + q * kThreads];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) collect(a[q], i1 + q * kThreads);
-    }
-    for (; i1 < V; i1 += kThreads) collect(x[i1], i1);
+    for_each_logit(x, V, collect);
     __syncthreads();
     const int n = sm.count;
     if (n <= kCand) {
