@@ -32,6 +32,7 @@ from workloads import synth  # noqa: E402
 
 METRIC = "paged decode tokens/s & KV-read GB/s (% of B200 HBM peak) per batch step"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024  # B200 L2
 
 
 # ----------------------------------------------------------------------------
@@ -269,7 +270,9 @@ class Workload:
     def launches_per_step(self):
         """Library kernel launches in one step: block copies (480 pairs per
         launch), the cache write, the decode plan and decode kernel (plus the
-        merge kernel on the CUDA-core path), the prefill kernel."""
+        shared-prefix launch on the tensor-core path for groups up to 8 and
+        2..1024 sequences, which returns at once when no prefix is shared, or
+        the merge kernel on the CUDA-core path), the prefill kernel."""
         lay = self.layout
         n = 1  # cache write
         if lay.copy_pairs.size:
@@ -278,6 +281,8 @@ class Workload:
             tensor_core = self.kernel == 2 or (
                 self.kernel == 0 and lay.head_dim == 128 and lay.group_size <= 16)
             n += 2 if tensor_core else 3
+            if tensor_core and lay.group_size <= 8 and 2 <= len(self.dec) <= 1024:
+                n += 1
         if len(self.pf):
             n += 1
         return n
@@ -318,31 +323,36 @@ def host_manager_timing(w: Workload, steps: int = 100):
 def sampler_timing(w: Workload, stream, reps: int = 50):
     """Device time of the fused sampler (``pa_sample``) for this batch's decode
     rows at two vocabulary sizes (32000, 152064), temperature 0.7, top-k 50,
-    top-p 0.9; CUDA events over ``reps`` back-to-back calls after warm-up."""
+    top-p 0.9; CUDA events over ``reps`` back-to-back calls after warm-up.
+    Consecutive calls read different logit buffers whose total is over twice
+    the L2, so every call streams its logits from HBM."""
     torch = w.torch
     rows = len(w.dec) if len(w.dec) else 1
     res = {}
     g = torch.Generator(device=w.dev)
     g.manual_seed(0)
     for vocab in (32000, 152064):
-        x = torch.randn(rows, vocab, device=w.dev, generator=g) * 3
+        nbuf = -(-2 * L2_BYTES // (rows * vocab * 4)) + 1
+        xs = [torch.randn(rows, vocab, device=w.dev, generator=g) * 3 for _ in range(nbuf)]
         T = torch.full((rows,), 0.7, device=w.dev)
         K = torch.full((rows,), 50, dtype=torch.int32, device=w.dev)
         P = torch.full((rows,), 0.9, device=w.dev)
         u = torch.rand(rows, device=w.dev, generator=g)
         out = torch.empty(rows, dtype=torch.int32, device=w.dev)
         with torch.cuda.stream(stream):
-            for _ in range(5):
-                w.pa.pa_sample(x, T, K, P, u, out=out, stream=stream)
+            for i in range(max(5, nbuf)):
+                w.pa.pa_sample(xs[i % nbuf], T, K, P, u, out=out, stream=stream)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for _ in range(reps):
-                w.pa.pa_sample(x, T, K, P, u, out=out, stream=stream)
+            for i in range(reps):
+                w.pa.pa_sample(xs[i % nbuf], T, K, P, u, out=out, stream=stream)
             e1.record(stream)
         torch.cuda.synchronize()
         res[str(vocab)] = round(e0.elapsed_time(e1) / reps * 1e3, 2)
+        del xs
     return {"us_per_call": res, "rows": rows, "temperature": 0.7, "top_k": 50, "top_p": 0.9,
+            "l2": "rotating logit buffers, over twice the L2 in total",
             "logits_gb_per_s": {k: round(rows * int(k) * 4 / (v * 1e-6) / 1e9, 1)
                                 for k, v in res.items()}}
 

@@ -77,29 +77,43 @@ int check_pool(const pa_pool_desc& pool) {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Runs of at least two sequences: at most num_seqs / 2 of them.
+static size_t max_runs(int S) { return size_t(S) / 2 + 1; }
+
 size_t decode_workspace_bytes(int S, int Hq, int Hkv, int D, int max_parts) {
-  const size_t slots = size_t(S) * size_t(max_parts);
-  size_t b = align256(4 * sizeof(int));
+  const size_t slots = size_t(S) * (size_t(max_parts) + 1);
+  size_t b = align256(8 * sizeof(int));
   b += align256(sizeof(int) * (size_t(S) + 1));
   b += align256(sizeof(int) * size_t(S) * size_t(Hkv));
   b += align256(sizeof(int2) * slots * size_t(Hkv));
+  b += 2 * align256(sizeof(int) * size_t(S));
+  b += align256(sizeof(int) * max_runs(S) * kRunInts);
+  b += align256(sizeof(int2) * max_runs(S) * size_t(Hkv) * size_t(max_parts));
   b += align256(sizeof(float) * slots * size_t(Hq) * size_t(D));
   b += align256(sizeof(float) * slots * size_t(Hq));
   return b;
 }
 
 DecodeWorkspace carve_decode_workspace(void* ws, int S, int Hq, int Hkv, int D, int max_parts) {
-  const size_t slots = size_t(S) * size_t(max_parts);
+  const size_t slots = size_t(S) * (size_t(max_parts) + 1);
   char* p = static_cast<char*>(ws);
   DecodeWorkspace w;
   w.header = reinterpret_cast<int*>(p);
-  p += align256(4 * sizeof(int));
+  p += align256(8 * sizeof(int));
   w.part_base = reinterpret_cast<int*>(p);
   p += align256(sizeof(int) * (size_t(S) + 1));
   w.merge_cnt = reinterpret_cast<int*>(p);
   p += align256(sizeof(int) * size_t(S) * size_t(Hkv));
   w.items = reinterpret_cast<int2*>(p);
   p += align256(sizeof(int2) * slots * size_t(Hkv));
+  w.seq_span = reinterpret_cast<int*>(p);
+  p += align256(sizeof(int) * size_t(S));
+  w.seq_pp = reinterpret_cast<int*>(p);
+  p += align256(sizeof(int) * size_t(S));
+  w.runs = reinterpret_cast<int*>(p);
+  p += align256(sizeof(int) * max_runs(S) * kRunInts);
+  w.pitems = reinterpret_cast<int2*>(p);
+  p += align256(sizeof(int2) * max_runs(S) * size_t(Hkv) * size_t(max_parts));
   w.part_o = reinterpret_cast<float*>(p);
   p += align256(sizeof(float) * slots * size_t(Hq) * size_t(D));
   w.part_lse = reinterpret_cast<float*>(p);
@@ -239,6 +253,12 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
   a.stream = as_stream(stream);
   if (!a.err) return PA_ERR_CUDA;
   a.item_heads = item_heads;
+  // shared prefixes read once for all their sharers (tensor-core kernel, and
+  // batches the plan can sort): items of 8 q columns for groups up to 4, of 16
+  // for groups up to 8 (room for two sharers at least)
+  a.casc_cols = 0;
+  if (kind == PA_KERNEL_TCGEN05 && num_seqs >= 2 && num_seqs <= kCascMaxSeqs)
+    a.casc_cols = group <= 4 ? 8 : (group <= 8 ? 16 : 0);
 
   st = launch_decode_plan(a);
   if (st != PA_OK) return st;

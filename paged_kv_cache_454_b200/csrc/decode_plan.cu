@@ -20,7 +20,23 @@
 //    the rest.  (Up to kSortMax sequences.)  A hash set of first blocks finds
 //    whether any repeats; the sort runs only then, and only if some candidate
 //    length keeps every item at most 1/kLocalityShare of one SM's share.
-//  * It also clears the dynamic item counter and the per-(sequence, KV head)
+//  * Shared-prefix cascade (tensor-core kernel, when the caller enables it
+//    with `casc_cols`, the q columns of one shared-prefix item, 8 or 16):
+//    sequences sorted by first block form runs.  The longest run fixes the
+//    sharers per item M (at most casc_cols / G) and the KV heads per item HT
+//    (the most, up to 8, with G * HT * M <= casc_cols that divide the KV
+//    heads); runs are
+//    cut into sub-runs of at most M sequences, and a sub-run's shared span is
+//    the longest stretch of leading table entries all its members have in
+//    common (whole blocks inside every member's context).  A span of at least
+//    kMinCascSpan tokens becomes shared-prefix items (sub-run, KV-head group,
+//    partition) in a list of their own, read once for all members, with a
+//    partition length of their own (several items per SM: the sequences' own
+//    items start only when these are done); each member's own items then cover
+//    only its tokens after the span, and its partitions count the span's
+//    first.  header[4..7]: prefix items, their counter, log2 HT | M << 8,
+//    their partition length.
+//  * It also clears the dynamic item counters and the per-(sequence, KV head)
 //    counters the tensor-core kernel uses to find the last partition to finish.
 #include "common.cuh"
 #include "internal.h"
@@ -52,6 +68,10 @@ constexpr int kFirstSet = 2 * kSortMax;  // slots of the set that detects shared
 // 256-token items at this bound; longer items leave a long tail).
 constexpr int kLocalityShare = 16;
 static_assert(kFirstSet == 2048, "the set's hash keeps 11 bits");
+// A shared prefix shorter than this is left to each sequence's own items.
+constexpr int kMinCascSpan = 128;
+// Shared-prefix items per SM the prefix partition length aims for.
+constexpr int kCascItemsPerSm = 8;
 
 // Inclusive block-wide scan (sum or max) of one value per thread, 1024 threads.
 template <bool kMax>
@@ -82,11 +102,13 @@ __device__ __forceinline__ int block_scan(int x, int* warp_tot) {
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ context_lens,
                                                            const int32_t* __restrict__ block_tables,
                                                            int S, int max_blocks, int hkv,
-                                                           int min_part, int max_part,
+                                                           int kv_heads, int min_part, int max_part,
                                                            int target_items, int num_sms,
+                                                           int group, int casc_cols,
                                                            int* header, int* part_base,
                                                            int2* items, int* merge_cnt,
-                                                           unsigned int* err) {
+                                                           int* seq_span, int* seq_pp, int* runs,
+                                                           int2* pitems, unsigned int* err) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
   __shared__ int cand[4];      // items per KV-head group at each candidate length
@@ -99,6 +121,11 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   __shared__ int sflag[4];                        // [0] some first block repeats
   __shared__ int slens[kLensCache];               // context lengths as given (S <= kLensCache)
   __shared__ unsigned first_set[kFirstSet];       // open-addressing set of first blocks
+  __shared__ int sspan[kSortMax];                 // shared-prefix span per sequence (cascade)
+  __shared__ int nruns;                           // sub-runs (cascade)
+  __shared__ int rspan[kSortMax / 2];             // each sub-run's shared span (cascade)
+  __shared__ int rmax;                            // longest run of shared first blocks
+  __shared__ int cand_pp[4];                      // prefix items at each candidate length
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   // The decode kernel that follows may start its prologue now; it waits for
@@ -184,7 +211,8 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   __syncthreads();
   int part = -1;
   bool locality = false;
-  if (sortable && sflag[0]) {
+  bool casc = casc_cols >= 2 * group && sortable && sflag[0] != 0;
+  if (sortable && sflag[0] && !casc) {
     const long long share = static_cast<long long>(tiles_tot) * hkv;
     for (int k = ncand - 1; k >= 0; --k)
       if (static_cast<long long>(cand_mx[k]) * kLocalityShare * num_sms <= share) {
@@ -206,6 +234,147 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   const int unit = part / 64 > 16 ? part / 64 : 16;
   const int full_bucket = bucket_of(part / unit);
 
+  // ---- sort sequences by their first physical block ----
+  // Keys (first block << 32 | sequence) are distinct, so each sequence's
+  // sorted position is the number of keys below its own: one pass over the S
+  // keys per thread (shared-memory broadcasts) and two barriers.
+  if (locality || casc) {
+    unsigned long long* keys = reinterpret_cast<unsigned long long*>(run_tab);  // unsorted
+    unsigned long long k = 0;
+    if (tid < S) {
+      const int L = clamp_len(lens[tid], max_blocks, nullptr);
+      const unsigned first = L > 0 ? my_first : 0xffffffffu;
+      k = (static_cast<unsigned long long>(first) << 32) | static_cast<unsigned>(tid);
+      keys[tid] = k;
+    }
+    __syncthreads();
+    if (tid < S) {
+      int r = 0, j = 0;
+      for (; j + 8 <= S; j += 8) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) r += keys[j + q] < k;
+      }
+      for (; j < S; ++j) r += keys[j] < k;
+      skey[r] = k;
+    }
+    __syncthreads();
+  }
+  // ---- shared-prefix cascade: runs of sequences with a common first block,
+  // cut into sub-runs, and the span each sub-run's tables have in common ----
+  if (tid < kSortMax) sspan[tid] = 0;
+  if (tid < 4) cand_pp[tid] = 0;
+  if (tid == 0) {
+    nruns = 0;
+    rmax = 0;
+  }
+  __syncthreads();
+  int members = 0, hts = 0, pp_len = part;
+  if (casc) {
+    // thread i: sorted position i.  A run's length is stored at its start.
+    int* run_len = run_tab;           // by a run's first sorted position
+    int* sub_pos = run_tab + kSortMax;  // per sub-run: first sorted position | members << 16
+    const int i = tid;
+    unsigned long long f = 0xffffffffull;
+    bool head = false, last = false;
+    if (i < S) {
+      f = skey[i] >> 32;
+      head = i == 0 || f != (skey[i - 1] >> 32);
+      last = i == S - 1 || f != (skey[i + 1] >> 32);
+    }
+    const int start = block_scan<true>(head ? i : 0, warp_tot);
+    if (i < S && last && f != 0xffffffffull) {
+      run_len[start] = i - start + 1;
+      atomicMax(&rmax, i - start + 1);
+    }
+    __syncthreads();
+    // sharers per item and KV heads per item
+    members = min(rmax, casc_cols / group);
+    hts = 0;
+    while (hts < 3 && group * (2 << hts) * members <= casc_cols && kv_heads % (2 << hts) == 0) ++hts;
+    casc = members >= 2;
+    if (casc) {
+      // sub-runs: every members-th sequence of a run starts one, if at least
+      // one more follows it
+      bool sub = false;
+      int k = 0;
+      if (i < S && f != 0xffffffffull) {
+        const int w = i - start, n = run_len[start];
+        sub = w % members == 0 && n - w >= 2;
+        k = min(members, n - w);
+      }
+      const int idx = block_scan<false>(sub ? 1 : 0, warp_tot);
+      if (sub) sub_pos[idx - 1] = i | (k << 16);
+      if (tid == 1023) nruns = idx;
+      __syncthreads();
+      // a warp per sub-run: its members and the span of table entries they share
+      const int nr = nruns;
+      for (int r = warp; r < nr; r += 32) {
+        const int i0 = sub_pos[r] & 0xffff, k = sub_pos[r] >> 16;
+        int full = max_blocks;  // whole blocks inside every member's context
+        for (int q = 0; q < k; ++q) {
+          const int sq = static_cast<int>(skey[i0 + q] & 0xffffffffull);
+          full = min(full, clamp_len(lens[sq], max_blocks, nullptr) >> 4);
+        }
+        int lcp = full;
+        for (int b0 = 0; b0 < full; b0 += 32) {
+          const int bj = b0 + lane;
+          bool same = true;
+          if (bj < full) {
+            // every member's entry is loaded before any is compared, so the
+            // loads are in flight together
+            int32_t v[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              v[q] = q < k ? block_tables[static_cast<int64_t>(skey[i0 + q] & 0xffffffffull) * max_blocks + bj]
+                           : 0;
+#pragma unroll
+            for (int q = 1; q < 16; ++q) same = same && (q >= k || v[q] == v[0]);
+          }
+          const unsigned diff = __ballot_sync(0xffffffffu, !same);
+          if (diff) {
+            lcp = b0 + __ffs(diff) - 1;
+            break;
+          }
+        }
+        const int span = lcp * 16 >= kMinCascSpan ? lcp * 16 : 0;
+        int* rr = runs + static_cast<int64_t>(r) * kRunInts;
+        if (lane == 0) {
+          rr[0] = span;
+          rr[1] = k;
+          rspan[r] = span;
+        }
+        if (lane < k) {
+          const int sq = static_cast<int>(skey[i0 + lane] & 0xffffffffull);
+          rr[2 + lane] = sq;
+          sspan[sq] = span;
+        }
+      }
+      __syncthreads();
+      // prefix partition length: the longest candidate that still gives
+      // kCascItemsPerSm items per SM (the shortest when none does)
+      {
+        const int cg = kv_heads >> hts;
+        int cnt[4] = {0, 0, 0, 0};
+        for (int r = tid; r < nr; r += 1024) {
+          const int span = rspan[r];
+          for (int k = 0; k < ncand; ++k) cnt[k] += cg * ((span + (min_part << k) - 1) / (min_part << k));
+        }
+        for (int k = 0; k < ncand; ++k) {
+          int v = cnt[k];
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0 && v) atomicAdd(&cand_pp[k], v);
+        }
+      }
+      __syncthreads();
+      pp_len = min_part;
+      for (int k = ncand - 1; k > 0; --k)
+        if (static_cast<long long>(cand_pp[k]) >= static_cast<long long>(kCascItemsPerSm) * num_sms) {
+          pp_len = min_part << k;
+          break;
+        }
+    }
+  }
+
   // ---- partitions per sequence and their exclusive prefix ----
   if (tid == 0) carry = 0;
   if (tid < kMaxBuckets) bucket[tid] = 0;
@@ -215,10 +384,17 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     int np = 0;
     if (s < S) {
       const int L = clamp_len(lens[s], max_blocks, err);
-      np = (L + part - 1) / part;
+      // a shared span (cascade) first, then the sequence's own tokens
+      const int span = casc ? sspan[s] : 0;
+      const int pp = (span + pp_len - 1) / pp_len;
+      const int Ls = L - span;
+      np = pp + (Ls + part - 1) / part;
       if (np < 1) np = 1;
-      // bucket counts: full partitions, the tail, or an empty context
-      const int full = L / part, rem = L - full * part;
+      seq_span[s] = span;
+      seq_pp[s] = pp;
+      // bucket counts of the sequence's own items: full partitions, the tail,
+      // or an empty context
+      const int full = Ls / part, rem = Ls - full * part;
       if (full) atomicAdd(&bucket[full_bucket], full * hkv);
       if (rem) atomicAdd(&bucket[bucket_of((rem + unit - 1) / unit)], hkv);
       if (L == 0) atomicAdd(&bucket[bucket_of(0)], hkv);
@@ -270,49 +446,21 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
       acc += c[j];
     }
     if (lane == 0) {
+      int own = 0;  // the sequences' own items: every bucket
+      for (int b = 0; b < kMaxBuckets; ++b) own += bucket[b];
       part_base[S] = carry;
-      header[0] = carry * hkv;  // items
+      header[0] = own;          // items (the sequences' own)
       header[1] = carry;        // partitions
       header[2] = 0;            // dynamic item counter
       header[3] = part;         // partition length
+      header[5] = 0;            // dynamic counter of the shared-prefix items
+      header[6] = hts | (members << 8);  // log2 KV heads, sharers per shared-prefix item
+      header[7] = pp_len;       // partition length of the shared prefixes
     }
   }
   __syncthreads();
 
-  // ---- sort sequences by their first physical block ----
-  if (locality) {
-    int n2 = 1;
-    while (n2 < S) n2 <<= 1;
-    for (int i = tid; i < n2; i += 1024) {
-      unsigned long long k = ~0ull;
-      if (i < S) {
-        const int L = clamp_len(lens[i], max_blocks, nullptr);
-        const unsigned first = L > 0 ? (i == tid ? my_first
-                                                : static_cast<unsigned>(
-                                                      block_tables[static_cast<int64_t>(i) * max_blocks]))
-                                     : 0xffffffffu;
-        k = (static_cast<unsigned long long>(first) << 32) | static_cast<unsigned>(i);
-      }
-      skey[i] = k;
-    }
-    __syncthreads();
-    for (int k = 2; k <= n2; k <<= 1) {
-      for (int j = k >> 1; j > 0; j >>= 1) {
-        for (int i = tid; i < n2; i += 1024) {
-          const int ixj = i ^ j;
-          if (ixj > i) {
-            const unsigned long long a = skey[i], b = skey[ixj];
-            if ((a > b) == ((i & k) == 0)) {
-              skey[i] = b;
-              skey[ixj] = a;
-            }
-          }
-        }
-        __syncthreads();
-      }
-    }
-  }
-  if (locality) {
+  if (locality && !casc) {
     // thread i handles sorted position i (S <= 1024).  A run of equal first
     // blocks is laid out KV head by KV head, the run's sequences in each head.
     const int i = tid;
@@ -346,9 +494,10 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   }
 
   // ---- the work list, longest items first ----
-  for (int s = tid; s < S && !locality; s += 1024) {
+  for (int s = tid; s < S && (!locality || casc); s += 1024) {
     const int L = clamp_len(lens[s], max_blocks, nullptr);
-    const int full = L / part, rem = L - full * part;
+    const int Ls = L - (casc ? sspan[s] : 0);
+    const int full = Ls / part, rem = Ls - full * part;
     if (full) {
       int at = atomicAdd(&cursor[full_bucket], full * hkv);
       for (int g = 0; g < hkv; ++g)
@@ -363,7 +512,22 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
       for (int g = 0; g < hkv; ++g) items[at + g] = make_int2(s, g << 16);
     }
   }
-  for (int i = tid; i < S * hkv; i += 1024) merge_cnt[i] = 0;
+  // ---- the shared-prefix items: (sub-run, KV-head group, partition) ----
+  {
+    const int nr = casc ? nruns : 0;
+    int cnt = 0;
+    const int cg = kv_heads >> hts;
+    if (tid < nr) cnt = cg * ((rspan[tid] + pp_len - 1) / pp_len);
+    const int incl = block_scan<false>(cnt, warp_tot);  // (nr <= 512 < 1024)
+    if (tid < nr) {
+      const int np = cnt / cg;
+      int at = incl - cnt;
+      for (int g = 0; g < cg; ++g)
+        for (int q = 0; q < np; ++q) pitems[at++] = make_int2(tid, (g << 16) | q);
+    }
+    if (tid == 1023) header[4] = incl;  // shared-prefix items
+  }
+  for (int i = tid; i < S * kv_heads; i += 1024) merge_cnt[i] = 0;
 }
 
 }  // namespace
@@ -371,9 +535,10 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
 int launch_decode_plan(const DecodeArgs& a) {
   decode_plan_kernel<<<1, 1024, 0, a.stream>>>(
       a.context_lens, a.block_tables, a.num_seqs, a.max_blocks,
-      a.pool.num_kv_heads / a.item_heads, a.min_part,
-      a.max_part, a.target_items, num_sms(), a.ws.header, a.ws.part_base, a.ws.items,
-      a.ws.merge_cnt, a.err);
+      a.pool.num_kv_heads / a.item_heads, a.pool.num_kv_heads, a.min_part, a.max_part,
+      a.target_items, num_sms(), a.num_q_heads / a.pool.num_kv_heads, a.casc_cols,
+      a.ws.header, a.ws.part_base, a.ws.items, a.ws.merge_cnt, a.ws.seq_span, a.ws.seq_pp,
+      a.ws.runs, a.ws.pitems, a.err);
   return launch_status();
 }
 

@@ -44,6 +44,18 @@
 //   warps 7-10  epilogue: write the output, or the partition's partial result;
 //               the last partition of a (sequence, head group) to finish merges
 //               all of them by log-sum-exp (one pass over the partitions).
+// Shared prefixes (cascade): sequences whose tables start with the same
+// blocks (parallel samples of one prompt) are grouped by the plan into
+// sub-runs of up to M sharers.  A first launch runs only the sub-runs'
+// shared-prefix items: the tile is read once and scored against the q heads of
+// every sharer.  The q columns of a tile are ordered (KV head of the item,
+// sharer, q head of the group): a row's columns -- those of its KV head -- are
+// then M * G contiguous ones, exactly as a group of M * G q heads, so the
+// same softmax serves both.  Each sharer gets its own partial result for the
+// prefix partition.  The second launch runs every
+// sequence's own items over the tokens after its shared span.  Partitions of
+// both launches are merged per (sequence, KV head) by whichever partition
+// finishes last.
 // Tokens past the context (and pages with a bad block id) get p = 0 and their
 // V rows are zeroed before the second product, so NaN padding is never read
 // into a result.  Every wait is bounded and the softmax warps exchange data
@@ -120,12 +132,20 @@ struct __align__(64) TcParams {
   CUtensorMap tm_v;   // V as rows of 64 dims (two copies per page, one per half)
   CUtensorMap tm_v3;  // V as (64 dims, row, half): one copy per page
   CUtensorMap tm_q;
+  CUtensorMap tm_kc[4];  // shared-prefix launch: K and V maps for 1, 2, 4, 8 KV heads per tile
+  CUtensorMap tm_vc[4];
+  const uint16_t* q;     // shared-prefix launch: q rows are gathered with plain loads
+  int64_t q_stride;      // elements between sequences' q rows
   const int32_t* block_tables;
   const int32_t* context_lens;
   int* header;
   const int* part_base;
   int* merge_cnt;
   const int2* items;
+  const int2* pitems;    // shared-prefix items
+  const int* runs;       // sub-runs: span, members, member sequences
+  const int* seq_span;   // per sequence: tokens of its shared span
+  const int* seq_pp;     // per sequence: partitions of that span
   float* part_o;
   float* part_lse;
   uint16_t* out;
@@ -160,10 +180,12 @@ __device__ __forceinline__ void tmem_ld_o<16>(uint32_t taddr, float (&v)[32]) {
 
 // NH: q columns per tile.  GR: q columns a tile row scores against -- NH (any
 // group; every row computes all columns, masked to its own KV head's) or 1 (one
-// q head per KV head: each row has exactly one column).
-template <int NH, int GR>
+// q head per KV head: each row has exactly one column).  kCasc: the launch of
+// the shared-prefix items (GR == NH only).
+template <int NH, int GR, bool kCasc>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ TcParams p) {
   static_assert(GR == NH || (GR == 1 && NH <= 8), "row column modes");
+  static_assert(!kCasc || GR == NH, "shared-prefix items need every row's columns");
   using L = Smem<NH>;
   constexpr int kNpv = L::kNpv;
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, kNpv, true, false);
@@ -204,9 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int hts = p.ht_shift;
-  const int ht = 1 << hts;            // KV heads per tile
-  const int pages = 8 >> hts;         // pages per tile
+  constexpr bool casc = kCasc;  // the shared-prefix launch
+  if (casc) {
+    // most batches share no prefix: leave before any set-up (the launch after
+    // this one starts as these CTAs exit)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (p.header[4] == 0) return;
+  }
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -258,11 +284,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   // programmatic dependent launch): the set-up above overlaps it, and nothing
   // below reads the plan's results before the plan grid has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // KV heads per tile: fixed by the host, or chosen by the plan for shared prefixes
+  // (shared prefixes: sharers per item M in bits 8.. of the same word)
+  const int hword = casc ? p.header[6] : p.ht_shift;
+  const int hts = hword & 0xff;
+  const int ht = 1 << hts;            // KV heads per tile
+  const int pages = 8 >> hts;         // pages per tile
+  const int msh = casc ? hword >> 8 : 1;  // sharers per item (1: a sequence's own items)
+  const int cph = msh * p.group;      // q columns per KV head of an item
 
   if (warp == 6) {
     // =========================== scheduler ===========================
-    const int total = p.header[0];
-    const int part = p.header[3];
+    const int total = casc ? p.header[4] : p.header[0];
+    const int part = casc ? p.header[7] : p.header[3];
+    int* const counter = p.header + (casc ? 5 : 2);
     uint32_t d = 0;
     auto publish = [&](const TileDesc& td, int pbk) {
       const int slot = d % kDescSlots;
@@ -285,21 +320,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     };
     while (!*abort_flag) {
       int item = 0;
-      if (lane == 0) item = atomicAdd(p.header + 2, 1);
+      if (lane == 0) item = atomicAdd(counter, 1);
       item = __shfl_sync(0xffffffffu, item, 0);
       if (item >= total) break;
-      const int2 dd = p.items[item];
+      const int2 dd = casc ? p.pitems[item] : p.items[item];
       TileDesc td;
       td.s = dd.x;
       td.g = dd.y >> 16;
-      td.part = dd.y & 0xffff;
-      int Lc = p.context_lens[td.s];
-      const int cap = p.max_blocks * 16;
-      Lc = Lc < 0 ? 0 : (Lc > cap ? cap : Lc);
-      const int tok0 = td.part * part;
-      td.tok1 = min(Lc, tok0 + part);
-      td.pbase = p.part_base[td.s];
-      td.npart = p.part_base[td.s + 1] - td.pbase;
+      const int q = dd.y & 0xffff;
+      int tok0, srow;
+      if (casc) {
+        // a sub-run (s = its index; npart = its members) over its shared span,
+        // read through its first member's table
+        const int* rr = p.runs + static_cast<int64_t>(td.s) * kRunInts;
+        const int span = rr[0];
+        td.npart = rr[1];
+        srow = rr[2];
+        td.part = q;
+        td.pbase = 0;
+        tok0 = q * part;
+        td.tok1 = min(span, tok0 + part);
+      } else {
+        // a sequence's own tokens, after its shared span (if any)
+        int Lc = p.context_lens[td.s];
+        const int cap = p.max_blocks * 16;
+        Lc = Lc < 0 ? 0 : (Lc > cap ? cap : Lc);
+        srow = td.s;
+        td.part = p.seq_pp[td.s] + q;
+        tok0 = p.seq_span[td.s] + q * part;
+        td.tok1 = min(Lc, tok0 + part);
+        td.pbase = p.part_base[td.s];
+        td.npart = p.part_base[td.s + 1] - td.pbase;
+      }
       const int npages = td.tok1 > tok0 ? (td.tok1 - tok0 + 15) / 16 : 0;
       if (npages == 0) {
         td.tok0 = tok0;
@@ -307,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         publish(td, -1);
         continue;
       }
-      const int32_t* row = p.block_tables + static_cast<int64_t>(td.s) * p.max_blocks + (tok0 >> 4);
+      const int32_t* row = p.block_tables + static_cast<int64_t>(srow) * p.max_blocks + (tok0 >> 4);
       for (int p0 = 0; p0 < npages; p0 += 32) {
         // lane l reads page p0 + l of the item
         int pb = -1;
@@ -326,6 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
       }
     }
+    // the launch after this one may start as this CTA's last items drain
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // end of the stream (after a timeout: in every slot, without waiting)
     if (!*abort_flag) {
       TileDesc td{};
@@ -339,6 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     uint32_t d = 0, t = 0, nq = 0;
     const uint64_t pol = l2_policy_evict_first();
     const uint32_t page_bytes = 4u * 2048u * static_cast<uint32_t>(ht);  // K and V, both halves
+    const CUtensorMap* tmk = casc ? &p.tm_kc[hts] : &p.tm_k;
+    const CUtensorMap* tmv = casc ? &p.tm_vc[hts] : &p.tm_v3;
     while (true) {
       const int slot = d % kDescSlots;
       mbar_wait(&desc_full[slot], (d / kDescSlots) & 1, abort_flag, p.err);
@@ -352,8 +408,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           // q of the item's KV-head group into the next q slot
           const int qs = nq & 1;
           mbar_wait(&q_empty[qs], ((nq >> 1) & 1) ^ 1, abort_flag, p.err);
-          if (!*abort_flag && lane == 0) {
-            const uint32_t q0 = sbase + L::kOffQ + qs * kQBytes;
+          const uint32_t q0 = sbase + L::kOffQ + qs * kQBytes;
+          if (casc) {
+            // the sharers' q heads of the item's KV heads, column by column
+            // (row h of the slot: KV head hh = h / cph of the item, sharer
+            // m = h % cph / G, q head j = h % G of the group; rows of absent
+            // sharers and past HT * cph zero), with plain loads in the
+            // swizzled layout
+            if (!*abort_flag) {
+              const int nsh = td->npart;
+              const int my_s = lane < nsh ? p.runs[static_cast<int64_t>(s) * kRunInts + 2 + lane] : 0;
+#pragma unroll
+              for (int j = 0; j < 16 * NH / 32; ++j) {
+                const int i = j * 32 + lane;
+                const int h = i >> 4, c = i & 15;  // q column, 16-byte chunk of the 256-byte row
+                const int hh = h / cph, w = h - hh * cph, m = w / p.group;
+                const int sm = __shfl_sync(0xffffffffu, my_s, m & 31);
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (hh < ht && m < nsh)
+                  v = __ldg(reinterpret_cast<const uint4*>(
+                      p.q + static_cast<int64_t>(sm) * p.q_stride +
+                      static_cast<int64_t>((g * ht + hh) * p.group + w - m * p.group) * kD + c * 8));
+                sts128(q0 + (c >> 3) * kQRegion + swz(h, c & 7), v);
+              }
+              // rows NH..15 of the q region (a 16-row operand) stay as they are:
+              // no product column reads them
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&q_full[qs]);
+            }
+          } else if (!*abort_flag && lane == 0) {
             mbar_arrive_expect_tx(&q_full[qs], kQBytes);
             tma_load_3d(q0, &p.tm_q, 0, g * p.nq, s, &q_full[qs]);
             tma_load_3d(q0 + kQRegion, &p.tm_q, 64, g * p.nq, s, &q_full[qs]);
@@ -371,10 +455,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             const int prow = (pb * p.hkv + (g << hts)) * 16;
             const uint32_t kdst = stage + lane * (ht * 2048);
             const uint32_t vdst = stage + kKBytes + lane * (ht * 4096);
-            tma_load_2d_hint(kdst, &p.tm_k, 0, prow, &full[st], pol);
-            tma_load_2d_hint(kdst + kRegion, &p.tm_k, 64, prow, &full[st], pol);
-            if (ht < 8) {
-              tma_load_3d_hint(vdst, &p.tm_v3, 0, prow, 0, &full[st], pol);  // both halves
+            tma_load_2d_hint(kdst, tmk, 0, prow, &full[st], pol);
+            tma_load_2d_hint(kdst + kRegion, tmk, 64, prow, &full[st], pol);
+            if (ht < 8 || casc) {
+              tma_load_3d_hint(vdst, tmv, 0, prow, 0, &full[st], pol);  // both halves
             } else {
               // a 128-row page: two 16 KiB copies ran faster than one of 32 KiB
               tma_load_2d_hint(vdst, &p.tm_v, 0, prow, &full[st], pol);
@@ -514,93 +598,140 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_wait(ebar, ek & 1, abort_flag, p.err);
       ++ek;
     };
-    const int nq = p.nq;
+    // Column h of an item: KV head h / cph of the item, sharer (h % cph) / G,
+    // q head (h / cph) * G + h % G among the item's q heads of that sequence.
+    auto sharer_cols = [&](int m) {  // the columns of sharer m
+      uint32_t mm = 0;
+      for (int hh = 0; hh < ht; ++hh) mm |= ((1u << p.group) - 1u) << (hh * cph + m * p.group);
+      return mm & ((1u << NH) - 1u);
+    };
+    // q head of column h among the item's q heads of its sequence
+    auto col_qhead = [&](int h) { return casc ? (h / cph) * p.group + h % p.group : h; };
     while (!*abort_flag) {
       mbar_wait(res_full, k & 1, abort_flag, p.err);
-      const int npart = resmeta[3];
+      const int npart = resmeta[3];  // shared-prefix items: the sharers
       if (npart < 0 || *abort_flag) break;
       const int s = resmeta[0], g = resmeta[1], part = resmeta[2], pbase = resmeta[4];
+      const int nsh = casc ? npart : 1;  // sequences of the item
       float res[NH], l2[NH];
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        res[h] = h < nq ? resbuf[h * 128 + e] : 0.f;
+        res[h] = resbuf[h * 128 + e];
         l2[h] = reslse[h];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(res_empty);
       ++k;
-      const int qh0 = g * nq;  // first q head of the group
-      if (npart == 1) {
+      // lane m of every epilogue warp holds sequence m of the item: its index,
+      // first partition record and partition count
+      int my_s = s, my_pb = pbase, my_np = npart;
+      if (casc) {
+        my_s = lane < nsh ? p.runs[static_cast<int64_t>(s) * kRunInts + 2 + lane] : 0;
+        my_pb = lane < nsh ? p.part_base[my_s] : 0;
+        my_np = lane < nsh ? p.part_base[my_s + 1] - my_pb : 1;
+      }
+      const int qh0 = g * ht * p.group;  // first q head of the item in each sequence
+      bool any_multi = false;
+      for (int m = 0; m < nsh; ++m) {
+        const int sm = __shfl_sync(0xffffffffu, my_s, m);
+        const int pbm = __shfl_sync(0xffffffffu, my_pb, m);
+        const int npm = __shfl_sync(0xffffffffu, my_np, m);
+        const uint32_t mm = casc ? sharer_cols(m) : (1u << (ht * p.group)) - 1u;
+        any_multi |= npm > 1;
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-          if (h < nq) {
-            const int64_t o = static_cast<int64_t>(s) * p.hq + qh0 + h;
-            p.out[o * kD + e] = f32_to_bf16_bits(res[h]);
-            if (e == 0 && p.lse) p.lse[o] = l2[h] * kLn2;
-          }
-        }
-        continue;
-      }
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        if (h < nq) {
-          const int64_t rec = static_cast<int64_t>(pbase + part) * p.hq + qh0 + h;
-          __stcg(p.part_o + rec * kD + e, res[h]);
-          if (e == 0) __stcg(p.part_lse + rec, l2[h]);
-        }
-      }
-      // the last partition of (s, g) to finish merges all of them
-      eexchange();
-      if (e == 0) {
-        __threadfence();
-        const int old = atomicAdd(p.merge_cnt + s * p.ngroups + g, 1);
-        merge_flag[k & 1] = (old == npart - 1);
-      }
-      eexchange();
-      if (!merge_flag[k & 1]) continue;
-      __threadfence();
-      float M[NH], W[NH], A[NH];
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        M[h] = -CUDART_INF_F;
-        W[h] = 0.f;
-        A[h] = 0.f;
-      }
-      const int64_t rec0 = static_cast<int64_t>(pbase) * p.hq + qh0;
-      for (int q = 0; q < npart; ++q) {
-        float li[NH], oi[NH];
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          if (h < nq) {
-            const int64_t rec = rec0 + static_cast<int64_t>(q) * p.hq + h;
-            li[h] = __ldcg(p.part_lse + rec);
-            oi[h] = __ldcg(p.part_o + rec * kD + e);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          if (h < nq && li[h] != -CUDART_INF_F) {
-            // one-pass log-sum-exp merge: rescale when a larger partition max appears
-            if (li[h] > M[h]) {
-              const float sc = exp2f(M[h] - li[h]);
-              W[h] = W[h] * sc + 1.f;
-              A[h] = A[h] * sc + oi[h];
-              M[h] = li[h];
+          if ((mm >> h) & 1u) {
+            const int qh = qh0 + col_qhead(h);
+            if (npm == 1) {
+              const int64_t o = static_cast<int64_t>(sm) * p.hq + qh;
+              p.out[o * kD + e] = f32_to_bf16_bits(res[h]);
+              if (e == 0 && p.lse) p.lse[o] = l2[h] * kLn2;
             } else {
-              const float f = exp2f(li[h] - M[h]);
-              W[h] += f;
-              A[h] += f * oi[h];
+              const int64_t rec = static_cast<int64_t>(pbm + part) * p.hq + qh;
+              __stcg(p.part_o + rec * kD + e, res[h]);
+              if (e == 0) __stcg(p.part_lse + rec, l2[h]);
             }
           }
         }
       }
+      if (!any_multi) continue;
+      // The last partition of a (sequence, KV head) to finish merges all of
+      // them.  Thread e < ht * M counts (KV head g ht + e / M, sharer e % M),
+      // whose G columns are [e G, (e + 1) G).
+      __threadfence();
+      eexchange();
+      if (warp == 7) {
+        bool last = false;
+        const int hh = e / msh, m = e - hh * msh;
+        const int sm = __shfl_sync(0xffffffffu, my_s, m & 31);
+        const int npm = __shfl_sync(0xffffffffu, my_np, m & 31);
+        if (e < ht * msh && m < nsh && npm > 1) {
+          const int old =
+              atomicAdd(p.merge_cnt + static_cast<int64_t>(sm) * p.hkv + g * ht + hh, 1);
+          last = old == npm - 1;
+        }
+        const unsigned done = __ballot_sync(0xffffffffu, last);
+        if (lane == 0) merge_flag[k & 1] = static_cast<int>(done);
+      }
+      eexchange();
+      const unsigned done = static_cast<unsigned>(merge_flag[k & 1]);
+      if (!done) continue;
+      __threadfence();
+      // bit b of `done`: q columns [b G, (b + 1) G)
+      uint32_t colsel = 0;
+      for (unsigned bits = done; bits; bits &= bits - 1)
+        colsel |= ((1u << p.group) - 1u) << ((__ffs(bits) - 1) * p.group);
+      for (int m = 0; m < nsh; ++m) {
+        const int sm = __shfl_sync(0xffffffffu, my_s, m);
+        const int pbm = __shfl_sync(0xffffffffu, my_pb, m);
+        const int npm = __shfl_sync(0xffffffffu, my_np, m);
+        const uint32_t mc = casc ? colsel & sharer_cols(m) : colsel;
+        if (!mc) continue;
+        float M[NH], W[NH], A[NH];
 #pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        if (h < nq) {
-          const bool live = W[h] > 0.f;
-          const int64_t o = static_cast<int64_t>(s) * p.hq + qh0 + h;
-          p.out[o * kD + e] = f32_to_bf16_bits(live ? A[h] / W[h] : 0.f);
-          if (e == 0 && p.lse) p.lse[o] = live ? (M[h] + log2f(W[h])) * kLn2 : -CUDART_INF_F;
+        for (int h = 0; h < NH; ++h) {
+          M[h] = -CUDART_INF_F;
+          W[h] = 0.f;
+          A[h] = 0.f;
+        }
+        const int64_t rec0 = static_cast<int64_t>(pbm) * p.hq + qh0;
+        for (int q = 0; q < npm; ++q) {
+          float li[NH], oi[NH];
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            li[h] = -CUDART_INF_F;
+            oi[h] = 0.f;
+            if ((mc >> h) & 1u) {
+              const int64_t rec = rec0 + static_cast<int64_t>(q) * p.hq + col_qhead(h);
+              li[h] = __ldcg(p.part_lse + rec);
+              oi[h] = __ldcg(p.part_o + rec * kD + e);
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            if (li[h] != -CUDART_INF_F) {
+              // one-pass log-sum-exp merge: rescale when a larger partition max appears
+              if (li[h] > M[h]) {
+                const float sc = exp2f(M[h] - li[h]);
+                W[h] = W[h] * sc + 1.f;
+                A[h] = A[h] * sc + oi[h];
+                M[h] = li[h];
+              } else {
+                const float f = exp2f(li[h] - M[h]);
+                W[h] += f;
+                A[h] += f * oi[h];
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          if ((mc >> h) & 1u) {
+            const bool live = W[h] > 0.f;
+            const int64_t o = static_cast<int64_t>(sm) * p.hq + qh0 + col_qhead(h);
+            p.out[o * kD + e] = f32_to_bf16_bits(live ? A[h] / W[h] : 0.f);
+            if (e == 0 && p.lse) p.lse[o] = live ? (M[h] + log2f(W[h])) * kLn2 : -CUDART_INF_F;
+          }
         }
       }
     }
@@ -768,8 +899,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     const int pj = r >> (4 + hts);
     // row r of the V tile: page pj holds its rows for dims 0-63, then 64-127
     const uint32_t v_row_off = pj * (ht * 4096) + (r & ((16 << hts) - 1)) * 128;
-    const int c_lo = ((r >> 4) & (ht - 1)) * p.group;  // this row's q columns [c_lo, c_lo + G)
-    const int c_hi = c_lo + p.group;
+    // this row's q columns start at its KV head's block of cph columns; an
+    // item with k sharers uses the first k * G of them
+    const int c_row = ((r >> 4) & (ht - 1)) * cph;
     const int rtok = (pj << 4) | (r & 15);
     uint32_t d = 0, t = 0, xk = 0, nfin = 0;
     // all four softmax warps have passed this point (bounded, unlike bar.sync)
@@ -836,10 +968,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         tc_fence_before();
         mbar_arrive(&s_free[b]);
         const bool valid = tok0 + rtok < tok1 && mypb >= 0;
+        // the row's columns: its KV head's G q heads for each of the item's sharers
+        const uint32_t cm = ((1u << ((casc ? npart : 1) * p.group)) - 1u) << c_row;
         float x[NH];
 #pragma unroll
         for (int h = 0; h < NH; ++h)
-          x[h] = (valid && h >= c_lo && h < c_hi) ? sv[h] * p.scale_log2 : -CUDART_INF_F;
+          x[h] = (valid && ((cm >> h) & 1u)) ? sv[h] * p.scale_log2 : -CUDART_INF_F;
         // tile max per q column: warp shuffle, then across the four softmax warps
         float* rm = red_max + (t & 1) * 4 * NH;
 #pragma unroll
@@ -939,9 +1073,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int NH, int GR>
+template <int NH, int GR, bool kCasc = false>
 int launch_nh(const TcParams& prm, int64_t item_bound, cudaStream_t stream) {
-  auto kern = decode_tc_kernel<NH, GR>;
+  auto kern = decode_tc_kernel<NH, GR, kCasc>;
   static KernelLaunchCache cache;
   const int per_sm =
       cache.blocks_per_sm(reinterpret_cast<const void*>(kern), kThreads, Smem<NH>::kBytes);
@@ -1023,12 +1157,33 @@ int launch_decode_tcgen05(const DecodeArgs& a) {
     const uint32_t box[3] = {64, 16, 1};
     if (!encode_bf16_map(&p.tm_q, a.q, 3, dims, strides, box)) return PA_ERR_CUDA;
   }
+  const bool casc = a.casc_cols == 8 || a.casc_cols == 16;
+  if (casc) {
+    // shared-prefix launch: the plan picks 1, 2, 4 or 8 KV heads per tile
+    for (int h = 0; h < 4; ++h) {
+      if (a.pool.num_kv_heads % (1 << h)) continue;  // never chosen
+      const uint64_t dk[2] = {static_cast<uint64_t>(kD), static_cast<uint64_t>(rows)};
+      const uint64_t sk[1] = {kD * 2};
+      const uint32_t bk[2] = {64, static_cast<uint32_t>(16 << h)};
+      if (!encode_bf16_map(&p.tm_kc[h], a.k_pool, 2, dk, sk, bk)) return PA_ERR_CUDA;
+      const uint64_t dv[3] = {64, static_cast<uint64_t>(rows), 2};
+      const uint64_t sv[2] = {kD * 2, 128};
+      const uint32_t bv[3] = {64, static_cast<uint32_t>(16 << h), 2};
+      if (!encode_bf16_map(&p.tm_vc[h], a.v_pool, 3, dv, sv, bv)) return PA_ERR_CUDA;
+    }
+  }
+  p.q = a.q;
+  p.q_stride = a.q_stride;
   p.block_tables = a.block_tables;
   p.context_lens = a.context_lens;
   p.header = a.ws.header;
   p.part_base = a.ws.part_base;
   p.merge_cnt = a.ws.merge_cnt;
   p.items = a.ws.items;
+  p.pitems = a.ws.pitems;
+  p.runs = a.ws.runs;
+  p.seq_span = a.ws.seq_span;
+  p.seq_pp = a.ws.seq_pp;
   p.part_o = a.ws.part_o;
   p.part_lse = a.ws.part_lse;
   p.out = a.out;
@@ -1043,7 +1198,14 @@ int launch_decode_tcgen05(const DecodeArgs& a) {
   p.ngroups = a.pool.num_kv_heads >> sh.ht_shift;
   p.nq = group << sh.ht_shift;
   p.scale_log2 = a.scale * kLog2e;
-  const int64_t bound = static_cast<int64_t>(a.num_seqs) * a.max_parts * p.ngroups;
+  if (casc) {
+    // the shared-prefix items first (none unless the plan found shared prefixes)
+    const int64_t pbound = static_cast<int64_t>(a.num_seqs / 2 + 1) * a.max_parts * a.pool.num_kv_heads;
+    const int st = a.casc_cols == 8 ? launch_nh<8, 8, true>(p, pbound, a.stream)
+                                     : launch_nh<16, 16, true>(p, pbound, a.stream);
+    if (st != PA_OK) return st;
+  }
+  const int64_t bound = static_cast<int64_t>(a.num_seqs) * (a.max_parts + 1) * p.ngroups;
   if (group == 1) return launch_nh<8, 1>(p, bound, a.stream);
   if (sh.nh == 8) return launch_nh<8, 8>(p, bound, a.stream);
   return launch_nh<16, 16>(p, bound, a.stream);

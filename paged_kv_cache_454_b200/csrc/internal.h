@@ -59,21 +59,36 @@ inline int launch_status() {
 // Decode: the work plan shared by the decode kernels and the merge.
 // ---------------------------------------------------------------------------
 // The workspace holds, in order:
-//   header       int32[4]: total items, total partitions, dynamic item counter,
-//                partition length chosen by the plan
+//   header       int32[8]: total items, total partitions, dynamic item counter,
+//                partition length chosen by the plan, shared-prefix items,
+//                their dynamic counter, log2 of the KV heads per shared-prefix
+//                item, the shared prefixes' partition length
 //   part_base    int32[num_seqs + 1]: exclusive prefix of partitions per sequence
-//   merge_cnt    int32[num_seqs * Hkv]: partitions finished per (sequence, KV-head group)
+//   merge_cnt    int32[num_seqs * Hkv]: partitions finished per (sequence, KV head)
 //   work list    int2[num_seqs * max_parts * Hkv]: (seq, head group << 16 | partition)
-//                in the plan's order; a head group is item_heads KV heads
-//   partial out  float[num_seqs * max_parts * Hq * D]
-//   partial lse  float[num_seqs * max_parts * Hq]   (base-2 log-sum-exp)
+//                in the plan's order; a head group is item_heads KV heads; the
+//                partition counts from the end of the sequence's shared prefix
+//   seq_span     int32[num_seqs]: tokens of the sequence's shared prefix (0: none)
+//   seq_pp       int32[num_seqs]: partitions of that prefix
+//   runs         int32[num_seqs / 2 * kRunInts]: per run of sequences sharing a
+//                prefix: its length in tokens, its member count, the members
+//   prefix list  int2[num_seqs / 2 * Hkv * max_parts]: (run, head group << 16 |
+//                partition) of the shared-prefix items
+//   partial out  float[num_seqs * (max_parts + 1) * Hq * D]
+//   partial lse  float[num_seqs * (max_parts + 1) * Hq]   (base-2 log-sum-exp)
 // max_parts is the partition count of the longest possible context at the
-// shortest partition length the call may use.
+// shortest partition length the call may use; a sequence with a shared prefix
+// may have one partition more (the prefix and the rest are split separately).
+constexpr int kRunInts = 18;  // span, members, up to 16 member sequences
 struct DecodeWorkspace {
   int* header;
   int* part_base;
   int* merge_cnt;
   int2* items;
+  int* seq_span;
+  int* seq_pp;
+  int* runs;
+  int2* pitems;
   float* part_o;
   float* part_lse;
 };
@@ -102,6 +117,11 @@ struct DecodeArgs {
   int target_items;  // the plan lengthens partitions while at least this many items remain
   int max_parts;     // workspace bound (partitions of the longest context at min_part)
   int item_heads = 1;  // KV heads per work item (the tensor-core kernel packs small groups)
+  // Shared-prefix cascade (tensor-core kernel): sequences that share their
+  // first blocks read the shared span once, in items whose casc_cols (8 or 16)
+  // q columns are the sharers' q heads (the plan picks the sharers and KV
+  // heads per item).  0: no cascade.
+  int casc_cols = 0;
   DecodeWorkspace ws;
   unsigned int* err;
   cudaStream_t stream;
@@ -123,6 +143,8 @@ constexpr int kSimtPartition = 512;
 constexpr int kTcPartition = 1024;
 constexpr int kTcMaxPartition = 8192;
 constexpr int kTcItemsPerSm = 2;
+// The plan finds shared prefixes in batches of up to this many sequences.
+constexpr int kCascMaxSeqs = 1024;
 
 struct PrefillArgs {
   const uint16_t* q;

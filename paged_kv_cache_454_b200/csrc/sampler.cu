@@ -45,9 +45,11 @@ __device__ __forceinline__ float float_of(uint32_t k) {
 }
 
 // Calls f(value, index) for every element of row x[0, V), each thread keeping
-// four loads in flight: 16-byte vectors when the row is 16-byte aligned (64 KiB
-// in flight per CTA, what one SM needs to stream at its share of HBM), single
-// floats otherwise.  Elements reach f in no particular order.
+// kInflight loads in flight: 16-byte vectors when the row is 16-byte aligned
+// (128 KiB in flight per CTA: one CTA per row streams a row at about its SM's
+// share of HBM), single floats otherwise.  Each thread sees its elements in
+// increasing index order.
+constexpr int kInflight = 8;
 template <typename F>
 __device__ __forceinline__ void for_each_logit(const float* __restrict__ x, int V, F f) {
   const int tid = threadIdx.x;
@@ -55,12 +57,12 @@ __device__ __forceinline__ void for_each_logit(const float* __restrict__ x, int 
     const float4* x4 = reinterpret_cast<const float4*>(x);
     const int V4 = V >> 2;
     int i = tid;
-    for (; i + 3 * kThreads < V4; i += 4 * kThreads) {
-      float4 a[4];
+    for (; i + (kInflight - 1) * kThreads < V4; i += kInflight * kThreads) {
+      float4 a[kInflight];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) a[q] = __ldg(x4 + i + q * kThreads);
+      for (int q = 0; q < kInflight; ++q) a[q] = __ldg(x4 + i + q * kThreads);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < kInflight; ++q) {
         const int b = 4 * (i + q * kThreads);
         f(a[q].x, b);
         f(a[q].y, b + 1);
@@ -79,14 +81,37 @@ __device__ __forceinline__ void for_each_logit(const float* __restrict__ x, int 
     return;
   }
   int i = tid;
-  for (; i + 3 * kThreads < V; i += 4 * kThreads) {
-    float a[4];
+  for (; i + (kInflight - 1) * kThreads < V; i += kInflight * kThreads) {
+    float a[kInflight];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) a[q] = x[i + q * kThreads];
+    for (int q = 0; q < kInflight; ++q) a[q] = x[i + q * kThreads];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) f(a[q], i + q * kThreads);
+    for (int q = 0; q < kInflight; ++q) f(a[q], i + q * kThreads);
   }
   for (; i < V; i += kThreads) f(x[i], i);
+}
+
+// As for_each_logit, but hands 16-byte vectors to f4(vector, index of its
+// first element) and single elements to f1(value, index).
+template <typename F4, typename F1>
+__device__ __forceinline__ void for_each_logit4(const float* __restrict__ x, int V, F4 f4, F1 f1) {
+  const int tid = threadIdx.x;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) == 0) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const int V4 = V >> 2;
+    int i = tid;
+    for (; i + (kInflight - 1) * kThreads < V4; i += kInflight * kThreads) {
+      float4 a[kInflight];
+#pragma unroll
+      for (int q = 0; q < kInflight; ++q) a[q] = __ldg(x4 + i + q * kThreads);
+#pragma unroll
+      for (int q = 0; q < kInflight; ++q) f4(a[q], 4 * (i + q * kThreads));
+    }
+    for (; i < V4; i += kThreads) f4(__ldg(x4 + i), 4 * i);
+    for (int j = 4 * V4 + tid; j < V; j += kThreads) f1(x[j], j);
+    return;
+  }
+  for_each_logit(x, V, f1);
 }
 
 // Mass of logit x in 32.32 fixed point: exp2((x - xmax) * scale) * 2^32.
@@ -153,6 +178,34 @@ __device__ void block_sort(uint64_t* v, int n2, bool desc) {
   }
 }
 
+// Sort of the n <= kThreads distinct entries v[0, n) by rank: thread t counts
+// the entries ahead of v[t] and writes it to that position of tmp (which must
+// not overlap v[0, n)), then v takes tmp.  Descending if `desc`.  Two barriers
+// in all, against the bitonic network's one per stage.  Ends with a barrier.
+__device__ void rank_sort(uint64_t* v, int n, uint64_t* tmp, bool desc) {
+  const int t = threadIdx.x;
+  if (t < n) {
+    const uint64_t x = v[t];
+    int r = 0;
+    int j = 0;
+    for (; j + 8 <= n; j += 8) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint64_t y = v[j + q];
+        r += desc ? (y > x) : (y < x);
+      }
+    }
+    for (; j < n; ++j) {
+      const uint64_t y = v[j];
+      r += desc ? (y > x) : (y < x);
+    }
+    tmp[r] = x;
+  }
+  __syncthreads();
+  if (t < n) v[t] = tmp[t];
+  __syncthreads();
+}
+
 // Inclusive scan of one uint64 per thread over the CTA; `tot` gets the total.
 __device__ uint64_t block_scan64(uint64_t x, uint64_t* wbuf, uint64_t* tot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -187,6 +240,7 @@ struct Smem {
   uint32_t tmax[kThreads];    // each thread's largest key (pass 1)
   unsigned long long red64;
   int count;
+  int overflow;
   int cut;
   int bin;
   uint32_t above_cnt;
@@ -210,17 +264,57 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
   float u = uniform[row];
   u = (u >= 0.f && u < 1.f) ? u : 0.f;
 
-  // ---- pass 1: the largest key, lowest index among equals ----
-  uint32_t bk = 0;
-  int bi = 0x7fffffff;
-  auto take = [&](float v, int i) {
-    const uint32_t k = key_of(v);
-    if (k > bk || (k == bk && i < bi)) {
-      bk = k;
-      bi = i;
+  // ---- pass 1: the largest key, lowest index among equals; each thread also
+  // keeps its four best elements (key descending, index ascending), which
+  // usually hold every Top-K candidate it has ----
+  constexpr int kNone = 0x7fffffff;  // index of an empty slot
+  uint32_t k0 = 0, k1 = 0, k2 = 0, k3 = 0;
+  int i0 = kNone, i1 = kNone, i2 = kNone, i3 = kNone;
+  // indices arrive in increasing order, so an equal key ranks below a kept
+  // one unless that slot is empty: an element enters the four when its key
+  // beats the fourth's or the fourth slot is empty
+  auto insert = [&](uint32_t k, int i) {
+    if (k > k3 || i3 == kNone) {
+      if (k > k2 || (k == k2 && i < i2)) {
+        k3 = k2;
+        i3 = i2;
+        if (k > k1 || (k == k1 && i < i1)) {
+          k2 = k1;
+          i2 = i1;
+          if (k > k0 || (k == k0 && i < i0)) {
+            k1 = k0;
+            i1 = i0;
+            k0 = k;
+            i0 = i;
+          } else {
+            k1 = k;
+            i1 = i;
+          }
+        } else {
+          k2 = k;
+          i2 = i;
+        }
+      } else {
+        k3 = k;
+        i3 = i;
+      }
     }
   };
-  for_each_logit(x, V, take);
+  // the common case -- none of a vector's four elements enters -- costs one
+  // compare against the fourth kept key
+  auto take4 = [&](float4 a, int b) {
+    const uint32_t ka = key_of(a.x), kb = key_of(a.y), kc = key_of(a.z), kd = key_of(a.w);
+    if (__builtin_expect(max(max(ka, kb), max(kc, kd)) > k3 || i3 == kNone, 0)) {
+      insert(ka, b);
+      insert(kb, b + 1);
+      insert(kc, b + 2);
+      insert(kd, b + 3);
+    }
+  };
+  auto take1 = [&](float v, int i) { insert(key_of(v), i); };
+  for_each_logit4(x, V, take4, take1);
+  uint32_t bk = k0;
+  int bi = i0;
   sm.tmax[tid] = bk;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -274,26 +368,55 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
       }
       t0 = prefix;
     }
-    if (tid == 0) sm.count = 0;
+    if (tid == 0) {
+      sm.count = 0;
+      sm.overflow = 0;
+    }
     __syncthreads();
-    auto collect = [&](float v, int i) {
-      const uint32_t k = key_of(v);
-      if (k >= t0) {
-        const int pos = atomicAdd(&sm.count, 1);
-        // (key, -index): descending order is by logit, then by index
-        if (pos < kCand)
-          sm.cand[pos] = (static_cast<uint64_t>(k) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
-      }
+    // (key, -index): descending order is by logit, then by index
+    auto pack = [](uint32_t k, int i) {
+      return (static_cast<uint64_t>(k) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
     };
-    for_each_logit(x, V, collect);
+    // Every element at or above t0 is among its thread's four kept ones unless
+    // the fourth is too (the thread may have more): then the row is read again.
+    if (i3 != kNone && k3 >= t0) sm.overflow = 1;
+    {
+      const int c = (i0 != kNone && k0 >= t0) + (i1 != kNone && k1 >= t0) +
+                    (i2 != kNone && k2 >= t0) + (i3 != kNone && k3 >= t0);
+      if (c) {
+        int pos = atomicAdd(&sm.count, c);
+        if (pos < kCand) sm.cand[pos] = pack(k0, i0);
+        if (c > 1 && ++pos < kCand) sm.cand[pos] = pack(k1, i1);
+        if (c > 2 && ++pos < kCand) sm.cand[pos] = pack(k2, i2);
+        if (c > 3 && ++pos < kCand) sm.cand[pos] = pack(k3, i3);
+      }
+    }
     __syncthreads();
+    if (sm.overflow) {
+      __syncthreads();
+      if (tid == 0) sm.count = 0;
+      __syncthreads();
+      auto collect = [&](float v, int i) {
+        const uint32_t k = key_of(v);
+        if (k >= t0) {
+          const int pos = atomicAdd(&sm.count, 1);
+          if (pos < kCand) sm.cand[pos] = pack(k, i);
+        }
+      };
+      for_each_logit(x, V, collect);
+      __syncthreads();
+    }
     const int n = sm.count;
     if (n <= kCand) {
       int n2 = 1;
       while (n2 < n) n2 <<= 1;
-      for (int i = n + tid; i < n2; i += kThreads) sm.cand[i] = 0ull;  // below every real entry
-      __syncthreads();
-      block_sort(sm.cand, n2, true);
+      if (n <= kThreads) {
+        rank_sort(sm.cand, n, sm.cand + kThreads, true);
+      } else {
+        for (int i = n + tid; i < n2; i += kThreads) sm.cand[i] = 0ull;  // below every real entry
+        __syncthreads();
+        block_sort(sm.cand, n2, true);
+      }
       const uint32_t tk = static_cast<uint32_t>(sm.cand[K - 1] >> 32);
       // survivors of Top-K: the leading K entries and any ties with the K-th
       if (tid == 0) {
@@ -348,7 +471,10 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
                             : ~0ull;
       }
       __syncthreads();
-      block_sort(sm.cand, n2, false);
+      if (m2 <= kThreads)
+        rank_sort(sm.cand, m2, sm.cand + kThreads, false);
+      else
+        block_sort(sm.cand, n2, false);
       uint64_t mine2 = 0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {

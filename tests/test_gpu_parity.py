@@ -137,6 +137,52 @@ def lay_g12():
                               num_kv_heads=3, head_dim=128)
 
 
+# Shared-prefix cascade: runs of sequences over common prompt blocks.  The plan
+# takes the longest run for the sharers per item (at most 16 / group) and packs
+# KV heads into the rest of the item's 16 q columns.
+def lay_casc_mha4():
+    # runs of 4: four sharers x four KV heads per item; a run of 3 and one of 2
+    # under-fill their items; an unshared sequence; two prompt lengths
+    return synth.prefix_runs("casc_mha4", 121, [4, 4, 4, 4, 2, 3, 1], [300, 600, 300, 600, 300, 600, 300],
+                             400, num_q_heads=8, num_kv_heads=8)
+
+
+def lay_casc_mha17():
+    # a run of 17: sixteen sharers x one KV head per item, the 17th on its own
+    return synth.prefix_runs("casc_mha17", 122, [17, 4, 2], 200, 150, num_q_heads=4,
+                             num_kv_heads=4)
+
+
+def lay_casc_gqa8():
+    # group 8: two sharers per item; long prompts over several partitions; a run
+    # of 5 cut into 2 + 2 + 1
+    return synth.prefix_runs("casc_gqa8", 123, [2, 2, 3, 1, 5], [1000, 2000, 700, 0, 1500], 1500,
+                             num_q_heads=16, num_kv_heads=2)
+
+
+def lay_casc_gqa5():
+    # group 5: three sharers (15 of 16 columns); a run of 4 cut into 3 + 1
+    return synth.prefix_runs("casc_gqa5", 124, [3, 3, 2, 4], 500, 300, num_q_heads=10,
+                             num_kv_heads=2)
+
+
+def lay_casc_gqa4():
+    # group 4, runs of 2: two sharers x two KV heads per item
+    return synth.prefix_runs("casc_gqa4", 125, [2, 2, 2], 900, 700, num_q_heads=16,
+                             num_kv_heads=4)
+
+
+def lay_casc_edges():
+    # empty contexts (no prompt, empty suffix), a prompt of 128 tokens whose
+    # shared span (7 whole blocks after the copy-on-write) is too short to
+    # cascade, suffixes of zero tokens after a shared prompt
+    return synth.prefix_runs("casc_edges", 126, [4, 1, 1, 2, 3], [256, 0, 0, 128, 400], 20,
+                             num_q_heads=8, num_kv_heads=8, min_suffix=0)
+
+
+CASCADE_LAYOUTS = ["casc_mha4", "casc_mha17", "casc_gqa8", "casc_gqa5", "casc_gqa4", "casc_edges"]
+
+
 DECODE_LAYOUTS = {
     "tiny": synth.tiny,
     "mha128": lay_mha128,
@@ -156,6 +202,12 @@ DECODE_LAYOUTS = {
     "short_g16": lay_short_g16,
     "short_g12": lay_short_g12,
     "g12": lay_g12,
+    "casc_mha4": lay_casc_mha4,
+    "casc_mha17": lay_casc_mha17,
+    "casc_gqa8": lay_casc_gqa8,
+    "casc_gqa5": lay_casc_gqa5,
+    "casc_gqa4": lay_casc_gqa4,
+    "casc_edges": lay_casc_edges,
 }
 
 
@@ -252,7 +304,8 @@ def test_decode_simt(name, partition):
 
 @pytest.mark.parametrize("name", ["gqa8", "gqa5", "g16", "shared_prefix", "shared_many", "mha128",
                                   "short_gqa", "short_mha", "gqa4", "gqa2_h6", "mha_h5",
-                                  "mha_h16", "gqa8_h3", "short_g16", "short_g12", "g12"])
+                                  "mha_h16", "gqa8_h3", "short_g16", "short_g12", "g12"]
+                         + CASCADE_LAYOUTS)
 @pytest.mark.parametrize("partition", [0, 128, 1024, 1 << 20])
 def test_decode_tcgen05(name, partition):
     st, ref = _step_and_ref(name)
@@ -266,6 +319,113 @@ def test_decode_tcgen05(name, partition):
         raise
     H.compare_step(got, ref, what=f"{name} tcgen05 p={partition}")
     assert pa().pa_get_device_error() == 0
+
+
+@pytest.mark.parametrize("tail", [0, 5], ids=["whole_blocks", "ragged"])
+@pytest.mark.parametrize("partition", [0, 128])
+def test_decode_cascade_identical_tables(tail, partition):
+    # sequences whose tables are identical over their whole context: the shared
+    # span is every whole block, so a sequence with no tokens after it has no
+    # items of its own and the shared-prefix items alone produce its output
+    # (written directly when it has a single partition).  Decode only, on the
+    # pool as drawn: no new tokens are written into the shared blocks.
+    import torch
+    rng = np.random.default_rng(127)
+    lens, tables, nb = [], [], 0
+    for n, blocks in [(4, 20), (3, 8), (2, 40), (5, 9)]:
+        row = list(range(nb, nb + blocks))
+        nb += blocks
+        for j in range(n):
+            lens.append(16 * blocks - (tail if j % 2 else 0))
+            tables.append(row)
+    S = len(lens)
+    mb = max(len(r) for r in tables)
+    tab = np.full((S, mb), synth.INT32_MAX, np.int32)
+    for s, r in enumerate(tables):
+        tab[s, :len(r)] = r
+    perm = rng.permutation(nb).astype(np.int32)
+    tab = np.where(tab == synth.INT32_MAX, tab, perm[np.minimum(tab, nb - 1)])
+    hq, hkv, d = 8, 8, 128
+    kp = synth.normal_bf16(rng, (nb, hkv, 16, d))
+    vp = synth.normal_bf16(rng, (nb, hkv, 16, d))
+    q = synth.normal_bf16(rng, (S, hq, d))
+    lens = np.asarray(lens, np.int32)
+    want, want_lse = oracle.decode(q, kp, vp, tab, lens, 1 / np.sqrt(d))
+    out, lse = pa().pa_decode(H.dev_bf16(q), H.dev_bf16(kp), H.dev_bf16(vp), H.dev_i32(tab),
+                              H.dev_i32(lens), float(1 / np.sqrt(d)),
+                              kernel=pa().PA_KERNEL_TCGEN05, partition_tokens=partition,
+                              want_lse=True)
+    torch.cuda.synchronize()
+    H.assert_close(H.host_f64(out), want, what=f"identical tables tail={tail}")
+    H.assert_lse_close(H.host_f64(lse), want_lse, what=f"identical tables tail={tail}")
+    assert pa().pa_get_device_error() == 0
+
+
+def _expected_cascade(lay):
+    """Sharers per item and log2 of the KV heads per item the plan should pick
+    (items of 8 q columns for groups up to 4, of 16 up to 8), and whether any
+    sub-run's shared span reaches 128 tokens."""
+    G, hkv = lay.group_size, lay.num_kv_heads
+    cols = 8 if G <= 4 else 16
+    lens, tab = lay.context_lens, lay.block_tables
+    runs = {}
+    for s in range(lay.num_seqs):
+        if lens[s] > 0:
+            runs.setdefault(int(tab[s, 0]), []).append(s)
+    rmax = max(len(v) for v in runs.values())
+    M = min(rmax, cols // G)
+    hts = 0
+    while hts < 3 and G * (2 << hts) * M <= cols and hkv % (2 << hts) == 0:
+        hts += 1
+    any_span = False
+    for members in runs.values():
+        members = sorted(members)
+        for i in range(0, len(members), M):
+            sub = members[i:i + M]
+            if len(sub) < 2:
+                continue
+            full = min(int(lens[s]) // 16 for s in sub)
+            lcp = 0
+            while lcp < full and all(tab[s, lcp] == tab[sub[0], lcp] for s in sub):
+                lcp += 1
+            any_span |= lcp * 16 >= 128
+    return M, hts, any_span
+
+
+@pytest.mark.parametrize("name", CASCADE_LAYOUTS + ["shared_prefix", "mha128"])
+def test_decode_cascade_plan(name):
+    # white box: the plan's header in the caller's workspace (int32 [8]: own
+    # items, partitions, their counter, partition length, shared-prefix items,
+    # their counter, log2 KV heads | sharers << 8 per shared-prefix item,
+    # their partition length) shows the cascade ran where the layout has shared prompts, with
+    # the expected sharers and heads per item, and that every item was taken
+    import torch
+    st, ref = _step_and_ref(name)
+    lay = st.layout
+    S, hq = lay.num_seqs, lay.num_q_heads
+    n = pa().pa_decode_workspace_size(S, hq, st.k_pool, lay.max_blocks)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    got = {}
+    if lay.copy_pairs.size:
+        pa().pa_copy_blocks(st.k_pool, st.v_pool, lay.copy_pairs)
+    pa().pa_reshape_and_cache(st.key, st.value, st.k_pool, st.v_pool, st.slot_mapping)
+    out, lse = pa().pa_decode(st.q, st.k_pool, st.v_pool, st.tables, st.lens, lay.scale,
+                              workspace=ws, kernel=pa().PA_KERNEL_TCGEN05, want_lse=True)
+    torch.cuda.synchronize()
+    hdr = ws[:32].view(torch.int32).cpu().numpy()
+    H.compare_step({"decode": (out, lse)}, {"decode": ref["decode"]}, what=f"{name} cascade")
+    # every item was taken (each CTA's last, empty grab also counts)
+    assert hdr[2] >= hdr[0] and hdr[5] >= hdr[4], hdr
+    shared = len(set(int(lay.block_tables[s, 0]) for s in range(S) if lay.context_lens[s] > 0)) < \
+        int((lay.context_lens > 0).sum())
+    if not shared:
+        assert hdr[4] == 0, hdr
+        return
+    M, hts, any_span = _expected_cascade(lay)
+    assert hdr[6] & 0xff == hts and hdr[6] >> 8 == M, (hdr, M, hts)
+    assert (hdr[4] > 0) == any_span, hdr
+    if any_span:
+        assert hdr[7] % 128 == 0 and hdr[7] >= 128, hdr
 
 
 def test_decode_default_kernel_choice():

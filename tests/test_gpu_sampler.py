@@ -96,6 +96,28 @@ def test_edges_greedy_ties_nan_and_neg_inf():
     assert got[3] == 1   # top-k 1 keeps both tied maxima; u = 0.75 draws the second
 
 
+@pytest.mark.parametrize("vocab", [4096, 152064])
+def test_clustered_top_logits(vocab):
+    # The largest logits sit next to each other in runs of 16, so a thread's
+    # elements (four consecutive ones per 16-byte load) hold more than four Top-K
+    # candidates: the kernel cannot take its candidates from the four it keeps
+    # per thread and reads the row a second time.
+    rng = np.random.default_rng(11)
+    rows = 16
+    x = rng.normal(size=(rows, vocab)).astype(np.float32)
+    for r in range(rows):
+        for start in rng.choice(vocab // 16 - 1, size=4, replace=False) * 16 + rng.integers(0, 4):
+            x[r, start:start + 16] = 8 + rng.normal(size=16)
+    T = rng.choice([0.5, 1.0], size=rows).astype(np.float32)
+    K = rng.choice([1, 5, 20, 50, 64, 200], size=rows).astype(np.int32)
+    P = rng.choice([0.5, 0.9, 1.0], size=rows).astype(np.float32)
+    u = rng.random(rows).astype(np.float32)
+    got = run(x, T, K, P, u)
+    for r in range(rows):
+        ok = acceptable(x[r], float(T[r]), int(K[r]), float(P[r]), float(u[r]))
+        assert int(got[r]) in ok, (r, float(T[r]), int(K[r]), float(P[r]), float(u[r]), got[r], ok)
+
+
 def test_same_inputs_same_tokens():
     rng = np.random.default_rng(2)
     x = rng.normal(size=(64, 5000)).astype(np.float32)

@@ -259,6 +259,64 @@ def llama13b_sampling(seed: int = 2, groups: int = 64, samples: int = 4,
                   notes=f"{groups} groups x {samples} samples; {prefix}-token shared prefix")
 
 
+def prefix_runs(name: str, seed: int, run_sizes, prefix, max_suffix: int, *, num_q_heads: int,
+                num_kv_heads: int, head_dim: int = 128, min_suffix: int = 1,
+                cow: bool = True) -> Layout:
+    """Runs of sequences sharing a prompt: run ``r`` has ``run_sizes[r]``
+    sequences that all point at the same physical blocks for the first
+    ``prefix[r]`` tokens (``prefix`` may be one number for every run).  With
+    ``cow`` the sequences after the first take a copy-on-write copy of the last
+    prompt block (``copy_pairs``); each then owns a private suffix of uniform
+    [min_suffix, max_suffix] tokens.  A run of size 1 is an unshared sequence;
+    a prefix of 0 gives an empty context when the suffix is empty too.  Pool
+    1.25x the blocks needed, shuffled."""
+    rng = np.random.default_rng(seed)
+    bs = BLOCK_SIZE
+    run_sizes = [int(n) for n in run_sizes]
+    prefix = [int(prefix)] * len(run_sizes) if np.isscalar(prefix) else [int(x) for x in prefix]
+    S = int(sum(run_sizes))
+    suffix = rng.integers(min_suffix, max_suffix + 1, size=S)
+    lens = np.zeros(S, np.int64)
+    need = 0
+    s = 0
+    for n, pre in zip(run_sizes, prefix):
+        pb = -(-pre // bs)
+        need += pb + (n - 1 if cow and pb else 0)
+        for j in range(n):
+            lens[s] = pre + suffix[s]
+            need += -(-int(lens[s]) // bs) - pb
+            s += 1
+    num_blocks = max(1, int(math.ceil(1.25 * need)))
+    order = _alloc_order(rng, num_blocks, True)
+    max_blocks = max(1, max(-(-int(L) // bs) for L in lens))
+    tables = np.full((S, max_blocks), INT32_MAX, dtype=np.int32)
+    pairs = []
+    k = 0
+    s = 0
+    for n, pre in zip(run_sizes, prefix):
+        pb = -(-pre // bs)
+        shared = order[k:k + pb]
+        k += pb
+        for j in range(n):
+            tables[s, :pb] = shared
+            if j > 0 and cow and pb:
+                tables[s, pb - 1] = order[k]
+                pairs.append((shared[-1], order[k]))
+                k += 1
+            for b in range(pb, -(-int(lens[s]) // bs)):
+                tables[s, b] = order[k]
+                k += 1
+            s += 1
+    ref = np.zeros(num_blocks, np.int32)
+    for s in range(S):
+        for b in range(-(-int(lens[s]) // bs)):
+            ref[tables[s, b]] += 1
+    return Layout(name, seed, num_q_heads, num_kv_heads, head_dim, bs, num_blocks,
+                  lens.astype(np.int32), tables, np.ones(S, np.int32), np.zeros(S, bool),
+                  copy_pairs=np.asarray(pairs, np.int64).reshape(-1, 2), ref_counts=ref,
+                  notes=f"runs {run_sizes} sharing prompt prefixes")
+
+
 def gqa70b_long(seed: int = 3, batch: int = 128) -> Layout:
     """70B-like GQA long context: 64 q heads / 8 KV heads, head_dim 128,
     contexts log-uniform in [1024, 32768] (floor of exp(U(ln 1024, ln 32768))),
@@ -312,17 +370,23 @@ def _poison_slots(layout: Layout):
     if layout.copy_pairs.size:
         referenced[layout.copy_pairs[:, 0]] = True
     unused = np.nonzero(~referenced)[0]
+    # A copy-on-write source is copied whole to its destinations, whose
+    # sequences may read past the source owner's context: its slots stay finite.
+    src = set(layout.copy_pairs[:, 0].tolist()) if layout.copy_pairs.size else set()
     blocks, offs = [], []
     for s in range(layout.num_seqs):
         L = int(layout.context_lens[s])
         if L % bs:
             last = int(layout.block_tables[s, L // bs])
+            if last in src:
+                continue
             for o in range(L % bs, bs):
                 blocks.append(last)
                 offs.append(o)
     sm = layout.slot_mapping()
-    blocks.extend((sm // bs).tolist())
-    offs.extend((sm % bs).tolist())
+    keep = np.array([int(b) not in src for b in (sm // bs).tolist()], bool)
+    blocks.extend((sm[keep] // bs).tolist())
+    offs.extend((sm[keep] % bs).tolist())
     if layout.copy_pairs.size:
         for dst in layout.copy_pairs[:, 1]:
             for o in range(bs):
