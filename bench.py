@@ -270,9 +270,7 @@ class Workload:
     def launches_per_step(self):
         """Library kernel launches in one step: block copies (480 pairs per
         launch), the cache write, the decode plan and decode kernel (plus the
-        shared-prefix launch on the tensor-core path for groups up to 8 and
-        2..1024 sequences, which returns at once when no prefix is shared, or
-        the merge kernel on the CUDA-core path), the prefill kernel."""
+        merge kernel on the CUDA-core path), the prefill kernel."""
         lay = self.layout
         n = 1  # cache write
         if lay.copy_pairs.size:
@@ -281,8 +279,6 @@ class Workload:
             tensor_core = self.kernel == 2 or (
                 self.kernel == 0 and lay.head_dim == 128 and lay.group_size <= 16)
             n += 2 if tensor_core else 3
-            if tensor_core and lay.group_size <= 8 and 2 <= len(self.dec) <= 1024:
-                n += 1
         if len(self.pf):
             n += 1
         return n

@@ -254,11 +254,11 @@ int pa_decode_ex(const void* q, int64_t q_stride, const void* k_pool, const void
   if (!a.err) return PA_ERR_CUDA;
   a.item_heads = item_heads;
   // shared prefixes read once for all their sharers (tensor-core kernel, and
-  // batches the plan can sort): items of 8 q columns for groups up to 4, of 16
-  // for groups up to 8 (room for two sharers at least)
+  // batches the plan can sort): items of 8 q columns, so groups up to 4 (two
+  // sharers at least), run in the same launch as the sequences' own items
   a.casc_cols = 0;
-  if (kind == PA_KERNEL_TCGEN05 && num_seqs >= 2 && num_seqs <= kCascMaxSeqs)
-    a.casc_cols = group <= 4 ? 8 : (group <= 8 ? 16 : 0);
+  if (kind == PA_KERNEL_TCGEN05 && num_seqs >= 2 && num_seqs <= kCascMaxSeqs && group <= 4)
+    a.casc_cols = 8;
 
   st = launch_decode_plan(a);
   if (st != PA_OK) return st;

@@ -21,7 +21,7 @@
 //    whether any repeats; the sort runs only then, and only if some candidate
 //    length keeps every item at most 1/kLocalityShare of one SM's share.
 //  * Shared-prefix cascade (tensor-core kernel, when the caller enables it
-//    with `casc_cols`, the q columns of one shared-prefix item, 8 or 16):
+//    with `casc_cols`, the q columns of one shared-prefix item):
 //    sequences sorted by first block form runs.  The longest run fixes the
 //    sharers per item M (at most casc_cols / G) and the KV heads per item HT
 //    (the most, up to 8, with G * HT * M <= casc_cols that divide the KV
@@ -31,8 +31,8 @@
 //    common (whole blocks inside every member's context).  A span of at least
 //    kMinCascSpan tokens becomes shared-prefix items (sub-run, KV-head group,
 //    partition) in a list of their own, read once for all members, with a
-//    partition length of their own (several items per SM: the sequences' own
-//    items start only when these are done); each member's own items then cover
+//    partition length of their own (several items per SM, so they end
+//    together); each member's own items then cover
 //    only its tokens after the span, and its partitions count the span's
 //    first.  header[4..7]: prefix items, their counter, log2 HT | M << 8,
 //    their partition length.
@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   __shared__ int sspan[kSortMax];                 // shared-prefix span per sequence (cascade)
   __shared__ int nruns;                           // sub-runs (cascade)
   __shared__ int rspan[kSortMax / 2];             // each sub-run's shared span (cascade)
+  __shared__ int roff[kSortMax / 2];              // each sub-run's first prefix item (cascade)
   __shared__ int rmax;                            // longest run of shared first blocks
   __shared__ int cand_pp[4];                      // prefix items at each candidate length
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -519,13 +520,26 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     const int cg = kv_heads >> hts;
     if (tid < nr) cnt = cg * ((rspan[tid] + pp_len - 1) / pp_len);
     const int incl = block_scan<false>(cnt, warp_tot);  // (nr <= 512 < 1024)
-    if (tid < nr) {
-      const int np = cnt / cg;
-      int at = incl - cnt;
-      for (int g = 0; g < cg; ++g)
-        for (int q = 0; q < np; ++q) pitems[at++] = make_int2(tid, (g << 16) | q);
+    if (tid < nr) roff[tid] = incl - cnt;
+    __shared__ int ptotal;
+    if (tid == 1023) {
+      header[4] = incl;  // shared-prefix items
+      ptotal = incl;
     }
-    if (tid == 1023) header[4] = incl;  // shared-prefix items
+    __syncthreads();
+    // item i: the sub-run whose first item is the last one <= i (binary
+    // search), then KV-head group and partition within it; consecutive
+    // threads write consecutive items
+    for (int i = tid; i < ptotal; i += 1024) {
+      int lo = 0, hi = nr - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (roff[mid] <= i) lo = mid; else hi = mid - 1;
+      }
+      const int np = (rspan[lo] + pp_len - 1) / pp_len;
+      const int o = i - roff[lo];
+      pitems[i] = make_int2(lo, ((o / np) << 16) | (o % np));
+    }
   }
   for (int i = tid; i < S * kv_heads; i += 1024) merge_cnt[i] = 0;
 }

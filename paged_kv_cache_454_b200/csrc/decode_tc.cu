@@ -42,20 +42,23 @@
 //               normalised result and its log-sum-exp to the epilogue through a
 //               shared-memory buffer and move on.
 //   warps 7-10  epilogue: write the output, or the partition's partial result;
-//               the last partition of a (sequence, head group) to finish merges
+//               the last partition of a (sequence, KV head) to finish merges
 //               all of them by log-sum-exp (one pass over the partitions).
-// Shared prefixes (cascade): sequences whose tables start with the same
-// blocks (parallel samples of one prompt) are grouped by the plan into
-// sub-runs of up to M sharers.  A first launch runs only the sub-runs'
-// shared-prefix items: the tile is read once and scored against the q heads of
-// every sharer.  The q columns of a tile are ordered (KV head of the item,
-// sharer, q head of the group): a row's columns -- those of its KV head -- are
-// then M * G contiguous ones, exactly as a group of M * G q heads, so the
-// same softmax serves both.  Each sharer gets its own partial result for the
-// prefix partition.  The second launch runs every
-// sequence's own items over the tokens after its shared span.  Partitions of
-// both launches are merged per (sequence, KV head) by whichever partition
-// finishes last.
+// Shared prefixes (cascade; groups up to 4): sequences whose tables start
+// with the same blocks (parallel samples of one prompt, "vLLM 基本原理",
+// PagedAttention / 内存共享) are grouped by the plan into sub-runs of up to M
+// sharers, and the span their tables have in common becomes shared-prefix
+// items, which the scheduler hands out before the sequences' own items (those
+// then cover only each sequence's tokens after its span).  A shared-prefix
+// tile is read once and scored against the q heads of every sharer: the q
+// columns are ordered (KV head of the item, sharer, q head of the group), so a
+// row's columns -- those of its KV head -- are M * G contiguous ones, exactly
+// as for a group of M * G q heads, and the same softmax serves both kinds.
+// The two kinds pack different numbers of KV heads per tile (the plan picks
+// the shared-prefix one), so each role keeps both tile geometries and takes
+// the one a tile's descriptor names.  Each sharer gets its own partial result
+// for a shared-prefix partition; all partitions of a (sequence, KV head) are
+// merged by whichever finishes last.
 // Tokens past the context (and pages with a bad block id) get p = 0 and their
 // V rows are zeroed before the second product, so NaN padding is never read
 // into a result.  Every wait is bounded and the softmax warps exchange data
@@ -103,9 +106,8 @@ struct Smem {
   // res_full, res_empty; epilogue exchange
   static constexpr int kNumBars = 2 * kStages + 14 + 2 * kDescSlots + 2 + 3;
   static constexpr int kOffRed = kOffBar + kNumBars * 8;
-  // tile max (x2), l sums (x2); for single-column rows (NH = 8 only) also
-  // alpha (x2) and the final max (x2)
-  static constexpr int kRedFloats = 2 * 4 * NH + 2 * 4 * NH + (NH <= 8 ? 4 * NH : 0);
+  // tile max (x2), l sums (x2)
+  static constexpr int kRedFloats = 2 * 4 * NH + 2 * 4 * NH;
   static constexpr int kOffMisc = kOffRed + kRedFloats * 4;
   static constexpr int kUsed = kOffMisc + 64;
   static constexpr int kBytes = kUsed + 1024;  // slack to align the base to 1024
@@ -117,8 +119,8 @@ constexpr int kThreads = 352;  // 11 warps
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, kN, false, false);
 
-// Tile descriptor flags.
-constexpr int kFirst = 1, kLast = 2, kEmpty = 4, kEnd = 8;
+// Tile descriptor flags (kPre: a tile of a shared-prefix item).
+constexpr int kFirst = 1, kLast = 2, kEmpty = 4, kEnd = 8, kPre = 16;
 
 struct TileDesc {
   int s, g, part, npart;         // g: KV-head group of the item
@@ -178,14 +180,12 @@ __device__ __forceinline__ void tmem_ld_o<16>(uint32_t taddr, float (&v)[32]) {
   tmem_ld32(taddr, v);
 }
 
-// NH: q columns per tile.  GR: q columns a tile row scores against -- NH (any
-// group; every row computes all columns, masked to its own KV head's) or 1 (one
-// q head per KV head: each row has exactly one column).  kCasc: the launch of
-// the shared-prefix items (GR == NH only).
-template <int NH, int GR, bool kCasc>
+// NH: q columns per tile (every row computes all of them, masked to its own
+// KV head's).  kCasc: the launch also runs the plan's shared-prefix items,
+// before the sequences' own items.
+template <int NH, bool kCasc>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ TcParams p) {
-  static_assert(GR == NH || (GR == 1 && NH <= 8), "row column modes");
-  static_assert(!kCasc || GR == NH, "shared-prefix items need every row's columns");
+  static_assert(!kCasc || NH == 8, "shared-prefix items use 8 q columns");
   using L = Smem<NH>;
   constexpr int kNpv = L::kNpv;
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, kNpv, true, false);
@@ -213,26 +213,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   uint64_t* ebar = res_empty + 1;   // epilogue warps' exchange barrier
   float* resbuf = reinterpret_cast<float*>(sptr + L::kOffRes);        // [NH][128]
   float* reslse = resbuf + NH * 128;                                  // [NH]
-  int* resmeta = reinterpret_cast<int*>(reslse + NH);                 // s, g, part, npart, pbase
+  int* resmeta = reinterpret_cast<int*>(reslse + NH);                 // s, g, part, npart, pbase, kind
   TileDesc* descs = reinterpret_cast<TileDesc*>(sptr + L::kOffDesc);
   float* red = reinterpret_cast<float*>(sptr + L::kOffRed);
   float* red_max = red;                // [2][4][NH]
   float* red_l = red + 2 * 4 * NH;     // [2][4][NH]
-  float* red_alpha = red_l + 2 * 4 * NH;  // [2][NH] (single-column rows)
-  float* red_mfin = red_alpha + 2 * NH;   // [2][NH] (single-column rows)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sptr + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + L::kOffMisc + 4);
   volatile int* merge_flag = reinterpret_cast<volatile int*>(sptr + L::kOffMisc + 8);  // [2]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  constexpr bool casc = kCasc;  // the shared-prefix launch
-  if (casc) {
-    // most batches share no prefix: leave before any set-up (the launch after
-    // this one starts as these CTAs exit)
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (p.header[4] == 0) return;
-  }
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -264,17 +255,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     prefetch_tmap(&p.tm_q);
   }
   if (warp == 1) tmem_alloc(tmem_slot, L::kTmemCols);
-  if (GR == 1 && warp >= 2 && warp <= 5) {
-    // Single-column rows: each row writes only its own column of P, so the rest
-    // of P stays zero for the whole kernel; a warp only writes the reduction
-    // slots of its own columns, so the others hold the identity.
-    for (int i = tid - 64; i < 2 * L::kPBytes / 16; i += 128) sts128_zero(sbase + L::kOffP + i * 16);
-    for (int i = tid - 64; i < 2 * 4 * NH; i += 128) {
-      red_max[i] = -CUDART_INF_F;
-      red_l[i] = 0.f;
-    }
-    fence_proxy_async_smem();
-  }
   fence_barrier_init();
   tc_fence_before();
   __syncthreads();
@@ -284,21 +264,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   // programmatic dependent launch): the set-up above overlaps it, and nothing
   // below reads the plan's results before the plan grid has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // KV heads per tile: fixed by the host, or chosen by the plan for shared prefixes
-  // (shared prefixes: sharers per item M in bits 8.. of the same word)
-  const int hword = casc ? p.header[6] : p.ht_shift;
-  const int hts = hword & 0xff;
-  const int ht = 1 << hts;            // KV heads per tile
-  const int pages = 8 >> hts;         // pages per tile
-  const int msh = casc ? hword >> 8 : 1;  // sharers per item (1: a sequence's own items)
-  const int cph = msh * p.group;      // q columns per KV head of an item
+  // Tile geometry of the two item kinds.  A sequence's own items pack 2^hts_o
+  // KV heads per tile (fixed by the host); shared-prefix items pack 2^hts_p
+  // KV heads and msh_p sharers (chosen by the plan: log2 HT | M << 8).  A tile
+  // holds 8 / HT pages; an item's q columns are cph = M G per KV head.
+  const int hts_o = p.ht_shift;
+  int hts_p = hts_o, msh_p = 1;
+  if (kCasc) {
+    const int hw = p.header[6];
+    hts_p = hw & 0xff;
+    msh_p = hw >> 8 > 0 ? hw >> 8 : 1;
+  }
+  const int cph_p = msh_p * p.group;
 
   if (warp == 6) {
     // =========================== scheduler ===========================
-    const int total = casc ? p.header[4] : p.header[0];
-    const int part = casc ? p.header[7] : p.header[3];
-    int* const counter = p.header + (casc ? 5 : 2);
+    // shared-prefix items first (their own list and counter), then the
+    // sequences' own items
+    const int ptotal = kCasc ? p.header[4] : 0;
+    const int ppart = kCasc ? p.header[7] : 0;
+    const int total = p.header[0];
+    const int part = p.header[3];
+    bool pre = ptotal > 0;
     uint32_t d = 0;
+    int pages = 8 >> hts_o;
     auto publish = [&](const TileDesc& td, int pbk) {
       const int slot = d % kDescSlots;
       mbar_wait(&desc_empty[slot], ((d / kDescSlots) & 1) ^ 1, abort_flag, p.err);
@@ -320,16 +309,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     };
     while (!*abort_flag) {
       int item = 0;
-      if (lane == 0) item = atomicAdd(counter, 1);
+      if (lane == 0) item = atomicAdd(p.header + (pre ? 5 : 2), 1);
       item = __shfl_sync(0xffffffffu, item, 0);
-      if (item >= total) break;
-      const int2 dd = casc ? p.pitems[item] : p.items[item];
+      if (pre && item >= ptotal) {
+        pre = false;
+        continue;
+      }
+      if (!pre && item >= total) break;
+      const int2 dd = pre ? p.pitems[item] : p.items[item];
       TileDesc td;
       td.s = dd.x;
       td.g = dd.y >> 16;
       const int q = dd.y & 0xffff;
       int tok0, srow;
-      if (casc) {
+      pages = 8 >> (pre ? hts_p : hts_o);
+      const int kind = pre ? kPre : 0;
+      if (pre) {
         // a sub-run (s = its index; npart = its members) over its shared span,
         // read through its first member's table
         const int* rr = p.runs + static_cast<int64_t>(td.s) * kRunInts;
@@ -338,8 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         srow = rr[2];
         td.part = q;
         td.pbase = 0;
-        tok0 = q * part;
-        td.tok1 = min(span, tok0 + part);
+        tok0 = q * ppart;
+        td.tok1 = min(span, tok0 + ppart);
       } else {
         // a sequence's own tokens, after its shared span (if any)
         int Lc = p.context_lens[td.s];
@@ -355,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const int npages = td.tok1 > tok0 ? (td.tok1 - tok0 + 15) / 16 : 0;
       if (npages == 0) {
         td.tok0 = tok0;
-        td.flags = kFirst | kLast | kEmpty;
+        td.flags = kFirst | kLast | kEmpty | kind;
         publish(td, -1);
         continue;
       }
@@ -373,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         for (int k = 0; k < 32 && p0 + k < npages; k += pages) {
           const int pbk = __shfl_sync(0xffffffffu, pb, (k + (lane & (pages - 1))) & 31);
           td.tok0 = tok0 + (p0 + k) * 16;
-          td.flags = (p0 + k == 0 ? kFirst : 0) | (p0 + k + pages >= npages ? kLast : 0);
+          td.flags = (p0 + k == 0 ? kFirst : 0) | (p0 + k + pages >= npages ? kLast : 0) | kind;
           publish(td, p0 + k + (lane & (pages - 1)) < npages ? pbk : -1);
         }
       }
@@ -392,9 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     // =========================== producer ===========================
     uint32_t d = 0, t = 0, nq = 0;
     const uint64_t pol = l2_policy_evict_first();
-    const uint32_t page_bytes = 4u * 2048u * static_cast<uint32_t>(ht);  // K and V, both halves
-    const CUtensorMap* tmk = casc ? &p.tm_kc[hts] : &p.tm_k;
-    const CUtensorMap* tmv = casc ? &p.tm_vc[hts] : &p.tm_v3;
+    const CUtensorMap* tmk_p = &p.tm_kc[hts_p];
+    const CUtensorMap* tmv_p = &p.tm_vc[hts_p];
     while (true) {
       const int slot = d % kDescSlots;
       mbar_wait(&desc_full[slot], (d / kDescSlots) & 1, abort_flag, p.err);
@@ -402,6 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const int flags = td->flags;
       if (flags & kEnd) break;
       if (!(flags & kEmpty)) {
+        const bool pre = kCasc && (flags & kPre);
+        const int hts = pre ? hts_p : hts_o;
+        const int ht = 1 << hts, pages = 8 >> hts;
+        const uint32_t page_bytes = 4u * 2048u * static_cast<uint32_t>(ht);  // K and V, both halves
         const int pb = lane < pages ? td->pb[lane] : -1;
         const int s = td->s, g = td->g;
         if (flags & kFirst) {
@@ -409,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           const int qs = nq & 1;
           mbar_wait(&q_empty[qs], ((nq >> 1) & 1) ^ 1, abort_flag, p.err);
           const uint32_t q0 = sbase + L::kOffQ + qs * kQBytes;
-          if (casc) {
+          if (pre) {
             // the sharers' q heads of the item's KV heads, column by column
             // (row h of the slot: KV head hh = h / cph of the item, sharer
             // m = h % cph / G, q head j = h % G of the group; rows of absent
@@ -422,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
               for (int j = 0; j < 16 * NH / 32; ++j) {
                 const int i = j * 32 + lane;
                 const int h = i >> 4, c = i & 15;  // q column, 16-byte chunk of the 256-byte row
-                const int hh = h / cph, w = h - hh * cph, m = w / p.group;
+                const int hh = h / cph_p, w = h - hh * cph_p, m = w / p.group;
                 const int sm = __shfl_sync(0xffffffffu, my_s, m & 31);
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
                 if (hh < ht && m < nsh)
@@ -455,10 +453,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             const int prow = (pb * p.hkv + (g << hts)) * 16;
             const uint32_t kdst = stage + lane * (ht * 2048);
             const uint32_t vdst = stage + kKBytes + lane * (ht * 4096);
+            const CUtensorMap* tmk = pre ? tmk_p : &p.tm_k;
             tma_load_2d_hint(kdst, tmk, 0, prow, &full[st], pol);
             tma_load_2d_hint(kdst + kRegion, tmk, 64, prow, &full[st], pol);
-            if (ht < 8 || casc) {
-              tma_load_3d_hint(vdst, tmv, 0, prow, 0, &full[st], pol);  // both halves
+            if (ht < 8 || pre) {
+              tma_load_3d_hint(vdst, pre ? tmv_p : &p.tm_v3, 0, prow, 0, &full[st], pol);  // both halves
             } else {
               // a 128-row page: two 16 KiB copies ran faster than one of 32 KiB
               tma_load_2d_hint(vdst, &p.tm_v, 0, prow, &full[st], pol);
@@ -493,11 +492,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       // a product then costs only constant adds (the single issuing thread is
       // otherwise bound by its own address arithmetic).
       const uint64_t desc_k0 = smem_desc_sw128(sbase, 16, 1024);
-      const uint64_t desc_v0 = smem_desc_sw128(sbase + kKBytes, ht * 2048, 1024);
-      // rows 16k.. of the V tile: page k >> hts, its (k & (ht-1))-th 16 rows
-      uint32_t voff[kRows / 16];
+      // V of a tile of HT heads: its two 64-dim halves HT * 2 KiB apart; rows
+      // 16k.. are page k >> log2 HT, its (k & (HT - 1))-th 16 rows (own items
+      // and shared-prefix items each have their HT)
+      const uint64_t desc_v0_o = smem_desc_sw128(sbase + kKBytes, (1 << hts_o) * 2048, 1024);
+      const uint64_t desc_v0_p = smem_desc_sw128(sbase + kKBytes, (1 << hts_p) * 2048, 1024);
+      uint32_t voff_o[kRows / 16], voff_p[kRows / 16];
 #pragma unroll
-      for (int k = 0; k < kRows / 16; ++k) voff[k] = 2048u * (k + ((k >> hts) << hts));
+      for (int k = 0; k < kRows / 16; ++k) {
+        voff_o[k] = 2048u * (k + ((k >> hts_o) << hts_o));
+        voff_p[k] = 2048u * (k + ((k >> hts_p) << hts_p));
+      }
+      uint32_t pre_tiles = 0;  // bit t % 32: tile t is a shared-prefix tile
       const uint64_t desc_q0 = smem_desc_sw128(sbase + L::kOffQ, 16, 1024);
       const uint64_t desc_p0 = smem_desc_sw128(sbase + L::kOffP, 16, 1024);
       uint32_t d = 0, ts = 0, tpv = 0, mq = 0;  // ts: next S tile; tpv: next O tile
@@ -512,12 +518,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           if (mbar_test_wait(&p_full[b], bph) && mbar_test_wait(&o_free[b], bph ^ 1)) {
             tc_fence_after();
             const int st = tpv % kStages;
-            const uint64_t a0 = desc_add(desc_v0, st * kStageBytes);
+            const bool pt = kCasc && ((pre_tiles >> (tpv & 31)) & 1u);
+            const uint64_t a0 = desc_add(pt ? desc_v0_p : desc_v0_o, st * kStageBytes);
             const uint64_t b0 = desc_add(desc_p0, b * L::kPBytes);
             const uint32_t dt = tmem + 2 * kN + b * kNpv;
-            // A = V^T (MN-major): 16 rows = 2 groups of 8; D halves ht*2 KiB apart
+            // A = V^T (MN-major): 16 rows = 2 groups of 8; D halves HT*2 KiB apart
             // B = P (K-major, kNpv rows = q columns): row half k/4, 32 bytes per 16 rows
-            if (ht == 8) {  // one page: slices 2 KiB apart (constant offsets)
+            if (!kCasc && hts_o == 3) {  // one page: slices 2 KiB apart (constant offsets)
 #pragma unroll
               for (int k = 0; k < kRows / 16; ++k)
                 umma_ss(dt, desc_add(a0, k * 2048),
@@ -526,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             } else {
 #pragma unroll
               for (int k = 0; k < kRows / 16; ++k)
-                umma_ss(dt, desc_add(a0, voff[k]),
+                umma_ss(dt, desc_add(a0, pt ? voff_p[k] : voff_o[k]),
                         desc_add(b0, (k >> 2) * (kNpv * 128) + (k & 3) * 32), kIdescO,
                         k > 0 ? 1u : 0u);
             }
@@ -566,6 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
               umma_ss(dt, desc_add(a0, (k >> 2) * kRegion + (k & 3) * 32),
                       desc_add(b0, (k >> 2) * kQRegion + (k & 3) * 32), kIdescS, k > 0 ? 1u : 0u);
             umma_commit(&s_full[b]);
+            if (kCasc) pre_tiles = (flags & kPre) ? (pre_tiles | (1u << (ts & 31))) : (pre_tiles & ~(1u << (ts & 31)));
             if (flags & kLast) {
               umma_commit(&q_empty[qs]);
               ++mq;
@@ -599,20 +607,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       ++ek;
     };
     // Column h of an item: KV head h / cph of the item, sharer (h % cph) / G,
-    // q head (h / cph) * G + h % G among the item's q heads of that sequence.
-    auto sharer_cols = [&](int m) {  // the columns of sharer m
-      uint32_t mm = 0;
-      for (int hh = 0; hh < ht; ++hh) mm |= ((1u << p.group) - 1u) << (hh * cph + m * p.group);
-      return mm & ((1u << NH) - 1u);
-    };
-    // q head of column h among the item's q heads of its sequence
-    auto col_qhead = [&](int h) { return casc ? (h / cph) * p.group + h % p.group : h; };
+    // q head (h / cph) * G + h % G among the item's q heads of that sequence
+    // (an own item: one sequence, cph = G, so q head h).
     while (!*abort_flag) {
       mbar_wait(res_full, k & 1, abort_flag, p.err);
       const int npart = resmeta[3];  // shared-prefix items: the sharers
       if (npart < 0 || *abort_flag) break;
       const int s = resmeta[0], g = resmeta[1], part = resmeta[2], pbase = resmeta[4];
-      const int nsh = casc ? npart : 1;  // sequences of the item
+      const bool pre = kCasc && resmeta[5];
+      const int hts = pre ? hts_p : hts_o, ht = 1 << hts;
+      const int msh = pre ? msh_p : 1, cph = pre ? cph_p : p.group;
+      auto sharer_cols = [&](int m) {  // the columns of sharer m
+        uint32_t mm = 0;
+        for (int hh = 0; hh < ht; ++hh) mm |= ((1u << p.group) - 1u) << (hh * cph + m * p.group);
+        return mm & ((1u << NH) - 1u);
+      };
+      auto col_qhead = [&](int h) { return pre ? (h / cph) * p.group + h % p.group : h; };
+      const int nsh = pre ? npart : 1;  // sequences of the item
       float res[NH], l2[NH];
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
@@ -625,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       // lane m of every epilogue warp holds sequence m of the item: its index,
       // first partition record and partition count
       int my_s = s, my_pb = pbase, my_np = npart;
-      if (casc) {
+      if (pre) {
         my_s = lane < nsh ? p.runs[static_cast<int64_t>(s) * kRunInts + 2 + lane] : 0;
         my_pb = lane < nsh ? p.part_base[my_s] : 0;
         my_np = lane < nsh ? p.part_base[my_s + 1] - my_pb : 1;
@@ -636,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         const int sm = __shfl_sync(0xffffffffu, my_s, m);
         const int pbm = __shfl_sync(0xffffffffu, my_pb, m);
         const int npm = __shfl_sync(0xffffffffu, my_np, m);
-        const uint32_t mm = casc ? sharer_cols(m) : (1u << (ht * p.group)) - 1u;
+        const uint32_t mm = pre ? sharer_cols(m) : (1u << (ht * p.group)) - 1u;
         any_multi |= npm > 1;
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
@@ -685,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         const int sm = __shfl_sync(0xffffffffu, my_s, m);
         const int pbm = __shfl_sync(0xffffffffu, my_pb, m);
         const int npm = __shfl_sync(0xffffffffu, my_np, m);
-        const uint32_t mc = casc ? colsel & sharer_cols(m) : colsel;
+        const uint32_t mc = pre ? colsel & sharer_cols(m) : colsel;
         if (!mc) continue;
         float M[NH], W[NH], A[NH];
 #pragma unroll
@@ -735,174 +746,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
       }
     }
-  } else if (GR == 1) {
-    // ===================== softmax, one column per row =====================
-    // Rows 16h..16h+15 of a page belong to KV head h of the tile, whose single
-    // q head is column h.  Lanes 0-15 and 16-31 of a warp hold one head each
-    // (the same head when the tile holds one KV head).
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;
-    const int wi = warp - 2;
-    const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-    const int pj = r >> (4 + hts);
-    // row r of the V tile: page pj holds its rows for dims 0-63, then 64-127
-    const uint32_t v_row_off = pj * (ht * 4096) + (r & ((16 << hts) - 1)) * 128;
-    const int col = (r >> 4) & (ht - 1);          // this row's q column
-    const int col0 = (2 * q4) & (ht - 1);         // column of lanes 0-15 (S load base)
-    const bool upper = ht > 1 && lane >= 16;      // lanes 16-31 hold column col0 + 1
-    const bool col_writer = lane == 0 || (upper && lane == 16);  // one lane per (warp, column)
-    const int rtok = (pj << 4) | (r & 15);
-    uint32_t d = 0, t = 0, xk = 0, nfin = 0;
-    auto exchange = [&]() {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xbar);
-      mbar_wait(xbar, xk & 1, abort_flag, p.err);
-      ++xk;
-    };
-    float m_run = -CUDART_INF_F, l_part = 0.f;
-    float acc[NH];
-#pragma unroll
-    for (int h = 0; h < NH; ++h) acc[h] = 0.f;
-    // O of tile u into acc; alpha of tile u comes from its column's owners
-    // (written before the exchange of tile u + 1, which every caller has passed)
-    auto fold = [&](uint32_t u) {
-      const int b = u & 1;
-      mbar_wait(&o_full[b], (u >> 1) & 1, abort_flag, p.err);
-      tc_fence_after();
-      float ov[2 * NH];
-      tmem_ld_o<NH>(tmem + lane_addr + 2 * kN + b * kNpv, ov);
-      tc_fence_before();
-      mbar_arrive(&o_free[b]);
-      const float* al = red_alpha + b * NH;
-#pragma unroll
-      for (int h = 0; h < NH; ++h) acc[h] = acc[h] * al[h] + ov[h] + ov[NH + h];
-    };
-    while (true) {
-      const int slot = d % kDescSlots;
-      mbar_wait(&desc_full[slot], (d / kDescSlots) & 1, abort_flag, p.err);
-      const TileDesc* td = descs + slot;
-      const int flags = td->flags;
-      if ((flags & kEnd) || *abort_flag) {
-        mbar_wait(res_empty, (nfin & 1) ^ 1, abort_flag, p.err);
-        if (r == 0) resmeta[3] = -1;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(res_full);
-        break;
-      }
-      const int s = td->s, g = td->g, part = td->part, npart = td->npart, pbase = td->pbase;
-      const int tok0 = td->tok0, tok1 = td->tok1;
-      const int mypb = td->pb[pj];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&desc_empty[slot]);
-      ++d;
-      if (flags & kFirst) {
-        m_run = -CUDART_INF_F;
-        l_part = 0.f;
-#pragma unroll
-        for (int h = 0; h < NH; ++h) acc[h] = 0.f;
-      }
-      if (!(flags & kEmpty)) {
-        const int st = t % kStages;
-        const int b = t & 1;
-        mbar_wait(&s_full[b], (t >> 1) & 1, abort_flag, p.err);
-        tc_fence_after();
-        float sv[2];
-        tmem_ld2(tmem + lane_addr + b * kN + col0, sv);
-        tc_fence_before();
-        mbar_arrive(&s_free[b]);
-        const bool valid = tok0 + rtok < tok1 && mypb >= 0;
-        const float x = valid ? (upper ? sv[1] : sv[0]) * p.scale_log2 : -CUDART_INF_F;
-        // max over this warp's rows of the column, then over the warps
-        float v = x;
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (ht == 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-        float* rm = red_max + (t & 1) * 4 * NH;
-        if (col_writer) rm[wi * NH + col] = v;
-        exchange();
-        const float tmax =
-            fmaxf(fmaxf(rm[col], rm[NH + col]), fmaxf(rm[2 * NH + col], rm[3 * NH + col]));
-        const float mn = fmaxf(m_run, tmax);
-        const float alpha = (mn == -CUDART_INF_F) ? 1.f : exp2f(m_run - mn);
-        const float pr = (x == -CUDART_INF_F) ? 0.f : exp2f(x - mn);
-        l_part = l_part * alpha + pr;
-        m_run = mn;
-        if (col_writer) red_alpha[b * NH + col] = alpha;
-        // p into P[b] at row col (and its bf16 remainder at row NH + col), column r
-        const uint32_t pbuf = sbase + L::kOffP + b * L::kPBytes + (r >> 6) * (kNpv * 128);
-        const int c = r & 63;
-        const uint16_t hi = f32_to_bf16_bits(pr);
-        const float rem = pr - __uint_as_float(static_cast<uint32_t>(hi) << 16);
-        sts16(pbuf + swz(col, c >> 3) + (c & 7) * 2, hi);
-        sts16(pbuf + swz(NH + col, c >> 3) + (c & 7) * 2, f32_to_bf16_bits(rem));
-        if (!valid) {
-          const uint32_t vrow = sbase + st * kStageBytes + kKBytes + v_row_off;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            sts128_zero(vrow + k * 16);
-            sts128_zero(vrow + ht * 2048 + k * 16);
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&p_full[b]);
-        if (!(flags & kFirst)) fold(t - 1);
-        ++t;
-      }
-      if (!(flags & kLast)) continue;
-      // the exchange below orders the last tile's alpha before its fold
-      float* rl = red_l + (nfin & 1) * 4 * NH;
-      float* mf = red_mfin + (nfin & 1) * NH;
-      {
-        float v = l_part;
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (ht == 1) v += __shfl_xor_sync(0xffffffffu, v, 16);
-        if (col_writer) {
-          rl[wi * NH + col] = v;
-          mf[col] = m_run;
-        }
-      }
-      exchange();
-      if (!(flags & kEmpty)) fold(t - 1);
-      float res[NH], lse2[NH];
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        const float l = rl[h] + rl[NH + h] + rl[2 * NH + h] + rl[3 * NH + h];
-        const float m = mf[h];
-        const bool live = m != -CUDART_INF_F && l > 0.f;
-        res[h] = live ? acc[h] / l : 0.f;
-        lse2[h] = live ? m + log2f(l) : -CUDART_INF_F;
-      }
-      mbar_wait(res_empty, (nfin & 1) ^ 1, abort_flag, p.err);
-#pragma unroll
-      for (int h = 0; h < NH; ++h) resbuf[h * 128 + r] = res[h];
-      if (r == 0) {
-#pragma unroll
-        for (int h = 0; h < NH; ++h) reslse[h] = lse2[h];
-        resmeta[0] = s;
-        resmeta[1] = g;
-        resmeta[2] = part;
-        resmeta[3] = npart;
-        resmeta[4] = pbase;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(res_full);
-      ++nfin;
-    }
   } else {
     // ============================ softmax =============================
     const int q4 = warp & 3;          // TMEM lane quadrant of this warp
     const int r = q4 * 32 + lane;     // tile row of S^T, output dim of O^T
     const int wi = warp - 2;          // index among the softmax warps
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-    // tile row r: page j, KV head hh of the tile, token j * 16 + r % 16
-    const int pj = r >> (4 + hts);
-    // row r of the V tile: page pj holds its rows for dims 0-63, then 64-127
-    const uint32_t v_row_off = pj * (ht * 4096) + (r & ((16 << hts) - 1)) * 128;
-    // this row's q columns start at its KV head's block of cph columns; an
-    // item with k sharers uses the first k * G of them
-    const int c_row = ((r >> 4) & (ht - 1)) * cph;
-    const int rtok = (pj << 4) | (r & 15);
+    // Tile row r, for either item kind (own: _o, shared prefix: _p): page pj,
+    // KV head (r >> 4) & (HT - 1) of the tile, token pj * 16 + r % 16.  Row r
+    // of the V tile: page pj holds its rows for dims 0-63, then 64-127.  The
+    // row's q columns start at its KV head's block of cph columns (an item
+    // with k sharers uses the first k G of them).
+    const int pj_o = r >> (4 + hts_o), pj_p = r >> (4 + hts_p);
+    const uint32_t vro_o = pj_o * ((1 << hts_o) * 4096) + (r & ((16 << hts_o) - 1)) * 128;
+    const uint32_t vro_p = pj_p * ((1 << hts_p) * 4096) + (r & ((16 << hts_p) - 1)) * 128;
+    const int crow_o = ((r >> 4) & ((1 << hts_o) - 1)) * p.group;
+    const int crow_p = ((r >> 4) & ((1 << hts_p) - 1)) * cph_p;
+    const int rtok_o = (pj_o << 4) | (r & 15), rtok_p = (pj_p << 4) | (r & 15);
     uint32_t d = 0, t = 0, xk = 0, nfin = 0;
     // all four softmax warps have passed this point (bounded, unlike bar.sync)
     auto exchange = [&]() {
@@ -945,6 +805,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       }
       const int s = td->s, g = td->g, part = td->part, npart = td->npart, pbase = td->pbase;
       const int tok0 = td->tok0, tok1 = td->tok1;
+      const bool pre = kCasc && (flags & kPre);
+      const int pj = pre ? pj_p : pj_o;
       const int mypb = td->pb[pj];
       __syncwarp();
       if (lane == 0) mbar_arrive(&desc_empty[slot]);
@@ -967,9 +829,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         tmem_ld16(tmem + lane_addr + b * kN, sv);
         tc_fence_before();
         mbar_arrive(&s_free[b]);
-        const bool valid = tok0 + rtok < tok1 && mypb >= 0;
+        const bool valid = tok0 + (pre ? rtok_p : rtok_o) < tok1 && mypb >= 0;
         // the row's columns: its KV head's G q heads for each of the item's sharers
-        const uint32_t cm = ((1u << ((casc ? npart : 1) * p.group)) - 1u) << c_row;
+        const uint32_t cm = ((1u << ((pre ? npart : 1) * p.group)) - 1u) << (pre ? crow_p : crow_o);
         float x[NH];
 #pragma unroll
         for (int h = 0; h < NH; ++h)
@@ -1008,11 +870,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         if (!valid) {
           // zero this row of V (both 64-dim halves) so padding never reaches O
-          const uint32_t vrow = sbase + st * kStageBytes + kKBytes + v_row_off;
+          const uint32_t vrow = sbase + st * kStageBytes + kKBytes + (pre ? vro_p : vro_o);
+          const uint32_t vhalf = (1u << (pre ? hts_p : hts_o)) * 2048u;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             sts128_zero(vrow + k * 16);
-            sts128_zero(vrow + ht * 2048 + k * 16);
+            sts128_zero(vrow + vhalf + k * 16);
           }
         }
         fence_proxy_async_smem();
@@ -1055,6 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         resmeta[2] = part;
         resmeta[3] = npart;
         resmeta[4] = pbase;
+        resmeta[5] = pre ? 1 : 0;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(res_full);
@@ -1073,9 +937,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int NH, int GR, bool kCasc = false>
+template <int NH, bool kCasc = false>
 int launch_nh(const TcParams& prm, int64_t item_bound, cudaStream_t stream) {
-  auto kern = decode_tc_kernel<NH, GR, kCasc>;
+  auto kern = decode_tc_kernel<NH, kCasc>;
   static KernelLaunchCache cache;
   const int per_sm =
       cache.blocks_per_sm(reinterpret_cast<const void*>(kern), kThreads, Smem<NH>::kBytes);
@@ -1157,7 +1021,7 @@ int launch_decode_tcgen05(const DecodeArgs& a) {
     const uint32_t box[3] = {64, 16, 1};
     if (!encode_bf16_map(&p.tm_q, a.q, 3, dims, strides, box)) return PA_ERR_CUDA;
   }
-  const bool casc = a.casc_cols == 8 || a.casc_cols == 16;
+  const bool casc = a.casc_cols == 8;
   if (casc) {
     // shared-prefix launch: the plan picks 1, 2, 4 or 8 KV heads per tile
     for (int h = 0; h < 4; ++h) {
@@ -1198,17 +1062,13 @@ int launch_decode_tcgen05(const DecodeArgs& a) {
   p.ngroups = a.pool.num_kv_heads >> sh.ht_shift;
   p.nq = group << sh.ht_shift;
   p.scale_log2 = a.scale * kLog2e;
-  if (casc) {
-    // the shared-prefix items first (none unless the plan found shared prefixes)
-    const int64_t pbound = static_cast<int64_t>(a.num_seqs / 2 + 1) * a.max_parts * a.pool.num_kv_heads;
-    const int st = a.casc_cols == 8 ? launch_nh<8, 8, true>(p, pbound, a.stream)
-                                     : launch_nh<16, 16, true>(p, pbound, a.stream);
-    if (st != PA_OK) return st;
-  }
-  const int64_t bound = static_cast<int64_t>(a.num_seqs) * (a.max_parts + 1) * p.ngroups;
-  if (group == 1) return launch_nh<8, 1>(p, bound, a.stream);
-  if (sh.nh == 8) return launch_nh<8, 8>(p, bound, a.stream);
-  return launch_nh<16, 16>(p, bound, a.stream);
+  const int64_t bound = static_cast<int64_t>(a.num_seqs) * (a.max_parts + 1) * p.ngroups +
+                        (casc ? static_cast<int64_t>(a.num_seqs / 2 + 1) * a.max_parts * a.pool.num_kv_heads : 0);
+  // one launch: the shared-prefix items (none unless the plan found shared
+  // prefixes) and then the sequences' own items
+  if (casc) return launch_nh<8, true>(p, bound, a.stream);
+  if (sh.nh == 8) return launch_nh<8>(p, bound, a.stream);
+  return launch_nh<16>(p, bound, a.stream);
 }
 
 }  // namespace pa

@@ -118,9 +118,9 @@ struct DecodeArgs {
   int max_parts;     // workspace bound (partitions of the longest context at min_part)
   int item_heads = 1;  // KV heads per work item (the tensor-core kernel packs small groups)
   // Shared-prefix cascade (tensor-core kernel): sequences that share their
-  // first blocks read the shared span once, in items whose casc_cols (8 or 16)
-  // q columns are the sharers' q heads (the plan picks the sharers and KV
-  // heads per item).  0: no cascade.
+  // first blocks read the shared span once, in items whose casc_cols q columns
+  // are the sharers' q heads (the plan picks the sharers and KV heads per
+  // item).  0: no cascade.
   int casc_cols = 0;
   DecodeWorkspace ws;
   unsigned int* err;

@@ -21,6 +21,8 @@
 //   NaN logits are never drawn (their key is the smallest).
 #include <cstdint>
 
+#include <math_constants.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "../../include/pa_sampler.h"
@@ -35,7 +37,8 @@ constexpr int kFastK = 1024;  // Top-K values the small-K path takes
 
 __device__ __forceinline__ uint32_t key_of(float x) {
   if (x != x) return 0u;  // NaN: below everything
-  const uint32_t b = __float_as_uint(x);
+  uint32_t b = __float_as_uint(x);
+  if ((b << 1) == 0u) b = 0u;  // -0 is the same logit as +0
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
@@ -264,57 +267,81 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
   float u = uniform[row];
   u = (u >= 0.f && u < 1.f) ? u : 0.f;
 
-  // ---- pass 1: the largest key, lowest index among equals; each thread also
-  // keeps its four best elements (key descending, index ascending), which
-  // usually hold every Top-K candidate it has ----
-  constexpr int kNone = 0x7fffffff;  // index of an empty slot
-  uint32_t k0 = 0, k1 = 0, k2 = 0, k3 = 0;
-  int i0 = kNone, i1 = kNone, i2 = kNone, i3 = kNone;
-  // indices arrive in increasing order, so an equal key ranks below a kept
-  // one unless that slot is empty: an element enters the four when its key
-  // beats the fourth's or the fourth slot is empty
-  auto insert = [&](uint32_t k, int i) {
-    if (k > k3 || i3 == kNone) {
-      if (k > k2 || (k == k2 && i < i2)) {
-        k3 = k2;
-        i3 = i2;
-        if (k > k1 || (k == k1 && i < i1)) {
-          k2 = k1;
-          i2 = i1;
-          if (k > k0 || (k == k0 && i < i0)) {
-            k1 = k0;
-            i1 = i0;
-            k0 = k;
-            i0 = i;
+  // ---- pass 1: each thread's four largest groups -- a group is a 16-byte
+  // vector of four logits, or a single logit where the row is not 16-byte
+  // aligned and in its tail -- by their largest value, the first group among
+  // equal ones.  The common case (a vector below the fourth kept one) costs
+  // three maxima and a compare. ----
+  constexpr int kNone = 0x7fffffff;  // group index of an empty slot
+  const int V4 = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 ? (V >> 2) : 0;  // vector elements: [0, 4 V4)
+  float g0 = -CUDART_INF_F, g1 = -CUDART_INF_F, g2 = -CUDART_INF_F, g3 = -CUDART_INF_F;
+  int b0 = kNone, b1 = kNone, b2 = kNone, b3 = kNone;
+  // groups arrive in increasing index order, so `>` keeps the first of equals;
+  // NaN and -inf maxima never enter
+  auto add_group = [&](float m, int b) {
+    if (m > g3) {
+      if (m > g2) {
+        g3 = g2;
+        b3 = b2;
+        if (m > g1) {
+          g2 = g1;
+          b2 = b1;
+          if (m > g0) {
+            g1 = g0;
+            b1 = b0;
+            g0 = m;
+            b0 = b;
           } else {
-            k1 = k;
-            i1 = i;
+            g1 = m;
+            b1 = b;
           }
         } else {
-          k2 = k;
-          i2 = i;
+          g2 = m;
+          b2 = b;
         }
       } else {
-        k3 = k;
-        i3 = i;
+        g3 = m;
+        b3 = b;
       }
     }
   };
-  // the common case -- none of a vector's four elements enters -- costs one
-  // compare against the fourth kept key
-  auto take4 = [&](float4 a, int b) {
-    const uint32_t ka = key_of(a.x), kb = key_of(a.y), kc = key_of(a.z), kd = key_of(a.w);
-    if (__builtin_expect(max(max(ka, kb), max(kc, kd)) > k3 || i3 == kNone, 0)) {
-      insert(ka, b);
-      insert(kb, b + 1);
-      insert(kc, b + 2);
-      insert(kd, b + 3);
+  for_each_logit4(
+      x, V, [&](float4 a, int b) { add_group(fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)), b); },
+      [&](float v, int i) { add_group(v, i); });
+  // the elements of group b (4 or 1) into v; returns how many
+  auto load_group = [&](int b, float (&v)[4]) {
+    if (b < 4 * V4) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(x) + (b >> 2));
+      v[0] = a.x;
+      v[1] = a.y;
+      v[2] = a.z;
+      v[3] = a.w;
+      return 4;
     }
+    v[0] = x[b];
+    return 1;
   };
-  auto take1 = [&](float v, int i) { insert(key_of(v), i); };
-  for_each_logit4(x, V, take4, take1);
-  uint32_t bk = k0;
-  int bi = i0;
+  // this thread's largest logit: the first element of its first largest group
+  // equal to that group's maximum
+  uint32_t bk = 0;
+  int bi = kNone;
+  if (b0 != kNone) {
+    float v[4];
+    const int w = load_group(b0, v);
+#pragma unroll
+    for (int j = 3; j >= 0; --j)
+      if (j < w && v[j] == g0) bi = b0 + j;
+    bk = key_of(g0);
+  } else {
+    // every element of this thread is -inf or NaN (or it has none)
+    for_each_logit(x, V, [&](float v, int i) {
+      const uint32_t k = key_of(v);
+      if (k > bk || (k == bk && i < bi)) {
+        bk = k;
+        bi = i;
+      }
+    });
+  }
   sm.tmax[tid] = bk;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -377,20 +404,28 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
     auto pack = [](uint32_t k, int i) {
       return (static_cast<uint64_t>(k) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
     };
-    // Every element at or above t0 is among its thread's four kept ones unless
-    // the fourth is too (the thread may have more): then the row is read again.
-    if (i3 != kNone && k3 >= t0) sm.overflow = 1;
-    {
-      const int c = (i0 != kNone && k0 >= t0) + (i1 != kNone && k1 >= t0) +
-                    (i2 != kNone && k2 >= t0) + (i3 != kNone && k3 >= t0);
-      if (c) {
-        int pos = atomicAdd(&sm.count, c);
-        if (pos < kCand) sm.cand[pos] = pack(k0, i0);
-        if (c > 1 && ++pos < kCand) sm.cand[pos] = pack(k1, i1);
-        if (c > 2 && ++pos < kCand) sm.cand[pos] = pack(k2, i2);
-        if (c > 3 && ++pos < kCand) sm.cand[pos] = pack(k3, i3);
+    // Every element at or above t0 lies in a group whose maximum is, so in one
+    // of its thread's four kept groups -- unless the fourth is at or above t0
+    // too (a fifth may be) or t0 admits -inf or NaN logits, which no group
+    // maximum tracks: then the row is read again.
+    if ((b3 != kNone && key_of(g3) >= t0) || t0 <= key_of(-CUDART_INF_F)) sm.overflow = 1;
+    auto gather = [&](float gm, int gb) {
+      if (gb == kNone || key_of(gm) < t0) return;
+      float v[4];
+      const int w = load_group(gb, v);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t k = j < w ? key_of(v[j]) : 0u;
+        if (j < w && k >= t0) {
+          const int pos = atomicAdd(&sm.count, 1);
+          if (pos < kCand) sm.cand[pos] = pack(k, gb + j);
+        }
       }
-    }
+    };
+    gather(g0, b0);
+    gather(g1, b1);
+    gather(g2, b2);
+    gather(g3, b3);
     __syncthreads();
     if (sm.overflow) {
       __syncthreads();

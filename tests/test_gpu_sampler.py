@@ -90,10 +90,18 @@ def test_edges_greedy_ties_nan_and_neg_inf():
     x = np.array([[1.0, 3.0, 3.0, 2.0],          # greedy tie -> index 1
                   [np.nan, 1.0, np.nan, 0.5],    # NaN never drawn
                   [-np.inf, -np.inf, 0.0, -np.inf],
-                  [5.0, 5.0, 1.0, 1.0]], np.float32)
-    got = run(x, [0.0, 1.0, 1.0, 1.0], [0, 0, 0, 1], [1.0, 1.0, 1.0, 1.0], [0.9, 0.5, 0.5, 0.75])
+                  [5.0, 5.0, 1.0, 1.0],
+                  [-0.0, 0.0, -1.0, -2.0],       # -0 and +0 are equal logits: greedy -> 0
+                  [-1.0, 0.0, -0.0, -3.0]],      # top-k 1 keeps both zeros; u = 0.75 -> 2
+                 np.float32)
+    got = run(x, [0.0, 1.0, 1.0, 1.0, 0.0, 1.0], [0, 0, 0, 1, 0, 1], [1.0] * 6,
+              [0.9, 0.5, 0.5, 0.75, 0.5, 0.75])
     assert got.tolist()[:3] == [1, 1, 2]
     assert got[3] == 1   # top-k 1 keeps both tied maxima; u = 0.75 draws the second
+    assert got[4] == 0 and got[5] == 2
+    for r in (4, 5):
+        assert sampler.sample(x[r].astype(np.float64), [0.0, 1.0][r - 4], [0, 1][r - 4], 1.0,
+                              0.5 if r == 4 else 0.75) == got[r]
 
 
 @pytest.mark.parametrize("vocab", [4096, 152064])
