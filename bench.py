@@ -319,9 +319,9 @@ def host_manager_timing(w: Workload, steps: int = 100):
 def sampler_timing(w: Workload, stream, reps: int = 50):
     """Device time of the fused sampler (``pa_sample``) for this batch's decode
     rows at two vocabulary sizes (32000, 152064), temperature 0.7, top-k 50,
-    top-p 0.9; CUDA events over ``reps`` back-to-back calls after warm-up.
-    Consecutive calls read different logit buffers whose total is over twice
-    the L2, so every call streams its logits from HBM."""
+    top-p 0.9; CUDA events around ``reps`` calls replayed from a CUDA graph
+    after warm-up.  Consecutive calls read different logit buffers whose total
+    is over twice the L2, so every call streams its logits from HBM."""
     torch = w.torch
     rows = len(w.dec) if len(w.dec) else 1
     res = {}
@@ -338,17 +338,27 @@ def sampler_timing(w: Workload, stream, reps: int = 50):
         with torch.cuda.stream(stream):
             for i in range(max(5, nbuf)):
                 w.pa.pa_sample(xs[i % nbuf], T, K, P, u, out=out, stream=stream)
+        torch.cuda.synchronize()
+        # the calls replayed from a CUDA graph, so the host's per-call binding
+        # overhead does not leave the GPU idle between them
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(reps):
+                w.pa.pa_sample(xs[i % nbuf], T, K, P, u, out=out,
+                               stream=torch.cuda.current_stream())
+        with torch.cuda.stream(stream):
+            graph.replay()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for i in range(reps):
-                w.pa.pa_sample(xs[i % nbuf], T, K, P, u, out=out, stream=stream)
+            graph.replay()
             e1.record(stream)
         torch.cuda.synchronize()
         res[str(vocab)] = round(e0.elapsed_time(e1) / reps * 1e3, 2)
-        del xs
+        del graph, xs
     return {"us_per_call": res, "rows": rows, "temperature": 0.7, "top_k": 50, "top_p": 0.9,
             "l2": "rotating logit buffers, over twice the L2 in total",
+            "launch": "calls replayed from a CUDA graph",
             "logits_gb_per_s": {k: round(rows * int(k) * 4 / (v * 1e-6) / 1e9, 1)
                                 for k, v in res.items()}}
 
@@ -695,7 +705,7 @@ def main():
         b = w.bytes_dec
         algo = b["unique"]
         achieved = algo / (comp["decode"] * 1e-3) / 1e9
-        roof = {"bound": "hbm", "kernel": "pa_decode (plan + decode + merge launches)",
+        roof = {"bound": "hbm", "kernel": "pa_decode (plan and decode launches)",
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": f"{peak_src} hbm_gbs",
@@ -749,16 +759,14 @@ def main():
 
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # decode kernel from an ncu capture, keyed by workload and the kernel sources
-# it was taken with (reported as null once those sources change).  The
-# gqa70b_long figure is the 48-sequence capture (1,760,201,728 bytes for
-# 1,755,018,024 algorithmic bytes) scaled by algorithmic bytes to the full
-# 128-sequence batch; the captures are summarised in profiles/.
+# it was taken with (reported as null once those sources change).  Both are
+# captures of a smaller batch of the same shape, scaled to the full batch by
+# algorithmic bytes: gqa70b_long from 48 sequences (1,759,932,928 bytes for
+# 1,755,018,024 algorithmic), llama13b_sampling from 64 sequences (558,502,144
+# for 542,159,500 unique); the captures are summarised in profiles/.
 TRAFFIC = {
-    # 48-sequence capture of the same shape (1.00295 x its algorithmic bytes), scaled
-    "gqa70b_long": {"bytes": 4774604438, "sources": "b0cf58fc4d2b"},
-    # full-size captures
-    "llama13b_sampling": {"bytes": 2156926208, "sources": "b0cf58fc4d2b"},
-    "llama7b_decode": {"bytes": 1121657600, "sources": "b0cf58fc4d2b"},
+    "gqa70b_long": {"bytes": 4773875309, "sources": "a229454128d1"},
+    "llama13b_sampling": {"bytes": 2173753832, "sources": "a229454128d1"},
 }
 
 

@@ -14,22 +14,24 @@
 // memory its scores came from (for each 16-key group: 8 columns of P_hi, then 8
 // of P_lo) and the second product reads it from there.
 //
-// Softmax: thread r of the softmax warpgroup owns row r of the tile whole
-// (every key column, every output dim), so no warp exchanges anything with
-// another.  A row is taken in four chunks of 32 keys, the next chunk's scores
-// loading from tensor memory while this one is processed.  The maximum is
-// raised lazily: each row keeps the maximum m it last used, and a chunk whose
-// scaled scores exceed m by more than 8 (log2 units) raises it -- by a whole
-// power of two, or to the chunk's maximum when the row had none -- rescaling
-// the row of O in tensor memory, the row sum and the weights already written
-// for the tile, all exactly (the factor is a power of two).  Otherwise
-// exp2(s - m) <= 256 is used as is; the final division by the row sum
-// accumulated with the same m makes the result exact either way.
+// Softmax: two warpgroups; warpgroup h owns key columns 64h .. 64h+63 of
+// every key tile and thread r of it row r of those, so no warp exchanges
+// anything with another inside an item.  Each half row keeps its own maximum
+// m, row sum l and accumulator O_h (P.V of keys 0-63 goes to O_0, of keys
+// 64-127 to O_1); at the end of an item the halves meet once in shared memory
+// and the result is O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / L with
+// M = max(m_0, m_1) and L the matching sum of l_0, l_1.  The maximum is kept
+// lazily: a half row with none yet takes its first visible tile's maximum;
+// after that the weights exp2(s - m) are formed with the maximum in use, and
+// only when they sum past 2^32 (or not to a finite number) is the tile's
+// maximum computed and, if it exceeds m by more than 32 (log2 units), m is
+// raised to it and the row of O_h, l and the tile's weights are rescaled.
+// Weights up to 2^32 cannot overflow fp32 sums, and the final division by l,
+// accumulated with the same m as O_h, makes the result exact either way.
 //
-// Tensor memory (512 columns): S/P of three key tiles (128 each) and O (128),
-// so the scores of the next two tiles are computed while the softmax works on
-// this one and the P.V of the previous one runs: the tensor core's work hides
-// behind the softmax.
+// Tensor memory (512 columns): S/P of two key tiles (128 each) and O_0, O_1
+// (128 each), so the scores of the next tile are computed while the softmax
+// works on this one and the P.V of the previous one runs.
 // Shared memory: q of one row tile, two K slots, three V slots (128-byte
 // swizzle).  K is laid out half by half (each 64-dim half of the 128 key rows
 // evenly spaced, as the first product needs), moved as two 2 KiB copies per
@@ -44,7 +46,7 @@
 //               tile and P.V of an earlier one, each as soon as its inputs are
 //               ready.
 //   warp 2      producer of V: each key tile's 8 pages.
-//   warps 4-7   softmax (thread = row).
+//   warps 4-11  softmax: two warpgroups, one per 64-key half of a tile.
 // Keys past a row's causal limit get p = 0; key rows past the context or in
 // pages with a bad block id are zeroed in V before the second product.  Every
 // wait is bounded; no unbounded barrier is used inside the role loops.

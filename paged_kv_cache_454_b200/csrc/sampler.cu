@@ -240,11 +240,12 @@ struct Smem {
   uint64_t hmass[256];
   uint64_t wsum[kWarps];
   uint64_t cand[kCand];       // small-K path: candidates, packed for sorting
-  uint32_t tmax[kThreads];    // each thread's largest key (pass 1)
+  uint32_t tmax[kThreads];    // each thread's largest key (K > 256)
   unsigned long long red64;
   int count;
   int overflow;
   int cut;
+  int cutk, cutp, cutt;  // first entry below the K-th / the Top-P cut / its ties
   int bin;
   uint32_t above_cnt;
   uint64_t above_mass;
@@ -342,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
       }
     });
   }
-  sm.tmax[tid] = bk;
+  const uint32_t kown = bk;  // this thread's largest key (the reduction below overwrites bk)
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const uint32_t k2 = __shfl_xor_sync(0xffffffffu, bk, o);
@@ -370,14 +371,53 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
   const float scale = kLog2e / T;
 
   // ---- small K: candidates in shared memory ----
-  // The K-th largest of the threads' maxima t0 is a lower bound of the K-th
-  // largest key (K distinct elements reach it), so every Top-K survivor has
-  // key >= t0.  When those elements fit in shared memory, everything else is
-  // done there: sort them, cut at the K-th, cut at Top-P, draw.
+  // t0 below is a lower bound of the K-th largest key, so every Top-K survivor
+  // has key >= t0.  When those elements fit in shared memory, everything else
+  // is done there: sort them, cut at the K-th, cut at Top-P, draw.
   if (K > 0 && K <= kFastK && K < V) {
-    // t0: the K-th largest of the 1024 thread maxima, by radix select
+    // t0.  K <= 256: each warp sorts its 32 threads' maxima (descending,
+    // across the lanes) and puts its kw = min(32, 2 ceil(K / 32)) largest into
+    // a pool of 32 kw >= K keys; t0 is the K-th largest key of the pool, by
+    // rank (a subset's K-th largest is at most the whole set's, and the pool
+    // misses a top maximum only when a warp holds more than kw of them).
+    // Larger K: the K-th largest of all 1024 maxima by radix select.  Either
+    // way K distinct elements are at or above t0.
     uint32_t t0 = 0;
-    {
+    if (tid == 0) {
+      sm.count = 0;
+      sm.overflow = 0;
+      sm.cutk = sm.cutp = sm.cutt = 0x7fffffff;
+    }
+    if (K <= 256) {
+      uint32_t v = kown;
+#pragma unroll
+      for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          const uint32_t o = __shfl_xor_sync(0xffffffffu, v, j);
+          // blocks of k lanes alternate descending / ascending; the last is descending
+          v = (((lane & j) == 0) == ((lane & k) == 0)) ? max(v, o) : min(v, o);
+        }
+      }
+      const int kw = min(32, 2 * ((K + 31) / 32));
+      // the pool: free space of the candidate array until the candidates come
+      uint32_t* pool = reinterpret_cast<uint32_t*>(sm.cand + kCand / 2);
+      if (lane < kw) pool[warp * kw + lane] = v;
+      __syncthreads();
+      const int np = kWarps * kw;
+      if (tid < np) {
+        const uint32_t x = pool[tid];
+        int r = 0;
+        for (int u = 0; u < np; ++u) {
+          const uint32_t y = pool[u];
+          r += (y > x) || (y == x && u < tid);
+        }
+        if (r == K - 1) sm.bin = static_cast<int>(x);
+      }
+      __syncthreads();
+      t0 = static_cast<uint32_t>(sm.bin);
+    } else {
+      sm.tmax[tid] = kown;
       uint32_t prefix = 0, pmask = 0, need = static_cast<uint32_t>(K);
       for (int dgt = 3; dgt >= 0; --dgt) {
         if (tid < 256) sm.hcnt[tid] = 0;
@@ -395,11 +435,6 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
       }
       t0 = prefix;
     }
-    if (tid == 0) {
-      sm.count = 0;
-      sm.overflow = 0;
-    }
-    __syncthreads();
     // (key, -index): descending order is by logit, then by index
     auto pack = [](uint32_t k, int i) {
       return (static_cast<uint64_t>(k) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
@@ -453,14 +488,12 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
         block_sort(sm.cand, n2, true);
       }
       const uint32_t tk = static_cast<uint32_t>(sm.cand[K - 1] >> 32);
-      // survivors of Top-K: the leading K entries and any ties with the K-th
-      if (tid == 0) {
-        int c = K;
-        while (c < n && static_cast<uint32_t>(sm.cand[c] >> 32) >= tk) ++c;
-        sm.count = c;
-      }
+      // survivors of Top-K: the leading K entries and every tie with the K-th,
+      // i.e. up to the first entry below it
+      for (int c = K + tid; c < n; c += kThreads)
+        if (static_cast<uint32_t>(sm.cand[c] >> 32) < tk) atomicMin(&sm.cutk, c);
       __syncthreads();
-      const int m = sm.count;
+      const int m = min(sm.cutk, n);
       // thread t owns sorted entries [4t, 4t + 4)
       const int j0 = 4 * tid;
       uint64_t ms[4];
@@ -479,24 +512,22 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
         uint64_t need = static_cast<uint64_t>(ceil(want));
         if (need < 1) need = 1;
         // the first sorted entry at which the running mass reaches `need`
-        if (tid == 0) sm.cut = m - 1;
-        __syncthreads();
+        // (the last one if rounding keeps the run short of it)
         uint64_t run = incl - mine;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int j = j0 + q;
-          if (j < m && run < need && run + ms[q] >= need) atomicMin(&sm.cut, j);
+          if (j < m && run < need && run + ms[q] >= need) atomicMin(&sm.cutp, j);
           run += ms[q];
         }
         __syncthreads();
-        if (tid == 0) {
-          const uint32_t cutkey = static_cast<uint32_t>(sm.cand[sm.cut] >> 32);
-          int c = sm.cut + 1;
-          while (c < m && static_cast<uint32_t>(sm.cand[c] >> 32) >= cutkey) ++c;  // ties
-          sm.count = c;
-        }
+        const int cut = min(sm.cutp, m - 1);
+        // and every tie with it: up to the first entry below it
+        const uint32_t cutkey = static_cast<uint32_t>(sm.cand[cut] >> 32);
+        for (int c = cut + 1 + tid; c < m; c += kThreads)
+          if (static_cast<uint32_t>(sm.cand[c] >> 32) < cutkey) atomicMin(&sm.cutt, c);
         __syncthreads();
-        m2 = sm.count;
+        m2 = min(sm.cutt, m);
       }
       // the draw: kept entries re-packed as (index, key) and sorted by index
       for (int i = tid; i < n2; i += kThreads) {

@@ -126,6 +126,25 @@ def test_clustered_top_logits(vocab):
         assert int(got[r]) in ok, (r, float(T[r]), int(K[r]), float(P[r]), float(u[r]), got[r], ok)
 
 
+@pytest.mark.parametrize("vocab", [3000, 32000, 152064])
+def test_top_k_across_the_threshold_paths(vocab):
+    # Top-K of 2..1024 on the small-K path: up to 256 the lower bound of the
+    # K-th largest logit comes from the warps' sorted maxima, above it from a
+    # radix select over every thread's maximum; both must keep every survivor.
+    rng = np.random.default_rng(vocab + 7)
+    Ks = [2, 33, 100, 255, 256, 257, 500, 700, 1000, 1024]
+    rows = len(Ks)
+    x = (rng.normal(size=(rows, vocab)) * rng.choice([1.0, 4.0], size=(rows, 1))).astype(np.float32)
+    T = np.full(rows, 1.0, np.float32)
+    K = np.array(Ks, np.int32)
+    P = rng.choice([0.9, 1.0], size=rows).astype(np.float32)
+    u = rng.random(rows).astype(np.float32)
+    got = run(x, T, K, P, u)
+    for r in range(rows):
+        ok = acceptable(x[r], float(T[r]), int(K[r]), float(P[r]), float(u[r]))
+        assert int(got[r]) in ok, (r, int(K[r]), float(P[r]), float(u[r]), got[r], ok)
+
+
 def test_same_inputs_same_tokens():
     rng = np.random.default_rng(2)
     x = rng.normal(size=(64, 5000)).astype(np.float32)
