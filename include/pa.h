@@ -153,6 +153,12 @@ PA_API int pa_copy_blocks(void* k_pool, void* v_pool, pa_pool_desc pool, const i
  *                  need no initialisation and are garbage afterwards.  Calls
  *                  that overlap on the GPU must not share a workspace.
  * Accumulation is fp32; the output is rounded to bf16 (nearest even).
+ * Stream order: the first kernel of the call (the work plan) is a programmatic
+ * dependent of the kernel before it on `stream`.  If that kernel signals that
+ * its dependents may start early (this library's cache write and prefill
+ * kernels do), the plan reads block_tables and context_lens while it still
+ * runs -- they must be final by then -- and no K/V is read before it has
+ * finished.  Kernels that do not signal (any other) are waited for as usual.
  */
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, pa_pool_desc pool,
                                 int32_t max_blocks_per_seq);

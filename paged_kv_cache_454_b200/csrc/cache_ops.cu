@@ -20,6 +20,9 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const uint4* __restrict__ key, const uint4* __restrict__ value, int64_t token_stride_chunks,
     uint4* __restrict__ k_pool, uint4* __restrict__ v_pool, int num_blocks, int hkv, int chunks,
     const int64_t* __restrict__ slot_mapping, int num_tokens, unsigned int* err) {
+  // the decode plan launched after this kernel may start now: it reads only
+  // the tables and lengths, and it waits for this grid before it completes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t per_token = static_cast<int64_t>(hkv) * chunks;
   const int64_t total = per_token * num_tokens;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;

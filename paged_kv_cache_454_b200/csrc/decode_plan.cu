@@ -542,17 +542,37 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     }
   }
   for (int i = tid; i < S * kv_heads; i += 1024) merge_cnt[i] = 0;
+  // The plan is a programmatic dependent of the kernel before it (the cache
+  // write that puts this step's tokens in the pool, or a prefill): it reads
+  // only the tables and lengths, so it runs while that kernel finishes, and
+  // it completes only after that kernel has -- the decode kernel, which waits
+  // for this grid, then sees the pool as written.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace
 
 int launch_decode_plan(const DecodeArgs& a) {
-  decode_plan_kernel<<<1, 1024, 0, a.stream>>>(
-      a.context_lens, a.block_tables, a.num_seqs, a.max_blocks,
-      a.pool.num_kv_heads / a.item_heads, a.pool.num_kv_heads, a.min_part, a.max_part,
-      a.target_items, num_sms(), a.num_q_heads / a.pool.num_kv_heads, a.casc_cols,
-      a.ws.header, a.ws.part_base, a.ws.items, a.ws.merge_cnt, a.ws.seq_span, a.ws.seq_pp,
-      a.ws.runs, a.ws.pitems, a.err);
+  // a programmatic dependent of the previous kernel on the stream (see the end
+  // of the kernel)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(1024);
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, decode_plan_kernel, a.context_lens, a.block_tables, a.num_seqs,
+                         a.max_blocks, a.pool.num_kv_heads / a.item_heads, a.pool.num_kv_heads,
+                         a.min_part, a.max_part, a.target_items, num_sms(),
+                         a.num_q_heads / a.pool.num_kv_heads, a.casc_cols, a.ws.header,
+                         a.ws.part_base, a.ws.items, a.ws.merge_cnt, a.ws.seq_span, a.ws.seq_pp,
+                         a.ws.runs, a.ws.pitems, a.err) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
   return launch_status();
 }
 

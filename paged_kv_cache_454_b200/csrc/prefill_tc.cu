@@ -294,6 +294,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
       }
     }
+    // this CTA has issued its last item: a programmatic dependent launched
+    // after this kernel (the decode plan) may start on the SMs that free up
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (*abort_flag && lane == 0) {
       for (uint32_t u = t > kKSlots ? t - kKSlots : 0; u < t; ++u)
         mbar_wait(&k_full[u % kKSlots], (u / kKSlots) & 1, nullptr, p.err);

@@ -235,6 +235,100 @@ __device__ uint64_t block_scan64(uint64_t x, uint64_t* wbuf, uint64_t* tot) {
   return r;
 }
 
+// The cuts and the draw of the small-K path by one warp, for n <= kWarpTail
+// candidates sorted by (key, -index) descending in cand[0, n): Top-K keeps the
+// first K and every tie with the K-th; Top-P keeps the shortest prefix whose
+// mass reaches P of the kept mass, and its ties; the draw is inverse-CDF in
+// vocabulary order, each kept entry's index-order prefix mass counted over
+// the kept entries.  `mass` is scratch for n masses.  Lane l holds entries
+// 8l .. 8l + 7 (so sorted order is lane-major).
+constexpr int kWarpTail = 256;
+__device__ void warp_tail(const uint64_t* cand, int n, int K, float P, float u, float xmax,
+                          float scale, uint64_t* mass, int32_t* token) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t tk = static_cast<uint32_t>(cand[K - 1] >> 32);
+  uint32_t key[8];
+  int first_below = n;  // the first entry past the K-th that is below it
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = 8 * lane + j;
+    key[j] = e < n ? static_cast<uint32_t>(cand[e] >> 32) : 0u;
+    if (e >= K && e < n && key[j] < tk) first_below = min(first_below, e);
+  }
+  const int m = __reduce_min_sync(0xffffffffu, first_below);
+  uint64_t ms[8], lsum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    ms[j] = 8 * lane + j < m ? mass_of(float_of(key[j]), xmax, scale) : 0ull;
+    lsum += ms[j];
+  }
+  uint64_t incl = lsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint64_t mk = __shfl_sync(0xffffffffu, incl, 31);
+  int m2 = m;
+  if (P < 1.f) {
+    const double want = static_cast<double>(P > 0.f ? P : 0.f) * static_cast<double>(mk);
+    uint64_t need = static_cast<uint64_t>(ceil(want));
+    if (need < 1) need = 1;
+    // the first entry at which the running mass reaches `need` (the last one
+    // if rounding keeps the run short of it), then its ties
+    uint64_t run = incl - lsum;
+    int cut_l = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = 8 * lane + j;
+      if (e < m && run < need && run + ms[j] >= need) cut_l = min(cut_l, e);
+      run += ms[j];
+    }
+    int cut = __reduce_min_sync(0xffffffffu, cut_l);
+    if (cut > m - 1) cut = m - 1;
+    const uint32_t cutkey = static_cast<uint32_t>(cand[cut] >> 32);
+    int tie_l = m;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = 8 * lane + j;
+      if (e > cut && e < m && key[j] < cutkey) tie_l = min(tie_l, e);
+    }
+    m2 = __reduce_min_sync(0xffffffffu, tie_l);
+  }
+  // the draw: kept entries e < m2, in vocabulary order
+  uint64_t total = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = 8 * lane + j;
+    if (e >= m2) ms[j] = 0ull;
+    if (e < n) mass[e] = ms[j];
+    total += ms[j];
+  }
+  for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+  __syncwarp();
+  const uint64_t tg = static_cast<uint64_t>(static_cast<double>(u) * static_cast<double>(total));
+  const uint64_t tgt = tg < total ? tg : total - 1;
+  uint32_t idx[8];
+  uint64_t pre[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    idx[j] = 0xffffffffu - static_cast<uint32_t>(cand[min(8 * lane + j, n - 1)]);
+    pre[j] = 0;
+  }
+  // each kept entry's mass before it in vocabulary order
+  for (int f = 0; f < m2; ++f) {
+    const uint32_t fi = 0xffffffffu - static_cast<uint32_t>(cand[f]);
+    const uint64_t fm = mass[f];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) pre[j] += fi < idx[j] ? fm : 0ull;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = 8 * lane + j;
+    if (e < m2 && ms[j] > 0 && pre[j] <= tgt && pre[j] + ms[j] > tgt) *token = static_cast<int32_t>(idx[j]);
+  }
+}
+
 struct Smem {
   uint32_t hcnt[256];
   uint64_t hmass[256];
@@ -486,6 +580,12 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
         for (int i = n + tid; i < n2; i += kThreads) sm.cand[i] = 0ull;  // below every real entry
         __syncthreads();
         block_sort(sm.cand, n2, true);
+      }
+      if (n <= kWarpTail) {
+        // Up to kWarpTail candidates (the usual case): one warp takes the
+        // cuts and the draw with shuffles and warp reductions, no barriers.
+        if (warp == 0) warp_tail(sm.cand, n, K, P, u, xmax, scale, sm.cand + kCand / 2, tokens + row);
+        return;
       }
       const uint32_t tk = static_cast<uint32_t>(sm.cand[K - 1] >> 32);
       // survivors of Top-K: the leading K entries and every tie with the K-th,
