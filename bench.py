@@ -722,15 +722,20 @@ def main():
                 "peak_source": f"{peak_src} hbm_gbs",
                 "frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
                 "algorithmic_bytes": algo, "logical_bytes": b["logical"],
-                "kernel_ms": round(comp["decode"], 4), "traffic": traffic_for(a.workload, w)}
-    elif len(w.pf):
+                "kernel_ms": round(comp["decode"], 4), "traffic": traffic_for(a.workload, "decode")}
+    # the chunked prefill's own roofline (the dominant kernel's when it is the
+    # longer part of the step)
+    roof_pf = None
+    if len(w.pf):
         achieved = w.flops_pf / (comp["prefill"] * 1e-3) / 1e12
         pk = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "kernel": "pa_chunked_prefill", "achieved": round(achieved, 1),
-                "peak": pk, "unit": "TFLOP/s", "frac": round(achieved / pk, 4),
-                "peak_source": f"{peak_src} bf16_tflops_sustained",
-                "algorithmic_flops": w.flops_pf, "kernel_ms": round(comp["prefill"], 4),
-                "traffic": None}
+        roof_pf = {"bound": "tensor", "kernel": "pa_chunked_prefill", "achieved": round(achieved, 1),
+                   "peak": pk, "unit": "TFLOP/s", "frac": round(achieved / pk, 4),
+                   "peak_source": f"{peak_src} bf16_tflops_sustained",
+                   "algorithmic_flops": w.flops_pf, "kernel_ms": round(comp["prefill"], 4),
+                   "traffic": traffic_for(a.workload, "prefill") if not a.num_seqs else None}
+        if roof is None:
+            roof = roof_pf
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms, 4),
@@ -752,6 +757,7 @@ def main():
         "prefill_ms_stats": step_stats(ev, "cache", "prefill") if len(w.pf) else None,
         "kv_gbs": round(w.bytes_dec["unique"] / (comp["decode"] * 1e-3) / 1e9, 1) if len(w.dec) else None,
         "roofline": roof,
+        "roofline_prefill": roof_pf if roof_pf is not roof else None,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": w.launches_per_step() * a.steps,
@@ -768,35 +774,43 @@ def main():
         pg.destroy_process_group()
 
 
-# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# decode kernel from an ncu capture, keyed by workload and the kernel sources
-# it was taken with (reported as null once those sources change).  Both are
-# captures of a smaller batch of the same shape, scaled to the full batch by
-# algorithmic bytes: gqa70b_long from 48 sequences (1,759,932,928 bytes for
-# 1,755,018,024 algorithmic), llama13b_sampling from 64 sequences (558,502,144
-# for 542,159,500 unique); the captures are summarised in profiles/.
+# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of a
+# kernel from an ncu capture, keyed by (workload, kernel) and the sources the
+# kernel was built from (reported as null once those sources change).  The
+# decode figures are captures of a smaller batch of the same shape, scaled to
+# the full batch by algorithmic bytes: gqa70b_long from 48 sequences
+# (1,760,207,872 bytes for 1,755,018,024 algorithmic), llama13b_sampling from
+# 64 sequences (558,156,288 for 542,159,500 unique).  The prefill figure is the
+# mixed step's prefill part itself (its 8 chunks, with the decode part shrunk
+# to 8 sequences: the prefill launch is the same).  The captures are
+# summarised in profiles/.
 TRAFFIC = {
-    "gqa70b_long": {"bytes": 4774621103, "sources": "978d8fa2d68c"},
-    "llama13b_sampling": {"bytes": 2172407721, "sources": "978d8fa2d68c"},
+    ("gqa70b_long", "decode"): {"bytes": 4774621103, "sources": "978d8fa2d68c"},
+    ("llama13b_sampling", "decode"): {"bytes": 2172407721, "sources": "978d8fa2d68c"},
+    ("mixed_qwen32b", "prefill"): {"bytes": 187142656, "sources": "2723f04b3083"},
 }
 
 
-# the sources the decode path's two kernels (plan, tensor-core decode) are built from
-DECODE_SOURCES = ("decode_plan.cu", "decode_tc.cu", "common.cuh", "tc_common.cuh")
+# the sources each path's kernels are built from: decode (plan, tensor-core
+# decode) and chunked prefill
+KERNEL_SOURCES = {
+    "decode": ("decode_plan.cu", "decode_tc.cu", "common.cuh", "tc_common.cuh"),
+    "prefill": ("prefill_tc.cu", "common.cuh", "tc_common.cuh"),
+}
 
 
-def kernel_source_digest():
+def kernel_source_digest(kind="decode"):
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "paged_kv_cache_454_b200", "csrc")
-    for f in DECODE_SOURCES:
+    for f in KERNEL_SOURCES[kind]:
         h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:12]
 
 
-def traffic_for(workload, w):
-    rec = TRAFFIC.get(workload)
-    if not rec or rec.get("sources") != kernel_source_digest():
+def traffic_for(workload, kind="decode"):
+    rec = TRAFFIC.get((workload, kind))
+    if not rec or rec.get("sources") != kernel_source_digest(kind):
         return None
     return rec["bytes"]
 

@@ -7,12 +7,16 @@
 // and shares every K/V tile among them.  Per 128-key tile of the paged context:
 //     S [128 rows x 128 keys] = Q_tile [128 x D] . K_tile^T         (8 MMAs, K = 16)
 //     O [128 rows x D]       += P [128 x 128 keys] . V_tile         (16 MMAs, K = 16)
-// with fp32 accumulators in tensor memory.  P = P_hi + P_lo, the bf16 rounding
-// of p and the bf16 rounding of what it left out, so the weights reach the
-// product with about 16 significant bits (bf16 p alone misses the output
-// tolerance on contexts of a few keys).  P is written back into the tensor
-// memory its scores came from (for each 16-key group: 8 columns of P_hi, then 8
-// of P_lo) and the second product reads it from there.
+// with fp32 accumulators in tensor memory.  P = P_hi + P_lo, p with its
+// mantissa cut to bf16 and the same cut of what that left out, so the weights
+// reach the product with about 16 significant bits where they need them: a
+// key half of a tile whose weights are at most a quarter of the half row's
+// sum so far (in every row of the tile) goes to the product as P_hi alone,
+// since its share of the output bounds what the cut can change; the first
+// tiles of a row, and every tile of a row of a few keys, take P_lo as well
+// (bf16 p alone misses the output tolerance on contexts of a few keys).  P is
+// written back into the tensor memory its scores came from (per 64-key half:
+// 32 columns of P_hi, then 32 of P_lo) and the second product reads it there.
 //
 // Softmax: two warpgroups; warpgroup h owns key columns 64h .. 64h+63 of
 // every key tile and thread r of it row r of those, so no warp exchanges
@@ -72,8 +76,9 @@ constexpr int kOffBar = kOffV + kVSlots * kTileBytes;
 // (per S/P buffer); o_free; drain; the halves' exchange at the end of an item
 constexpr int kNumBars = 2 * (kQSlots + kKSlots + kVSlots) + 3 * kSP + 1 + 1 + 1;
 constexpr int kMaskRing = 16;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem slot, abort flag, kmask ring
-constexpr int kOffX = kOffMisc + 16 + 4 * kMaskRing;  // [2 items][2 halves][128 rows] (m, l)
+constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem slot, abort flag, kmask ring, lo flags
+constexpr int kOffLo = kOffMisc + 16 + 4 * kMaskRing;  // [S/P buffer][key half] tile number
+constexpr int kOffX = kOffLo + 8 * kSP;  // [2 items][2 halves][128 rows] (m, l)
 constexpr int kSmemUsed = kOffX + 2 * 2 * 128 * 8;
 constexpr int kSmemBytes = kSmemUsed + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -83,6 +88,10 @@ constexpr int kOcol = kSP * 128;  // O_0 at kOcol, O_1 at kOcol + 128
 constexpr uint32_t kPageHalf = 16 * 128;  // one 64-dim half of one page: 2 KiB
 constexpr float kRescaleLog2 = 32.f;      // raise the row maximum only past 2^32
 constexpr float kRaiseSum = 4294967296.f;  // 2^32: weights summing to less need no raise
+// A half row's weights of a key tile go to the second product as P_hi alone
+// when they sum to at most a quarter of the half row's sum so far (their sum
+// is then at most 1/3 of the sum before the tile).
+constexpr float kLoSkipRatio = 3.f;
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);
@@ -113,6 +122,26 @@ struct PfItem {
   bool valid;
   int s, g, q0, i0, ntok, c, ctx, kv_end, ntiles;
 };
+
+// AND of `pred` over the 128 threads of a warpgroup (named barrier `id`).
+__device__ __forceinline__ bool warpgroup_all(int id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred q, a;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred a, %2, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, a;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ uint2 lds_volatile_u32x2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.volatile.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ int ld_early(const int32_t* ptr) {
   int x;
@@ -223,6 +252,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   // producer before the tile's copies; the softmax reads it after the tile's
   // scores, long before the producer can come round to the slot again)
   uint32_t* kmask = reinterpret_cast<uint32_t*>(sptr + kOffMisc + 16);
+  // lo_seq[2 b + h] = t + 1 when key half h of key tile t (in S/P buffer
+  // b = t % kSP) has P_lo written; then the MMA issues that half's P_lo
+  // products.  The first warp of each softmax warpgroup writes it, before its
+  // arrival on p_full; the MMA reads both halves' words in one load.
+  static_assert(kOffLo % 8 == 0, "lo_seq pairs are read as 8 bytes");
+  volatile uint32_t* lo_seq = reinterpret_cast<volatile uint32_t*>(sptr + kOffLo);
   float2* xbuf = reinterpret_cast<float2*>(sptr + kOffX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -248,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     mbar_init(drain, 1);
     mbar_init(xchg, 8);
     *abort_flag = 0;
+    for (int i = 0; i < kSP * 2; ++i) lo_seq[i] = 0;
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
     prefetch_tmap(&p.tm_q);
@@ -362,13 +398,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tc_fence_after();
             const uint64_t vb = desc_add(dv0, vs * kTileBytes);
             const uint32_t sp = tmem + sb * 128;
-            // keys 0-63 of the tile into O_0, keys 64-127 into O_1
+            // the halves' P_lo flags, read while the P_hi products issue
+            const uint2 lf = lds_volatile_u32x2(sbase + kOffLo + sb * 8);
+            // keys 0-63 of the tile into O_0, keys 64-127 into O_1; a half's
+            // 64 columns of P are 32 of P_hi, then 32 of P_lo
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              const uint64_t bd = desc_add(vb, k * 4096);
               const uint32_t oc = tmem + kOcol + (k >> 2) * 128;
-              umma_ts(oc, sp + 16 * k, bd, kIdescO, (first && (k & 3) == 0) ? 0u : 1u);
-              umma_ts(oc, sp + 16 * k + 8, bd, kIdescO, 1u);
+              umma_ts(oc, sp + 64 * (k >> 2) + 8 * (k & 3), desc_add(vb, k * 4096), kIdescO,
+                      (first && (k & 3) == 0) ? 0u : 1u);
+            }
+            const bool lo0 = lf.x == tpv + 1, lo1 = lf.y == tpv + 1;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              if ((k >> 2) ? lo1 : lo0)
+                umma_ts(tmem + kOcol + (k >> 2) * 128, sp + 64 * (k >> 2) + 32 + 8 * (k & 3),
+                        desc_add(vb, k * 4096), kIdescO, 1u);
             }
             umma_commit(&pv_done[sb]);
             umma_commit(&v_empty[vs]);
@@ -469,9 +514,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // visible keeps its warp on the unmasked path.
         const int nvis = min(max(limit - kv0, 0), 64);  // leading visible keys
         const bool all_vis = __all_sync(0xffffffffu, !row_ok || (nvis == 64 && vm == 0xfu));
-        // the half row of scores in registers (one wait), scaled
+        // The half row of scores in registers (one wait), scaled with the
+        // maximum in use; keys that are not visible become -inf (p = 0),
+        // whatever their score.
         float xv[64];
-        {
+        auto load_x = [&]() {
           uint32_t sa[32], sb2[32];
           tmem_ld32_nowait(scol, sa);
           tmem_ld32_nowait(scol + 32, sb2);
@@ -490,50 +537,53 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             xv[32 + k] = xb.x;
             xv[32 + k + 1] = xb.y;
           }
-        }
-        if (!all_vis) {
-          // keys that are not visible become -inf (p = 0), whatever their score
+          if (!all_vis) {
 #pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            const int nw = min(max(nvis - 32 * w, 0), 32);
-            const uint32_t lead = nw >= 32 ? 0xffffffffu : ((1u << nw) - 1u);
-            const uint32_t pg = (((vm >> (2 * w)) & 1u) ? 0x0000ffffu : 0u) |
-                                (((vm >> (2 * w + 1)) & 1u) ? 0xffff0000u : 0u);
-            const uint32_t vw = row_ok ? (lead & pg) : 0xffffffffu;
+            for (int w = 0; w < 2; ++w) {
+              const int nw = min(max(nvis - 32 * w, 0), 32);
+              const uint32_t lead = nw >= 32 ? 0xffffffffu : ((1u << nw) - 1u);
+              const uint32_t pg = (((vm >> (2 * w)) & 1u) ? 0x0000ffffu : 0u) |
+                                  (((vm >> (2 * w + 1)) & 1u) ? 0xffff0000u : 0u);
+              const uint32_t vw = row_ok ? (lead & pg) : 0xffffffffu;
 #pragma unroll
-            for (int k = 0; k < 32; ++k)
-              xv[32 * w + k] = ((vw >> k) & 1u) ? xv[32 * w + k] : -CUDART_INF_F;
+              for (int k = 0; k < 32; ++k)
+                xv[32 * w + k] = ((vw >> k) & 1u) ? xv[32 * w + k] : -CUDART_INF_F;
+            }
           }
-        }
-        // Weights of the half row with the maximum in use, written back over
-        // the scores as P_hi / P_lo (P_hi is p with its mantissa cut to bf16,
-        // P_lo the same cut of the remainder: p = P_hi + P_lo to within 2^-15
-        // of p), formed with integer masks and byte permutes, leaving the
-        // multi-function unit to ex2; returns the sum of the weights.
-        auto weights = [&]() -> float {
+        };
+        load_x();
+        // Weights of the half row with the maximum in use, in place of the
+        // scores, and P_hi (p with its mantissa cut to bf16, two keys a
+        // column) in hw, formed with byte permutes between the multi-function
+        // unit's ex2; returns the sum of the weights.
+        uint32_t hw[32];
+        auto exp_pass = [&]() -> float {
           float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t pw[32];
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              const int kk = 32 * c + k;
-              const float p0 = exp2f(xv[kk]);
-              const float p1 = exp2f(xv[kk + 1]);
-              const float2 pp = make_float2(p0, p1);
-              rs2[(k >> 1) & 1] = __fadd2_rn(rs2[(k >> 1) & 1], pp);
-              const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-              const float2 hi = make_float2(__uint_as_float(b0 & 0xffff0000u),
-                                            __uint_as_float(b1 & 0xffff0000u));
-              const float2 lo = __ffma2_rn(hi, neg1, pp);  // p - P_hi, exact
-              const int g = k >> 4, kg = k & 15;  // 16-key group within the chunk
-              pw[16 * g + (kg >> 1)] = __byte_perm(b0, b1, 0x7632);
-              pw[16 * g + 8 + (kg >> 1)] =
-                  __byte_perm(__float_as_uint(lo.x), __float_as_uint(lo.y), 0x7632);
-            }
-            tmem_st32_nowait(scol + 32 * c, pw);
+          for (int k = 0; k < 64; k += 2) {
+            const float p0 = exp2f(xv[k]);
+            const float p1 = exp2f(xv[k + 1]);
+            xv[k] = p0;
+            xv[k + 1] = p1;
+            rs2[(k >> 1) & 1] = __fadd2_rn(rs2[(k >> 1) & 1], make_float2(p0, p1));
+            hw[k >> 1] = __byte_perm(__float_as_uint(p0), __float_as_uint(p1), 0x7632);
           }
           return (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
+        };
+        // P_lo, the same cut of p - P_hi (so P_hi + P_lo is p to within 2^-15
+        // of p), in the next 32 columns, formed with integer masks and byte
+        // permutes.
+        auto store_lo = [&]() {
+          uint32_t lw[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float2 pp = make_float2(xv[2 * k], xv[2 * k + 1]);
+            const float2 hi = make_float2(__uint_as_float(__float_as_uint(pp.x) & 0xffff0000u),
+                                          __uint_as_float(__float_as_uint(pp.y) & 0xffff0000u));
+            const float2 lo = __ffma2_rn(hi, neg1, pp);  // p - P_hi, exact
+            lw[k] = __byte_perm(__float_as_uint(lo.x), __float_as_uint(lo.y), 0x7632);
+          }
+          tmem_st32_nowait(scol + 32, lw);
         };
         // Raise the maximum in use to the tile's maximum xm (scaled, relative
         // to the old one); then this half's row of O_h (earlier key tiles of
@@ -587,21 +637,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           const bool raise = m == -CUDART_INF_F ? xm != -CUDART_INF_F : xm > kRescaleLog2;
           if (__any_sync(0xffffffffu, raise)) raise_to(raise, xm);
         }
-        float rs = weights();
+        float rs = exp_pass();
         {
           const bool check = row_ok && !(rs <= kRaiseSum);
           if (__any_sync(0xffffffffu, check)) {
-            tmem_wait_st();
+            // the weights took the scores' registers: reload the scores
+            // (still in tensor memory) for the tile's maximum
+            load_x();
             const float xm = row_max();
             const bool raise = check && xm > kRescaleLog2;
-            if (__any_sync(0xffffffffu, raise)) {
-              raise_to(raise, xm);
-              rs = weights();
-            }
+            if (__any_sync(0xffffffffu, raise)) raise_to(raise, xm);
+            rs = exp_pass();
           }
         }
+        // P_lo is left out for this key half of the tile when, in every row
+        // of the warpgroup, the tile's weights are at most a quarter of the
+        // half row's sum with them: each such weight is then at most 1/4 of
+        // its final value's denominator, and the cut's relative error (below
+        // 2^-7) reaches the output scaled by that share.
+        tmem_st32_nowait(scol, hw);  // P_hi over the scores' first 32 columns
+        const bool with_lo =
+            !warpgroup_all(1 + hf, !row_ok || kLoSkipRatio * rs <= l);
+        if (with_lo) store_lo();
         tmem_wait_st();
         l += rs;
+        if (with_lo && q4 == 0 && lane == 0) lo_seq[sb * 2 + hf] = t + 1;
         // key rows of this half past the context or in an unloaded page: zero
         // them in V (threads 0-63 of the warpgroup, one key row each)
         if (j * 128 + 128 > I.ctx || vm != 0xfu) {
