@@ -787,7 +787,7 @@ def main():
 TRAFFIC = {
     ("gqa70b_long", "decode"): {"bytes": 4774621103, "sources": "978d8fa2d68c"},
     ("llama13b_sampling", "decode"): {"bytes": 2172407721, "sources": "978d8fa2d68c"},
-    ("mixed_qwen32b", "prefill"): {"bytes": 187142656, "sources": "2723f04b3083"},
+    ("mixed_qwen32b", "prefill"): {"bytes": 185013760, "sources": "d5dda8f04e86"},
 }
 
 

@@ -246,6 +246,16 @@ PA_API int pa_decode_noalloc(const void* q, int64_t q_stride, const void* k_pool
  *   context_lens int32 [num_seqs], device, including the chunk.
  *   out          bf16 [total_q][num_q_heads][head_dim], packed.
  *   lse          float [total_q][num_q_heads], or NULL.
+ *
+ * Precision (head_dim 128, tensor cores): scores and the P.V product
+ * accumulate in fp32; the softmax weights p enter P.V as p with its mantissa
+ * cut to bf16 plus, where needed, the same cut of the remainder (about 16
+ * significant bits together).  A 64-key half of a 128-key tile goes without
+ * the remainder when, in every row of the 128-row tile, its weights sum to at
+ * most a quarter of that half row's sum up to and including the tile: such a
+ * tile's weights are then at most a quarter of their final denominator, and
+ * each is short of itself by less than 2^-7 of itself.  pa_chunked_prefill_ex with
+ * PA_PREFILL_EXACT_WEIGHTS carries the remainder on every tile.
  */
 PA_API int pa_chunked_prefill(const void* q, int64_t q_stride, const int32_t* cu_q_lens,
                        int32_t total_q, int32_t max_q_len, const void* k_pool,
@@ -253,6 +263,20 @@ PA_API int pa_chunked_prefill(const void* q, int64_t q_stride, const int32_t* cu
                        int32_t max_blocks_per_seq, const int32_t* context_lens,
                        int32_t num_seqs, int32_t num_q_heads, float scale, void* out, float* lse,
                        void* stream);
+
+/*
+ * pa_chunked_prefill_ex -- pa_chunked_prefill with `flags`: 0, or
+ * PA_PREFILL_EXACT_WEIGHTS (every key tile's P.V takes the weights' bf16
+ * remainder as well, so each weight reaches the product to within 2^-15 of
+ * itself; slower).  Other bits: PA_ERR_ARG.
+ */
+#define PA_PREFILL_EXACT_WEIGHTS 0x1u
+PA_API int pa_chunked_prefill_ex(const void* q, int64_t q_stride, const int32_t* cu_q_lens,
+                          int32_t total_q, int32_t max_q_len, const void* k_pool,
+                          const void* v_pool, pa_pool_desc pool, const int32_t* block_tables,
+                          int32_t max_blocks_per_seq, const int32_t* context_lens,
+                          int32_t num_seqs, int32_t num_q_heads, float scale, void* out,
+                          float* lse, uint32_t flags, void* stream);
 
 /*
  * pa_gather_kv -- copy every sequence's paged K and V into contiguous,

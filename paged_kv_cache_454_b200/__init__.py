@@ -14,7 +14,7 @@ import numpy as np
 from . import _abi
 from ._abi import (PA_DEV_ERR_BLOCK_ID, PA_DEV_ERR_CONTEXT, PA_DEV_ERR_SLOT,  # noqa: F401
                    PA_DEV_ERR_TIMEOUT, PA_KERNEL_AUTO, PA_KERNEL_SIMT, PA_KERNEL_TCGEN05,
-                   PaError, PoolDesc)
+                   PA_PREFILL_EXACT_WEIGHTS, PaError, PoolDesc)
 
 __all__ = [
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size",
@@ -23,6 +23,7 @@ __all__ = [
     "pa_read_probe",
     "pool_desc", "lib",
     "PaError", "PA_KERNEL_AUTO", "PA_KERNEL_SIMT", "PA_KERNEL_TCGEN05",
+    "PA_PREFILL_EXACT_WEIGHTS",
 ]
 
 
@@ -169,9 +170,12 @@ def pa_decode_noalloc(q, k_pool, v_pool, block_tables, context_lens, scale, out=
 
 
 def pa_chunked_prefill(q, cu_q_lens, max_q_len, k_pool, v_pool, block_tables, context_lens,
-                       scale, out=None, lse=None, stream=None, want_lse=False):
+                       scale, out=None, lse=None, stream=None, want_lse=False,
+                       exact_weights=False):
     """Causal attention of each sequence's new chunk over its cached context plus
-    itself.  ``q`` bf16 [total_q, Hq, D]; ``cu_q_lens`` int32 [S+1] (device)."""
+    itself.  ``q`` bf16 [total_q, Hq, D]; ``cu_q_lens`` int32 [S+1] (device).
+    ``exact_weights`` asks for the weights' bf16 remainder on every key tile
+    (``pa_chunked_prefill_ex`` with ``PA_PREFILL_EXACT_WEIGHTS``)."""
     torch = _torch()
     _check_pools(k_pool, v_pool)
     _need_cuda("q", q, torch.bfloat16, contiguous=False)
@@ -188,10 +192,16 @@ def pa_chunked_prefill(q, cu_q_lens, max_q_len, k_pool, v_pool, block_tables, co
     if lse is not None:
         _need_cuda("lse", lse, torch.float32)
     S = context_lens.shape[0]
-    _abi.check("pa_chunked_prefill", lib().pa_chunked_prefill(
-        _ptr(q), qs, _ptr(cu_q_lens), total_q, int(max_q_len), _ptr(k_pool), _ptr(v_pool),
-        pool_desc(k_pool), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, hq,
-        float(scale), _ptr(out), _ptr(lse), _stream(stream)))
+    if exact_weights:
+        _abi.check("pa_chunked_prefill_ex", lib().pa_chunked_prefill_ex(
+            _ptr(q), qs, _ptr(cu_q_lens), total_q, int(max_q_len), _ptr(k_pool), _ptr(v_pool),
+            pool_desc(k_pool), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S,
+            hq, float(scale), _ptr(out), _ptr(lse), PA_PREFILL_EXACT_WEIGHTS, _stream(stream)))
+    else:
+        _abi.check("pa_chunked_prefill", lib().pa_chunked_prefill(
+            _ptr(q), qs, _ptr(cu_q_lens), total_q, int(max_q_len), _ptr(k_pool), _ptr(v_pool),
+            pool_desc(k_pool), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S,
+            hq, float(scale), _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
 
 

@@ -31,6 +31,7 @@ PA_DEV_ERR_TIMEOUT = 0x8
 PA_KERNEL_AUTO = 0
 PA_KERNEL_SIMT = 1
 PA_KERNEL_TCGEN05 = 2
+PA_PREFILL_EXACT_WEIGHTS = 0x1
 
 PA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
@@ -57,6 +58,9 @@ SIGNATURES = {
                                   c_i32, c_f32, c_vp, c_vp, c_vp]),
     "pa_chunked_prefill": (c_int, [c_vp, c_i64, c_vp, c_i32, c_i32, c_vp, c_vp, PoolDesc, c_vp,
                                    c_i32, c_vp, c_i32, c_i32, c_f32, c_vp, c_vp, c_vp]),
+    "pa_chunked_prefill_ex": (c_int, [c_vp, c_i64, c_vp, c_i32, c_i32, c_vp, c_vp, PoolDesc, c_vp,
+                                      c_i32, c_vp, c_i32, c_i32, c_f32, c_vp, c_vp, ctypes.c_uint32,
+                                      c_vp]),
     "pa_gather_kv": (c_int, [c_vp, c_vp, PoolDesc, c_vp, c_i32, c_vp, c_vp, c_i32, c_i32, c_vp,
                              c_vp, c_vp]),
     "pa_get_device_error": (c_int, [ctypes.POINTER(ctypes.c_uint32), c_vp]),

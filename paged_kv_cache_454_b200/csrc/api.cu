@@ -285,6 +285,19 @@ int pa_chunked_prefill(const void* q, int64_t q_stride, const int32_t* cu_q_lens
                        int32_t num_seqs, int32_t num_q_heads, float scale, void* out, float* lse,
                        void* stream) {
   PA_NVTX_RANGE("pa_chunked_prefill");
+  return pa_chunked_prefill_ex(q, q_stride, cu_q_lens, total_q, max_q_len, k_pool, v_pool, pool,
+                               block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                               num_q_heads, scale, out, lse, 0u, stream);
+}
+
+int pa_chunked_prefill_ex(const void* q, int64_t q_stride, const int32_t* cu_q_lens,
+                          int32_t total_q, int32_t max_q_len, const void* k_pool,
+                          const void* v_pool, pa_pool_desc pool, const int32_t* block_tables,
+                          int32_t max_blocks_per_seq, const int32_t* context_lens,
+                          int32_t num_seqs, int32_t num_q_heads, float scale, void* out,
+                          float* lse, uint32_t flags, void* stream) {
+  PA_NVTX_RANGE("pa_chunked_prefill_ex");
+  if (flags & ~static_cast<uint32_t>(PA_PREFILL_EXACT_WEIGHTS)) return PA_ERR_ARG;
   int st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || num_q_heads <= 0 ||
@@ -316,6 +329,7 @@ int pa_chunked_prefill(const void* q, int64_t q_stride, const int32_t* cu_q_lens
   a.scale = scale;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
+  a.exact_weights = (flags & PA_PREFILL_EXACT_WEIGHTS) != 0;
   a.err = device_error_word();
   a.stream = as_stream(stream);
   if (!a.err) return PA_ERR_CUDA;

@@ -163,6 +163,7 @@ struct PrefillArgs {
   float scale;
   uint16_t* out;
   float* lse;
+  bool exact_weights = false;  // PA_PREFILL_EXACT_WEIGHTS
   unsigned int* err;
   cudaStream_t stream;
 };

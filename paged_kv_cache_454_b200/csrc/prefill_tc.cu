@@ -115,6 +115,7 @@ struct __align__(64) PfParams {
   int num_seqs;
   int mt_max;   // row tiles of the longest chunk
   int total;    // virtual items: mt_max * num_seqs * hkv
+  int lo_always;  // every key tile's P.V takes P_lo as well
   float scale_log2;
 };
 
@@ -657,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // 2^-7) reaches the output scaled by that share.
         tmem_st32_nowait(scol, hw);  // P_hi over the scores' first 32 columns
         const bool with_lo =
-            !warpgroup_all(1 + hf, !row_ok || kLoSkipRatio * rs <= l);
+            !warpgroup_all(1 + hf, !p.lo_always && (!row_ok || kLoSkipRatio * rs <= l));
         if (with_lo) store_lo();
         tmem_wait_st();
         l += rs;
@@ -803,6 +804,7 @@ int launch_prefill_tcgen05(const PrefillArgs& a) {
   if (total >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
   p.total = static_cast<int>(total);
   p.scale_log2 = a.scale * kLog2e;
+  p.lo_always = a.exact_weights ? 1 : 0;
   if (p.total == 0) return PA_OK;
   static KernelLaunchCache cache;
   const int per_sm = cache.blocks_per_sm(reinterpret_cast<const void*>(prefill_tc_kernel),

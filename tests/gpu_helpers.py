@@ -99,7 +99,7 @@ class Step:
     def rows_tensor(self, rows):
         return torch().as_tensor(np.asarray(rows, np.int64), device="cuda")
 
-    def run_gpu(self, kernel=0, partition=0, want_lse=True):
+    def run_gpu(self, kernel=0, partition=0, want_lse=True, exact_weights=False):
         """copy_blocks -> reshape_and_cache -> decode (decode rows) and chunked
         prefill (prefill rows).  Returns dict of outputs keyed 'decode'/'prefill'."""
         import paged_kv_cache_454_b200 as pa
@@ -126,7 +126,7 @@ class Step:
                                              int(lay.q_lens[pf].max()), self.k_pool, self.v_pool,
                                              self.tables.index_select(0, r).contiguous(),
                                              self.lens.index_select(0, r).contiguous(), lay.scale,
-                                             want_lse=want_lse)
+                                             want_lse=want_lse, exact_weights=exact_weights)
             res["prefill"] = (out, lse)
         torch().cuda.synchronize()
         return res

@@ -465,6 +465,45 @@ def test_chunked_prefill_short_prompts(hq, hkv):
     H.compare_step(st.run_gpu(), st.run_oracle(), what=f"short prefill {hq}/{hkv}")
 
 
+@pytest.mark.parametrize("hq,hkv,short", [(10, 2, False), (32, 2, True), (4, 4, True)],
+                         ids=["g5_mixed", "g16_short", "mha_short"])
+def test_chunked_prefill_exact_weights(hq, hkv, short):
+    # With every key tile's P.V carrying the weights' bf16 remainder, each
+    # weight reaches the product to within 2^-15 of itself, so the output is
+    # the exact attention up to its own bf16 rounding (half an ulp: at most
+    # 2^-8 of the value) and fp32 accumulation.
+    if short:
+        chunks, cached = [2, 3, 5, 8, 16, 1, 4, 7], [0, 0, 0, 0, 0, 3, 2, 9]
+        lay = synth.build_layout("pf_exact", 112, [c + n for c, n in zip(cached, chunks)],
+                                 num_q_heads=hq, num_kv_heads=hkv, head_dim=128, q_lens=chunks,
+                                 is_prefill=[True] * len(chunks))
+    else:
+        lay = lay_mixed(hq, hkv, 128)
+    st = H.Step.from_host(lay)
+    ref = st.run_oracle()
+    got = st.run_gpu(exact_weights=True)
+    out = H.host_f64(got["prefill"][0])
+    want = ref["prefill"][0]
+    bound = 2.0 ** -8 * np.abs(want) * 1.001 + 1e-4
+    diff = np.abs(out - want)
+    assert np.all(diff <= bound), (
+        f"{int((diff > bound).sum())} of {diff.size} over; worst excess "
+        f"{float((diff - bound).max()):.3e}")
+    # the default (weights' remainder where a tile's share calls for it) stays
+    # inside the stated tolerance on the same inputs
+    H.compare_step(st.run_gpu(), ref, what=f"adaptive {hq}/{hkv}")
+    assert pa().pa_get_device_error() == 0
+
+
+def test_chunked_prefill_rejects_unknown_flags():
+    import ctypes
+    lib = pa().lib()
+    st = H.Step.from_host(lay_mixed(10, 2, 128))
+    assert lib.pa_chunked_prefill_ex(None, 0, None, 0, 0, None, None, pa().pool_desc(st.k_pool),
+                                     None, 1, None, 0, 10, ctypes.c_float(1.0), None, None,
+                                     ctypes.c_uint32(0x2), None) == 1  # PA_ERR_ARG
+
+
 def test_prefill_of_twelve_tokens_in_chunks_of_four_equals_one_chunk():
     # the pages' example (budget 6, 12-token prompt, 4 tokens a round), run as
     # three chunked-prefill calls against one 12-token call
