@@ -308,24 +308,18 @@ __device__ void warp_tail(const uint64_t* cand, int n, int K, float P, float u, 
   __syncwarp();
   const uint64_t tg = static_cast<uint64_t>(static_cast<double>(u) * static_cast<double>(total));
   const uint64_t tgt = tg < total ? tg : total - 1;
-  uint32_t idx[8];
-  uint64_t pre[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    idx[j] = 0xffffffffu - static_cast<uint32_t>(cand[min(8 * lane + j, n - 1)]);
-    pre[j] = 0;
-  }
-  // each kept entry's mass before it in vocabulary order
-  for (int f = 0; f < m2; ++f) {
-    const uint32_t fi = 0xffffffffu - static_cast<uint32_t>(cand[f]);
-    const uint64_t fm = mass[f];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) pre[j] += fi < idx[j] ? fm : 0ull;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int e = 8 * lane + j;
-    if (e < m2 && ms[j] > 0 && pre[j] <= tgt && pre[j] + ms[j] > tgt) *token = static_cast<int32_t>(idx[j]);
+  // each kept entry's mass before it in vocabulary order, a lane per entry
+  // (entries e0 + lane of each 32): the entry whose span holds tgt is drawn
+  for (int e0 = 0; e0 < m2; e0 += 32) {
+    const int e = e0 + lane;
+    const bool live = e < m2;
+    const uint32_t ie = live ? 0xffffffffu - static_cast<uint32_t>(cand[e]) : 0xffffffffu;
+    const uint64_t me = live ? mass[e] : 0ull;
+    uint64_t pre = 0;
+#pragma unroll 4
+    for (int f = 0; f < m2; ++f)
+      pre += (0xffffffffu - static_cast<uint32_t>(cand[f])) < ie ? mass[f] : 0ull;
+    if (live && me > 0 && pre <= tgt && pre + me > tgt) *token = static_cast<int32_t>(ie);
   }
 }
 
@@ -416,19 +410,21 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
     v[0] = x[b];
     return 1;
   };
-  // this thread's largest logit: the first element of its first largest group
-  // equal to that group's maximum
+  // The values of the two largest kept groups, loaded now so the loads are in
+  // flight while the row maximum and the Top-K bound are found (the others
+  // are loaded when needed: rarely does a thread keep more than two groups at
+  // or above the bound).
+  float pv0[4], pv1[4];
+  int pw0 = 0, pw1 = 0;
+  if (b0 != kNone) pw0 = load_group(b0, pv0);
+  if (b1 != kNone) pw1 = load_group(b1, pv1);
+  // this thread's largest key; its index (bi) is known here only when every
+  // element of the thread is -inf or NaN (or it has none)
   uint32_t bk = 0;
   int bi = kNone;
   if (b0 != kNone) {
-    float v[4];
-    const int w = load_group(b0, v);
-#pragma unroll
-    for (int j = 3; j >= 0; --j)
-      if (j < w && v[j] == g0) bi = b0 + j;
     bk = key_of(g0);
   } else {
-    // every element of this thread is -inf or NaN (or it has none)
     for_each_logit(x, V, [&](float v, int i) {
       const uint32_t k = key_of(v);
       if (k > bk || (k == bk && i < bi)) {
@@ -438,26 +434,39 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
     });
   }
   const uint32_t kown = bk;  // this thread's largest key (the reduction below overwrites bk)
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const uint32_t k2 = __shfl_xor_sync(0xffffffffu, bk, o);
-    const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
-    if (k2 > bk || (k2 == bk && i2 < bi)) {
-      bk = k2;
-      bi = i2;
-    }
+  bk = __reduce_max_sync(0xffffffffu, bk);
+  __shared__ uint32_t best;
+  __shared__ int best_i;
+  if (tid == 0) {
+    best = 0u;
+    best_i = 0x7fffffff;
   }
-  // (key, -index) packed so one 64-bit maximum finds both
-  __shared__ unsigned long long best;
-  if (tid == 0) best = 0ull;
   __syncthreads();
-  if (lane == 0)
-    atomicMax(&best, (static_cast<unsigned long long>(bk) << 32) |
-                         static_cast<unsigned long long>(0x7fffffff - bi));
+  if (lane == 0) atomicMax(&best, bk);
   __syncthreads();
-  const uint32_t kmax = static_cast<uint32_t>(best >> 32);
-  const int argmax = 0x7fffffff - static_cast<int>(best & 0xffffffffull);
+  const uint32_t kmax = best;
+  // The row's argmax, the first index of the largest key: every thread whose
+  // own largest key it is finds its first such element (in its first group of
+  // that maximum: groups come in index order) and the least index wins.  Only
+  // the paths that use it call this (every thread, at one point).
+  auto block_argmax = [&]() -> int {
+    int ci = 0x7fffffff;
+    if (kown == kmax) {
+      if (b0 != kNone) {
+#pragma unroll
+        for (int j = 3; j >= 0; --j)
+          if (j < pw0 && pv0[j] == g0) ci = b0 + j;
+      } else {
+        ci = bi;
+      }
+    }
+    ci = __reduce_min_sync(0xffffffffu, ci);
+    if (lane == 0 && ci != 0x7fffffff) atomicMin(&best_i, ci);
+    __syncthreads();
+    return best_i;
+  };
   if (!(T > 0.f) || kmax == 0u) {
+    const int argmax = block_argmax();
     if (tid == 0) tokens[row] = argmax;
     return;
   }
@@ -538,10 +547,16 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
     // too (a fifth may be) or t0 admits -inf or NaN logits, which no group
     // maximum tracks: then the row is read again.
     if ((b3 != kNone && key_of(g3) >= t0) || t0 <= key_of(-CUDART_INF_F)) sm.overflow = 1;
-    auto gather = [&](float gm, int gb) {
+    auto gather = [&](float gm, int gb, const float* pv, int pw) {
       if (gb == kNone || key_of(gm) < t0) return;
       float v[4];
-      const int w = load_group(gb, v);
+      int w = pw;
+      if (pv) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = pv[j];
+      } else {
+        w = load_group(gb, v);
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint32_t k = j < w ? key_of(v[j]) : 0u;
@@ -551,10 +566,10 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
         }
       }
     };
-    gather(g0, b0);
-    gather(g1, b1);
-    gather(g2, b2);
-    gather(g3, b3);
+    gather(g0, b0, pv0, pw0);
+    gather(g1, b1, pv1, pw1);
+    gather(g2, b2, nullptr, 0);
+    gather(g3, b3, nullptr, 0);
     __syncthreads();
     if (sm.overflow) {
       __syncthreads();
@@ -737,6 +752,8 @@ __global__ void __launch_bounds__(kThreads, 1) sample_kernel(const float* __rest
   }
 
   // ---- the draw: inverse CDF in vocabulary order over keys >= tcut ----
+  // (the argmax is the answer if rounding leaves no entry to draw)
+  const int argmax = block_argmax();
   // warp w owns the contiguous segment [w * seg, (w + 1) * seg)
   const int seg = (V + kWarps - 1) / kWarps;
   const int lo = min(V, warp * seg), hi = min(V, lo + seg);
