@@ -779,14 +779,14 @@ def main():
 # kernel was built from (reported as null once those sources change).  The
 # decode figures are captures of a smaller batch of the same shape, scaled to
 # the full batch by algorithmic bytes: gqa70b_long from 48 sequences
-# (1,760,207,872 bytes for 1,755,018,024 algorithmic), llama13b_sampling from
-# 64 sequences (558,156,288 for 542,159,500 unique).  The prefill figure is the
+# (1,759,879,168 bytes for 1,755,018,024 algorithmic), llama13b_sampling from
+# 64 sequences (558,791,168 for 542,159,500 unique).  The prefill figure is the
 # mixed step's prefill part itself (its 8 chunks, with the decode part shrunk
 # to 8 sequences: the prefill launch is the same).  The captures are
 # summarised in profiles/.
 TRAFFIC = {
-    ("gqa70b_long", "decode"): {"bytes": 4774621103, "sources": "978d8fa2d68c"},
-    ("llama13b_sampling", "decode"): {"bytes": 2172407721, "sources": "978d8fa2d68c"},
+    ("gqa70b_long", "decode"): {"bytes": 4773729483, "sources": "f7116353621e"},
+    ("llama13b_sampling", "decode"): {"bytes": 2174878746, "sources": "f7116353621e"},
     ("mixed_qwen32b", "prefill"): {"bytes": 185013760, "sources": "d5dda8f04e86"},
 }
 

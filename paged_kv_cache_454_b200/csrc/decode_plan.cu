@@ -70,6 +70,9 @@ constexpr int kLocalityShare = 16;
 static_assert(kFirstSet == 2048, "the set's hash keeps 11 bits");
 // A shared prefix shorter than this is left to each sequence's own items.
 constexpr int kMinCascSpan = 128;
+// sharers per sub-run at most (the span search compares this many tables per
+// entry; the columns of a tile, 8, already bound it)
+constexpr int kCascMaxMembers = 8;
 // Shared-prefix items per SM the prefix partition length aims for.
 constexpr int kCascItemsPerSm = 8;
 
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     }
     __syncthreads();
     // sharers per item and KV heads per item
-    members = min(rmax, casc_cols / group);
+    members = min(min(rmax, casc_cols / group), kCascMaxMembers);
     hts = 0;
     while (hts < 3 && group * (2 << hts) * members <= casc_cols && kv_heads % (2 << hts) == 0) ++hts;
     casc = members >= 2;
@@ -307,47 +310,69 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
       if (sub) sub_pos[idx - 1] = i | (k << 16);
       if (tid == 1023) nruns = idx;
       __syncthreads();
-      // a warp per sub-run: its members and the span of table entries they share
+      // a half-warp per sub-run (two per warp, so 64 sub-runs take one round
+      // of table loads): its members and the span of table entries they
+      // share.  Lane l of a half covers entries b0 + l and b0 + 16 + l of
+      // each 32-entry window.
       const int nr = nruns;
-      for (int r = warp; r < nr; r += 32) {
-        const int i0 = sub_pos[r] & 0xffff, k = sub_pos[r] >> 16;
-        int full = max_blocks;  // whole blocks inside every member's context
-        for (int q = 0; q < k; ++q) {
-          const int sq = static_cast<int>(skey[i0 + q] & 0xffffffffull);
-          full = min(full, clamp_len(lens[sq], max_blocks, nullptr) >> 4);
+      const int hl = lane & 15, hw = lane >> 4;
+      for (int r0 = 2 * warp; r0 < nr; r0 += 64) {
+        const int r = r0 + hw;
+        const bool live = r < nr;
+        int i0 = 0, k = 0;
+        int full = 0;  // whole blocks inside every member's context
+        if (live) {
+          i0 = sub_pos[r] & 0xffff;
+          k = sub_pos[r] >> 16;
+          full = max_blocks;
+          for (int q = 0; q < k; ++q) {
+            const int sq = static_cast<int>(skey[i0 + q] & 0xffffffffull);
+            full = min(full, clamp_len(lens[sq], max_blocks, nullptr) >> 4);
+          }
         }
         int lcp = full;
-        for (int b0 = 0; b0 < full; b0 += 32) {
-          const int bj = b0 + lane;
-          bool same = true;
-          if (bj < full) {
-            // every member's entry is loaded before any is compared, so the
-            // loads are in flight together
-            int32_t v[16];
+        bool open = live;  // this half has not found its first differing entry
+        for (int b0 = 0; __any_sync(0xffffffffu, open && b0 < full); b0 += 32) {
+          bool same0 = true, same1 = true;
+          if (open && b0 < full) {
+            // every member's entries are loaded before any is compared, so
+            // the loads are in flight together
+            int32_t v0[kCascMaxMembers], v1[kCascMaxMembers];
+            const int bj0 = b0 + hl, bj1 = b0 + 16 + hl;
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-              v[q] = q < k ? block_tables[static_cast<int64_t>(skey[i0 + q] & 0xffffffffull) * max_blocks + bj]
-                           : 0;
+            for (int q = 0; q < kCascMaxMembers; ++q) {
+              const int64_t rowq =
+                  q < k ? static_cast<int64_t>(skey[i0 + q] & 0xffffffffull) * max_blocks : 0;
+              v0[q] = q < k && bj0 < full ? block_tables[rowq + bj0] : 0;
+              v1[q] = q < k && bj1 < full ? block_tables[rowq + bj1] : 0;
+            }
 #pragma unroll
-            for (int q = 1; q < 16; ++q) same = same && (q >= k || v[q] == v[0]);
+            for (int q = 1; q < kCascMaxMembers; ++q) {
+              same0 = same0 && (q >= k || v0[q] == v0[0]);
+              same1 = same1 && (q >= k || v1[q] == v1[0]);
+            }
           }
-          const unsigned diff = __ballot_sync(0xffffffffu, !same);
-          if (diff) {
+          const unsigned d0 = (__ballot_sync(0xffffffffu, !same0) >> (16 * hw)) & 0xffffu;
+          const unsigned d1 = (__ballot_sync(0xffffffffu, !same1) >> (16 * hw)) & 0xffffu;
+          const unsigned diff = d0 | (d1 << 16);  // bit i: entry b0 + i differs
+          if (open && b0 < full && diff) {
             lcp = b0 + __ffs(diff) - 1;
-            break;
+            open = false;
           }
         }
-        const int span = lcp * 16 >= kMinCascSpan ? lcp * 16 : 0;
-        int* rr = runs + static_cast<int64_t>(r) * kRunInts;
-        if (lane == 0) {
-          rr[0] = span;
-          rr[1] = k;
-          rspan[r] = span;
-        }
-        if (lane < k) {
-          const int sq = static_cast<int>(skey[i0 + lane] & 0xffffffffull);
-          rr[2 + lane] = sq;
-          sspan[sq] = span;
+        if (live) {
+          const int span = lcp * 16 >= kMinCascSpan ? lcp * 16 : 0;
+          int* rr = runs + static_cast<int64_t>(r) * kRunInts;
+          if (hl == 0) {
+            rr[0] = span;
+            rr[1] = k;
+            rspan[r] = span;
+          }
+          if (hl < k) {
+            const int sq = static_cast<int>(skey[i0 + hl] & 0xffffffffull);
+            rr[2 + hl] = sq;
+            sspan[sq] = span;
+          }
         }
       }
       __syncthreads();
