@@ -180,7 +180,22 @@ def lay_casc_edges():
                              num_q_heads=8, num_kv_heads=8, min_suffix=0)
 
 
-CASCADE_LAYOUTS = ["casc_mha4", "casc_mha17", "casc_gqa8", "casc_gqa5", "casc_gqa4", "casc_edges"]
+def lay_casc_g2_many():
+    # group 2: 70 runs of two sharers -- more sub-runs than one round of the
+    # plan's span search takes (64) -- and four unshared sequences; prompts of
+    # 160 tokens (9 shared blocks after the copy-on-write)
+    return synth.prefix_runs("casc_g2_many", 127, [2] * 70 + [1] * 4, 160, 40, num_q_heads=8,
+                             num_kv_heads=4)
+
+
+def lay_casc_g3():
+    # group 3: two sharers per item; the run of 3 cut into 2 + 1
+    return synth.prefix_runs("casc_g3", 128, [2, 2, 3, 1], 400, 200, num_q_heads=12,
+                             num_kv_heads=4)
+
+
+CASCADE_LAYOUTS = ["casc_mha4", "casc_mha17", "casc_gqa8", "casc_gqa5", "casc_gqa4", "casc_edges",
+                   "casc_g2_many", "casc_g3"]
 
 
 DECODE_LAYOUTS = {
@@ -208,6 +223,8 @@ DECODE_LAYOUTS = {
     "casc_gqa5": lay_casc_gqa5,
     "casc_gqa4": lay_casc_gqa4,
     "casc_edges": lay_casc_edges,
+    "casc_g2_many": lay_casc_g2_many,
+    "casc_g3": lay_casc_g3,
 }
 
 
