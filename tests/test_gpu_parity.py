@@ -131,6 +131,18 @@ def lay_short_g12():
                               num_kv_heads=2, head_dim=128)
 
 
+def lay_gqa3():
+    # group 3 (3 of 8 columns live) over 4 KV heads: tiles of 2 heads
+    return synth.build_layout("gqa3", 130, [1, 15, 16, 17, 300, 2049], num_q_heads=12,
+                              num_kv_heads=4, head_dim=128)
+
+
+def lay_gqa7():
+    # group 7 (7 of 8 columns live) over 2 KV heads, short and long contexts
+    return synth.build_layout("gqa7", 131, [2, 9, 33, 640, 3000], num_q_heads=14,
+                              num_kv_heads=2, head_dim=128)
+
+
 def lay_g12():
     # group 12 (12 of 16 columns live) over several tiles, splits and tails
     return synth.build_layout("g12", 120, [1, 40, 300, 1100, 2600], num_q_heads=36,
@@ -217,6 +229,8 @@ DECODE_LAYOUTS = {
     "short_g16": lay_short_g16,
     "short_g12": lay_short_g12,
     "g12": lay_g12,
+    "gqa3": lay_gqa3,
+    "gqa7": lay_gqa7,
     "casc_mha4": lay_casc_mha4,
     "casc_mha17": lay_casc_mha17,
     "casc_gqa8": lay_casc_gqa8,
@@ -321,7 +335,8 @@ def test_decode_simt(name, partition):
 
 @pytest.mark.parametrize("name", ["gqa8", "gqa5", "g16", "shared_prefix", "shared_many", "mha128",
                                   "short_gqa", "short_mha", "gqa4", "gqa2_h6", "mha_h5",
-                                  "mha_h16", "gqa8_h3", "short_g16", "short_g12", "g12"]
+                                  "mha_h16", "gqa8_h3", "short_g16", "short_g12", "g12", "gqa3",
+                                  "gqa7"]
                          + CASCADE_LAYOUTS)
 @pytest.mark.parametrize("partition", [0, 128, 1024, 1 << 20])
 def test_decode_tcgen05(name, partition):
@@ -458,8 +473,9 @@ def test_decode_default_kernel_choice():
 # Chunked prefill
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("hq,hkv,d", [(10, 2, 128), (16, 2, 128), (4, 4, 128), (8, 2, 64),
-                                     (32, 2, 128), (24, 2, 128)],
-                         ids=["g5", "g8", "mha", "g4_d64", "g16", "g12"])
+                                     (32, 2, 128), (24, 2, 128), (8, 4, 128), (12, 4, 128),
+                                     (14, 2, 128)],
+                         ids=["g5", "g8", "mha", "g4_d64", "g16", "g12", "g2", "g3", "g7"])
 def test_chunked_prefill(hq, hkv, d):
     lay = lay_mixed(hq, hkv, d)
     st = H.Step.from_host(lay)
